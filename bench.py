@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the HiLS attention forward on B200 through the C-ABI library.
+
+A step is one pass of the whole hot path over one synthetic batch: the full
+prefill forward of the 128K-token GQA workload (B1, Hq32/Hkv8, d128, S64,
+k32, r32): calibration, landmark scoring, top-k selection, fusion weights,
+per-chunk attention and the fused merge.  The decode step (512K-token
+context, B1, H16, d64, k16) is timed in the same run and reported under
+"decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torch.distributed.run, one rank per GPU: every rank runs
+its own independent sequence (weak scaling, no data-path collective); the
+step time is the maximum over ranks.  ``--impl reference`` times the CPU
+oracle (plain fp64 C) on a bounded sample of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import hils_inputs as hi  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_KERNELS_PER_STEP = 6   # select, count, scan, scatter, attend, finish
+DECODE_KERNELS_PER_STEP = 2    # scan (+append, selection), attend (+merge)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: d[k] for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- work counts
+def prefill_counts(w: hi.Workload) -> dict:
+    """Algorithmic work of one prefill step (all rows of all sequences)."""
+    S, k, d, r = w.chunk_size, w.top_k, w.head_dim, w.calib_rank
+    i = np.arange(w.seq_len, dtype=np.int64)
+    c = i // S
+    n_sel = np.minimum(k, c + 1)
+    keys = (n_sel - 1) * S + (i % S + 1)
+    rows = w.batch * w.n_q_heads
+    att = float(rows * np.sum(4 * d * keys))                 # QK^T and PV, useful keys only
+    score = float(rows * np.sum(2 * d * (c + 1)))            # q~ . landmark, causal chunks
+    calib = float(rows * w.seq_len * 4 * d * r)
+    el = 2 if w.dtype == hi.DT_BF16 else 4
+    kv_bytes = w.batch * w.n_kv_heads * 2 * w.seq_len * d * el
+    q_bytes = rows * w.seq_len * d * el
+    lm_bytes = w.batch * w.n_kv_heads * ((w.seq_len + S - 1) // S) * d * el
+    return {"attention_flop": att, "score_flop": score, "calib_flop": calib,
+            "min_bytes": float(kv_bytes + 2 * q_bytes + lm_bytes), "pairs": float(rows * n_sel.sum())}
+
+
+def decode_bytes(w: hi.Workload, step: int) -> dict:
+    """Algorithmic HBM bytes of decode step ``step``: every visible landmark of
+    each KV head, the selected chunks' K and V per query head, q, out, and the
+    appended k/v."""
+    S, k, d = w.chunk_size, w.top_k, w.head_dim
+    t = w.seq_len + step
+    c = t // S
+    el = 2 if w.dtype == hi.DT_BF16 else 4
+    lm = w.batch * (c + 1) * w.n_kv_heads * d * el
+    n_sel = min(k, c + 1)
+    keys = (n_sel - 1) * S + (t % S + 1)
+    kv = w.batch * w.n_q_heads * keys * d * 2 * el
+    small = w.batch * (2 * w.n_q_heads + 2 * w.n_kv_heads) * d * el
+    return {"landmark_bytes": lm, "kv_bytes": kv, "total": lm + kv + small}
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.lines = []
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        sel = ["-i", vis[self.dev].strip()] if len(vis) > self.dev and vis[self.dev].strip() else \
+            ["-i", str(self.dev)]
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm
+def make_cache(hils, wl):
+    w = wl["workload"]
+    return hils.Cache(wl["pages"], wl["num_pages"], wl["block_table"], wl["max_chunks"],
+                      wl["landmarks"], wl.get("seq_lens"))
+
+
+def cfg_of(hils, w):
+    return hils.HilsConfig(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk_size, w.top_k,
+                           w.calib_rank, w.dtype)
+
+
+def time_prefill(hils, torch, wl, steps, warmup, barrier, maxreduce):
+    w = wl["workload"]
+    cfg = cfg_of(hils, w)
+    cache = make_cache(hils, wl)
+    L = w.seq_len
+    dt = torch.bfloat16 if w.dtype == hi.DT_BF16 else torch.float32
+    out = torch.empty((w.batch, L, w.n_q_heads, w.head_dim), dtype=dt, device="cuda")
+    nbytes = hils.workspace_size(cfg, hils.OP_PREFILL, L, wl["max_chunks"])
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hils.prefill(cfg, wl["q"], L, 0, wl["A"], wl["B"], cache, out, None, None, ws, nbytes,
+                     stream)
+
+    for _ in range(warmup):
+        step()
+    hils.device_status(stream)
+    hils.profile_reset()
+    hils.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    hils.profile_enable(False)
+    phases = hils.profile_read()
+    hils.device_status(stream)
+    ms = maxreduce(e0.elapsed_time(e1)) / steps
+    return ms, phases, clk.summary(), (out, ws, nbytes)
+
+
+def time_prefill_e2e(hils, torch, wl, steps, warmup):
+    """Same step through host buffers: pinned host inputs copied in, the result
+    copied out, every step, inside the timed region."""
+    w = wl["workload"]
+    cfg = cfg_of(hils, w)
+    stream = torch.cuda.current_stream()
+    host = {k: wl[k].cpu().pin_memory() for k in ("q", "pages", "landmarks", "block_table", "A", "B")}
+    dev = {k: torch.empty_like(wl[k]) for k in host}
+    L = w.seq_len
+    out = torch.empty_like(wl["q"])
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    nbytes = hils.workspace_size(cfg, hils.OP_PREFILL, L, wl["max_chunks"])
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    cache = hils.Cache(dev["pages"], wl["num_pages"], dev["block_table"], wl["max_chunks"],
+                       dev["landmarks"])
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out.numel() * out.element_size()
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        hils.prefill(cfg, dev["q"], L, 0, dev["A"], dev["B"], cache, out, None, None, ws, nbytes,
+                     stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def time_decode(hils, torch, wl, warmup_steps=8):
+    """All decode steps of the workload, one after another (each appends its
+    token); L2 is flushed before every step and only the step itself is timed."""
+    w = wl["workload"]
+    cfg = cfg_of(hils, w)
+    cache = make_cache(hils, wl)
+    dt = torch.bfloat16 if w.dtype == hi.DT_BF16 else torch.float32
+    nbytes = hils.workspace_size(cfg, hils.OP_DECODE, 1, wl["max_chunks"])
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=dt, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    seq0 = wl["seq_lens"].clone()
+
+    def run(n, timed):
+        wl["seq_lens"].copy_(seq0)
+        evs = []
+        for s in range(n):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            hils.decode(cfg, wl["q_dec"][s], wl["k_new"][s], wl["v_new"][s], wl["A"], wl["B"], cache,
+                        out, None, None, ws, nbytes, stream)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    run(warmup_steps, False)
+    hils.profile_reset()
+    hils.profile_enable(True)
+    times = run(w.decode_steps, True)
+    hils.profile_enable(False)
+    phases = hils.profile_read()
+    hils.device_status(stream)
+    wl["seq_lens"].copy_(seq0)
+    return times, phases
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+def oracle_prefill_sample(wl, budget_s: float, rng_seed: int = 0):
+    """Time the CPU oracle on a sample of the prefill workload's rows for about
+    ``budget_s`` seconds.  Returns (rows_done, seconds, threads, sample text)."""
+    from oracle import oracle
+    w = wl["workload"]
+    threads = oracle.set_threads(0)
+    pages = wl["pages"].cpu()
+    to_np = (lambda t: t.view(__import__("torch").int16).numpy().view(np.uint16)) \
+        if w.dtype == hi.DT_BF16 else (lambda t: t.numpy())
+    pages_np = to_np(pages)
+    lm_np = to_np(wl["landmarks"].cpu())
+    bt = wl["block_table"].cpu().numpy()
+    A, B = wl["A"].cpu().numpy(), wl["B"].cpu().numpy()
+    oc = oracle.cfg(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk_size, w.top_k,
+                    w.calib_rank, w.dtype)
+    rng = np.random.default_rng(rng_seed)
+    q = wl["q"]
+    done, t0, batches = 0, time.perf_counter(), 0
+    batch = max(threads * 4, 16)
+    while True:
+        pos = rng.integers(0, w.seq_len, size=batch)
+        hh = rng.integers(0, w.n_q_heads, size=batch)
+        bb = rng.integers(0, w.batch, size=batch)
+        import torch
+        ix = torch.from_numpy(np.stack([bb, pos, hh], 1)).to(q.device)
+        rows = to_np(q[ix[:, 0], ix[:, 1], ix[:, 2]].cpu())
+        oracle.hils_rows(oc, rows, bb, hh, pos, A, B, pages_np, bt, lm_np)
+        done += batch
+        batches += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    sample = (f"{done} query rows (random positions and heads, uniform over the "
+              f"{w.seq_len}-token sequence) in {batches} batches; tok/s = rows/s / Hq")
+    return done, el, threads, sample
+
+
+# ----------------------------------------------------------------- main
+def dist_setup(torch):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+
+        def barrier():
+            dist.barrier()
+
+        def maxreduce(x):
+            t = torch.tensor([x], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+        return ws, rank, barrier, maxreduce
+    torch.cuda.set_device(local)
+    return 1, 0, (lambda: None), (lambda x: x)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_128k_gqa")
+    ap.add_argument("--decode-workload", default="decode_512k")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    nworld, rank, barrier, maxreduce = dist_setup(torch)
+    w = hi.WORKLOADS[args.workload]
+    counts = prefill_counts(w)
+    tokens_per_rank = w.batch * w.seq_len
+    metric = "HiLS prefill tok/s @128K; decode us/step @512K; % of HBM/TC roofline"
+    config = {"workload": w.name, "global_batch": w.batch * nworld, "seq_len": w.seq_len,
+              "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+              "chunk_size": w.chunk_size, "top_k": w.top_k, "calib_rank": w.calib_rank,
+              "parallelism": f"replicas{nworld} (independent sequences)",
+              "l2": "inputs larger than L2 (q 1.07 GB, K/V 0.54 GB per step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        wl = hi.device_workload(w)
+        budget = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup) * 2)
+        per = []
+        for s in range(args.warmup + args.steps):
+            n, el, threads, sample = oracle_prefill_sample(wl, budget, rng_seed=s)
+            if s >= args.warmup:
+                per.append(n / el / w.n_q_heads)
+        v = statistics.median(per)
+        print(json.dumps({
+            "impl": "reference", "metric": metric, "value": v, "unit": "tok/s", "n_gpus": nworld,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.seq_len / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic N(0,1), seeded", "config": config,
+            "cpu_baseline": {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                             "sample": f"per step: {sample} (~{budget:.0f} s of oracle work)"},
+            "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    from chunk_sparse_long_b200 import build, hils
+    if rank == 0:
+        build.build()
+    barrier()
+    hils.load()
+    wl = hi.device_workload(w, seed_offset=rank)
+    torch.cuda.synchronize()
+    ms, phases, clocks, _keep = time_prefill(hils, torch, wl, args.steps, args.warmup, barrier,
+                                             maxreduce)
+    value = tokens_per_rank * nworld / (ms / 1e3)
+    pk, pk_src = peaks()
+    # dominant kernel of the prefill step
+    dom = max(phases.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms_total, dom_launches) = dom
+    dom_ms = dom_ms_total / max(1, dom_launches)
+    if dom_name == "prefill.attend":
+        work, what = counts["attention_flop"], "useful attention flop (QK^T + PV over selected keys)"
+    elif dom_name == "prefill.select":
+        work, what = counts["score_flop"] + counts["calib_flop"], "landmark scoring + calibration flop"
+    else:
+        work, what = counts["attention_flop"], "useful attention flop"
+    achieved = work / (dom_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
+                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                "work_per_launch": work, "work": what,
+                "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)"}
+    result = {
+        "metric": metric, "value": value, "unit": "tok/s", "n_gpus": nworld, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1), seeded", "config": config,
+        "clocks": clocks, "roofline": roofline,
+        "gpu_launches": PREFILL_KERNELS_PER_STEP * args.steps,
+        "kernels_ms_per_step": {k: v[0] / max(1, args.steps) for k, v in phases.items()},
+        "useful_attention_tflops": counts["attention_flop"] / (ms / 1e3) / 1e12,
+    }
+    del _keep
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_prefill_e2e(hils, torch, wl, max(1, min(args.steps, 3)), 1)
+        e2e_ms = maxreduce(e2e_ms)
+        result["e2e"] = {"value": tokens_per_rank * nworld / (e2e_ms / 1e3), "unit": "tok/s",
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del wl
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        dw = hi.WORKLOADS[args.decode_workload]
+        dwl = hi.device_workload(dw, seed_offset=rank)
+        times, dph = time_decode(hils, torch, dwl)
+        us = maxreduce(statistics.mean(times)) * 1e3
+        by = [decode_bytes(dw, s) for s in range(dw.decode_steps)]
+        tot = statistics.mean(b["total"] for b in by)
+        kvb = statistics.mean(b["kv_bytes"] for b in by)
+        lmb = statistics.mean(b["landmark_bytes"] for b in by)
+        dom_d = max(dph.items(), key=lambda kv: kv[1][0])
+        dn, (dms, dl) = dom_d
+        dms_per = dms / max(1, dl)
+        dbytes = lmb if dn == "decode.scan" else kvb
+        result["decode"] = {
+            "workload": dw.name, "us_per_step": us, "steps": dw.decode_steps,
+            "context": dw.seq_len, "bytes_per_step": tot, "landmark_bytes": lmb, "kv_bytes": kvb,
+            "step_gbs": tot / (us / 1e6) / 1e9,
+            "step_hbm_frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"],
+            "kernels_us_per_step": {k: v[0] / max(1, v[1]) * 1e3 for k, v in dph.items()},
+            "roofline": {"bound": "hbm", "kernel": dn, "achieved": dbytes / (dms_per / 1e3) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": dbytes / (dms_per / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk_src} HBM copy bandwidth"},
+            "l2": "flushed (256 MB write) before every step; only the step is timed",
+            "gpu_launches": DECODE_KERNELS_PER_STEP * dw.decode_steps,
+        }
+        del dwl
+    if rank == 0 and nworld == 1 and not args.no_cpu_baseline:
+        wl = hi.device_workload(w)
+        n, el, threads, sample = oracle_prefill_sample(wl, args.cpu_budget)
+        result["cpu_baseline"] = {"value": n / el / w.n_q_heads, "unit": "tok/s", "cores": threads,
+                                  "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(result))
+    if nworld > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

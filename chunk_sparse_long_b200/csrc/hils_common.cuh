@@ -1,0 +1,149 @@
+// Internal declarations shared by the HiLS CUDA kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/hils.h"
+
+namespace hils {
+
+constexpr int kChunk = 64;       // chunk_size the kernels are written for
+constexpr int kMaxTopK = 32;
+constexpr int kMaxRank = 64;
+
+// Device error word: kernels OR bits into it when a bounds check fires.
+enum DeviceError : int {
+  kErrPage = 1,      // block_table entry outside [0, num_pages)
+  kErrChunk = 2,     // selected chunk index outside [0, max_chunks)
+  kErrTimeout = 4,   // a bounded wait ran out
+};
+extern __device__ int g_device_error;
+
+__device__ __forceinline__ void set_device_error(int bit) { atomicOr(&g_device_error, bit); }
+
+// Plain parameters of one call, passed by value to every kernel.
+struct Params {
+  int B, Hq, Hkv, d, k, r, dtype;
+  int group;              // Hq / Hkv
+  float inv_sqrt_d;
+  const void* q;          // prefill [B][L][Hq][d]; decode [B][Hq][d]
+  int64_t L, pos0;
+  const float* A;         // [d][r]
+  const float* Bm;        // [r][d]
+  const void* pages;
+  int64_t num_pages;
+  const int32_t* block_table;
+  int max_chunks;
+  const void* landmarks;
+  int32_t* seq_lens;
+};
+
+// ---- storage loads ------------------------------------------------------
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+__device__ __forceinline__ float load_elem(const void* p, int dtype, int64_t i) {
+  if (dtype == HILS_F32) return ((const float*)p)[i];
+  return bf16_to_f32(((const uint16_t*)p)[i]);
+}
+
+// Eight consecutive elements starting at element i (i a multiple of 8, 16-byte aligned).
+__device__ __forceinline__ void load8(const void* p, int dtype, int64_t i, float* v) {
+  if (dtype == HILS_F32) {
+    const float4* f = reinterpret_cast<const float4*>((const float*)p + i);
+    float4 a = f[0], b = f[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 u = *reinterpret_cast<const uint4*>((const uint16_t*)p + i);
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      v[2 * a] = __uint_as_float(w[a] << 16);
+      v[2 * a + 1] = __uint_as_float(w[a] & 0xFFFF0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_elem(void* p, int dtype, int64_t i, float v) {
+  if (dtype == HILS_F32)
+    ((float*)p)[i] = v;
+  else
+    ((__nv_bfloat16*)p)[i] = __float2bfloat16_rn(v);
+}
+
+// Element offset of (page, kind, kv head g, slot s, element 0) in the page pool.
+__device__ __forceinline__ int64_t page_offset(const Params& P, int64_t page, int kind, int g,
+                                               int s) {
+  return (((page * 2 + kind) * P.Hkv + g) * (int64_t)kChunk + s) * P.d;
+}
+
+// Physical page of logical chunk j of sequence b, or -1 (and the error bit) if
+// the block table points outside the pool.
+__device__ __forceinline__ int64_t page_of(const Params& P, int b, int64_t j) {
+  if (j < 0 || j >= P.max_chunks) {
+    set_device_error(kErrChunk);
+    return -1;
+  }
+  int64_t page = P.block_table[(int64_t)b * P.max_chunks + j];
+  if (page < 0 || page >= P.num_pages) {
+    set_device_error(kErrPage);
+    return -1;
+  }
+  return page;
+}
+
+// RAII bracket of one kernel launch for the optional event profiler
+// (hils_profile_enable); a no-op unless profiling is on.
+class ProfileScope {
+ public:
+  ProfileScope(const char* phase, cudaStream_t s);
+  ~ProfileScope();
+
+ private:
+  const char* phase_;
+  cudaStream_t stream_;
+  void* start_ = nullptr;
+};
+#define HILS_PROFILE(name, stream) ::hils::ProfileScope _hils_prof_scope_(name, stream)
+
+// ---- launchers (each returns cudaError_t of its launches) -----------------
+cudaError_t launch_score(const Params& P, float* scores, int n_cols, cudaStream_t s);
+cudaError_t launch_topk(const Params& P, const float* scores, int n_cols, int32_t* idx, float* w,
+                        cudaStream_t s);
+
+struct PrefillWs {
+  int32_t* idx;      // [rows][k]
+  float* w;          // [rows][k]
+  int32_t* counts;   // [n_keys]
+  int32_t* offsets;  // [n_keys + 1] pair offsets
+  int32_t* tile_off; // [n_keys + 1] tile offsets
+  int32_t* cursor;   // [n_keys]
+  int32_t* pairs;    // [rows * k] pair ids (row * k + slot)
+  float* acc;        // [rows][d]
+  int n_keys;
+  int64_t max_tiles;
+};
+size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base);
+cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
+                           const PrefillWs& ws, cudaStream_t s);
+
+struct DecodeWs {
+  float* cand_s;       // [B][n_split][Hq][k-1]
+  int32_t* cand_j;     // same
+  int32_t* idx;        // [B][Hq][k]
+  float* w;            // [B][Hq][k]
+  float* part;         // [B][Hq][k][d]
+  int32_t* tickets;    // [B][Hq] scan tickets, [B][Hq] attention tickets, [B] head-done
+  int32_t* tpos;       // [B] position of this step's query
+  int n_split, chunks_per_split;
+};
+size_t decode_ws_bytes(const Params& P, DecodeWs* ws, char* base);
+cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,
+                          int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s);
+
+}  // namespace hils

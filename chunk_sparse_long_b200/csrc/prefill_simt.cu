@@ -1,0 +1,388 @@
+// Prefill forward on CUDA cores: a1..a7 without materialising scores.
+//
+//   select   one thread per query row: q~ in registers, landmark tiles of the
+//            row's KV head staged in shared memory, a running sorted list of
+//            the k-1 best candidates (strict '>' while chunks are visited in
+//            ascending order keeps the lower index on ties), then the fusion
+//            softmax over own + selected.
+//   bucket   counting sort of the (row, slot) pairs by (sequence, KV head,
+//            chunk), so that every chunk's K/V tile is read once per tile of
+//            up to kTilePairs rows that selected it (key-major grouping).
+//   attend   per tile: K/V of the chunk in shared memory, one warp per pair:
+//            scores, masked softmax (own chunk causal), P.V, and the
+//            w/l-scaled result added into a float32 accumulator row.
+//   finish   accumulator -> output dtype.
+#include <cfloat>
+
+#include "hils_common.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kSelThreads = 128;
+constexpr int kLmTile = 32;
+constexpr int kTilePairs = 128;
+constexpr int kAttThreads = 256;
+constexpr int kAttWarps = kAttThreads / 32;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(Params P, int32_t* idx, float* w) {
+  extern __shared__ float smem[];
+  const int t = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / P.group;
+  const int64_t i = (int64_t)blockIdx.x * kSelThreads + t;
+  const bool valid = i < P.L;
+  const int64_t pos = P.pos0 + (valid ? i : P.L - 1);
+  const int64_t own = pos / kChunk;
+  const int64_t r = ((int64_t)b * P.L + i) * P.Hq + h;
+  const int64_t i_last = min((int64_t)(blockIdx.x + 1) * kSelThreads, P.L) - 1;
+  const int64_t own_max = (P.pos0 + i_last) / kChunk;
+
+  float qt[D];
+#pragma unroll
+  for (int e = 0; e < D; e += 8) {
+    if (valid) {
+      load8(P.q, P.dtype, r * D + e, &qt[e]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) qt[e + u] = 0.f;
+    }
+  }
+
+  // a1: calibration, with A and B staged in shared memory (phase 1 layout)
+  if (P.r > 0) {
+    float* sA = smem;
+    float* sB = sA + D * P.r;
+    float* sT = sB + P.r * D;
+    for (int x = t; x < D * P.r; x += kSelThreads) {
+      sA[x] = P.A[x];
+      sB[x] = P.Bm[x];
+    }
+    __syncthreads();
+    for (int a = 0; a < P.r; ++a) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < D; ++e) acc = fmaf(qt[e], sA[e * P.r + a], acc);
+      sT[a * kSelThreads + t] = acc;
+    }
+    for (int a = 0; a < P.r; ++a) {
+      const float ta = sT[a * kSelThreads + t];
+#pragma unroll
+      for (int e = 0; e < D; ++e) qt[e] = fmaf(ta, sB[a * D + e], qt[e]);
+    }
+    __syncthreads();
+  }
+
+  // a2 + a3: stream the landmarks, keep the best k-1 candidates (phase 2 layout)
+  const int K = P.k - 1;
+  float* sLm = smem;
+  float* lsS = sLm + kLmTile * D;
+  int* lsJ = reinterpret_cast<int*>(lsS + kMaxTopK * kSelThreads);
+  int n = 0;
+  float thr = -INFINITY;
+  float s_own = 0.f;
+  for (int64_t j0 = 0; j0 <= own_max; j0 += kLmTile) {
+    __syncthreads();
+    for (int x = t; x < kLmTile * (D / 8); x += kSelThreads) {
+      const int jj = x / (D / 8), e8 = (x % (D / 8)) * 8;
+      const int64_t j = j0 + jj;
+      if (j <= own_max) {
+        load8(P.landmarks, P.dtype, (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * D + e8,
+              &sLm[jj * D + e8]);
+      }
+    }
+    __syncthreads();
+    for (int jj = 0; jj < kLmTile; ++jj) {
+      const int64_t j = j0 + jj;
+      if (j > own) break;
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < D; ++e) acc = fmaf(qt[e], sLm[jj * D + e], acc);
+      const float s = acc * P.inv_sqrt_d;
+      if (j == own) {
+        s_own = s;
+      } else if (K > 0 && (n < K || s > thr)) {
+        int p = n < K ? n : K - 1;
+        while (p > 0 && s > lsS[(p - 1) * kSelThreads + t]) {
+          lsS[p * kSelThreads + t] = lsS[(p - 1) * kSelThreads + t];
+          lsJ[p * kSelThreads + t] = lsJ[(p - 1) * kSelThreads + t];
+          --p;
+        }
+        lsS[p * kSelThreads + t] = s;
+        lsJ[p * kSelThreads + t] = (int)j;
+        if (n < K) ++n;
+        if (n == K) thr = lsS[(K - 1) * kSelThreads + t];
+      }
+    }
+  }
+  if (!valid) return;
+
+  // a4: fusion weights
+  float m = s_own;
+  for (int a = 0; a < n; ++a) m = fmaxf(m, lsS[a * kSelThreads + t]);
+  float z = __expf(s_own - m);
+  for (int a = 0; a < n; ++a) z += __expf(lsS[a * kSelThreads + t] - m);
+  const float iz = 1.f / z;
+  int32_t* ix = idx + r * P.k;
+  float* wr = w + r * P.k;
+  ix[0] = (int32_t)own;
+  wr[0] = __expf(s_own - m) * iz;
+  for (int a = 0; a < n; ++a) {
+    ix[1 + a] = lsJ[a * kSelThreads + t];
+    wr[1 + a] = __expf(lsS[a * kSelThreads + t] - m) * iz;
+  }
+  for (int a = n + 1; a < P.k; ++a) {
+    ix[a] = -1;
+    wr[a] = 0.f;
+  }
+}
+
+// ---- bucketing ------------------------------------------------------------
+__device__ __forceinline__ int64_t pair_key(const Params& P, int64_t r, int32_t j) {
+  const int h = (int)(r % P.Hq);
+  const int b = (int)(r / ((int64_t)P.L * P.Hq));
+  return ((int64_t)b * P.Hkv + h / P.group) * P.max_chunks + j;
+}
+
+__global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int64_t n_pairs) {
+  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n_pairs) return;
+  const int32_t j = idx[p];
+  if (j < 0) return;
+  if (j >= P.max_chunks) {
+    set_device_error(kErrChunk);
+    return;
+  }
+  atomicAdd(&counts[pair_key(P, p / P.k, j)], 1);
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n_keys,
+                                                    int32_t* offsets, int32_t* tile_off,
+                                                    int32_t* cursor) {
+  __shared__ int32_t sp[1024], stl[1024];
+  const int t = threadIdx.x;
+  const int per = (n_keys + 1023) / 1024;
+  const int k0 = min(t * per, n_keys), k1 = min(k0 + per, n_keys);
+  int32_t ps = 0, ts = 0;
+  for (int key = k0; key < k1; ++key) {
+    ps += counts[key];
+    ts += (counts[key] + kTilePairs - 1) / kTilePairs;
+  }
+  sp[t] = ps;
+  stl[t] = ts;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    int32_t a = t >= o ? sp[t - o] : 0, c = t >= o ? stl[t - o] : 0;
+    __syncthreads();
+    sp[t] += a;
+    stl[t] += c;
+    __syncthreads();
+  }
+  int32_t po = sp[t] - ps, to = stl[t] - ts;
+  for (int key = k0; key < k1; ++key) {
+    offsets[key] = po;
+    cursor[key] = po;
+    tile_off[key] = to;
+    po += counts[key];
+    to += (counts[key] + kTilePairs - 1) / kTilePairs;
+  }
+  if (t == 1023) {
+    offsets[n_keys] = sp[1023];
+    tile_off[n_keys] = stl[1023];
+  }
+}
+
+__global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, int32_t* pairs,
+                               int64_t n_pairs) {
+  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n_pairs) return;
+  const int32_t j = idx[p];
+  if (j < 0 || j >= P.max_chunks) return;
+  const int32_t at = atomicAdd(&cursor[pair_key(P, p / P.k, j)], 1);
+  pairs[at] = (int32_t)p;
+}
+
+// ---- attention over key-major tiles ------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kAttThreads) attend_kernel(Params P, PrefillWs ws) {
+  extern __shared__ float sm[];
+  constexpr int LD = D + 1;  // padded row stride: conflict-free column reads
+  float* sK = sm;
+  float* sV = sK + kChunk * LD;
+  float* sQ = sV + kChunk * LD;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x;
+  if (tile >= ws.tile_off[ws.n_keys]) return;
+  int lo = 0, hi = ws.n_keys - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ws.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int key = lo;
+  const int j = key % P.max_chunks;
+  const int bg = key / P.max_chunks;
+  const int g = bg % P.Hkv, b = bg / P.Hkv;
+  const int64_t page = page_of(P, b, j);
+  if (page < 0) return;
+  for (int x = tid; x < kChunk * (D / 8); x += kAttThreads) {
+    const int s = x / (D / 8), e8 = (x % (D / 8)) * 8;
+    float v[8];
+    load8(P.pages, P.dtype, page_offset(P, page, 0, g, s) + e8, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sK[s * LD + e8 + u] = v[u];
+    load8(P.pages, P.dtype, page_offset(P, page, 1, g, s) + e8, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sV[s * LD + e8 + u] = v[u];
+  }
+  __syncthreads();
+  const int p0 = ws.offsets[key] + (tile - ws.tile_off[key]) * kTilePairs;
+  const int p1 = min(p0 + kTilePairs, ws.offsets[key + 1]);
+  float* q = sQ + warp * D;
+  for (int p = p0 + warp; p < p1; p += kAttWarps) {
+    const int32_t pid = ws.pairs[p];
+    const int64_t r = pid / P.k;
+    const int64_t i = (r / P.Hq) % P.L;
+    const int64_t pos = P.pos0 + i;
+    const int nk = (pos / kChunk == j) ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
+    if (lane < D / 8) load8(P.q, P.dtype, r * D + lane * 8, &q[lane * 8]);
+    __syncwarp();
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) {
+      s0 = fmaf(q[e], sK[lane * LD + e], s0);
+      s1 = fmaf(q[e], sK[(lane + 32) * LD + e], s1);
+    }
+    s0 = lane < nk ? s0 * P.inv_sqrt_d : -INFINITY;
+    s1 = lane + 32 < nk ? s1 * P.inv_sqrt_d : -INFINITY;
+    const float m = warp_max(fmaxf(s0, s1));
+    const float e0 = __expf(s0 - m), e1 = __expf(s1 - m);
+    const float l = warp_sum(e0 + e1);
+    float o[D / 32];
+#pragma unroll
+    for (int a = 0; a < D / 32; ++a) o[a] = 0.f;
+    for (int kk = 0; kk < kChunk; ++kk) {
+      const float pk = __shfl_sync(0xffffffffu, kk < 32 ? e0 : e1, kk & 31);
+#pragma unroll
+      for (int a = 0; a < D / 32; ++a) o[a] = fmaf(pk, sV[kk * LD + lane + 32 * a], o[a]);
+    }
+    const float scale = ws.w[pid] / l;
+    float* acc = ws.acc + r * D;
+#pragma unroll
+    for (int a = 0; a < D / 32; ++a) atomicAdd(&acc[lane + 32 * a], o[a] * scale);
+    __syncwarp();
+  }
+}
+
+__global__ void finish_kernel(Params P, const float* acc, void* out, int64_t n) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < n) store_elem(out, P.dtype, x, acc[x]);
+}
+
+template <int D>
+size_t select_smem(int r) {
+  const size_t ph1 = (size_t)(2 * D * r + r * kSelThreads) * sizeof(float);
+  const size_t ph2 = (size_t)(kLmTile * D + 2 * kMaxTopK * kSelThreads) * sizeof(float);
+  return ph1 > ph2 ? ph1 : ph2;
+}
+
+template <int D>
+constexpr size_t attend_smem() {
+  return (size_t)(2 * kChunk * (D + 1) + kAttWarps * D) * sizeof(float);
+}
+
+template <int D>
+cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStream_t s) {
+  const int64_t rows = (int64_t)P.B * P.L * P.Hq;
+  const int64_t n_pairs = rows * P.k;
+  cudaError_t e;
+  // a1..a4
+  const size_t ssm = select_smem<D>(P.r);
+  e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+  if (e != cudaSuccess) return e;
+  dim3 sg((unsigned)((P.L + kSelThreads - 1) / kSelThreads), P.Hq, P.B);
+  {
+    HILS_PROFILE("prefill.select", s);
+    select_kernel<D><<<sg, kSelThreads, ssm, s>>>(P, ws.idx, ws.w);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // bucket by (sequence, KV head, chunk)
+  if ((e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ws.n_keys, s)) != cudaSuccess) return e;
+  const unsigned pb = (unsigned)((n_pairs + 255) / 256);
+  {
+    HILS_PROFILE("prefill.bucket", s);
+    count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs);
+    scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, ws.offsets, ws.tile_off, ws.cursor);
+    scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, n_pairs);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // a5 + a6
+  if ((e = cudaMemsetAsync(ws.acc, 0, sizeof(float) * rows * D, s)) != cudaSuccess) return e;
+  constexpr size_t asm_ = attend_smem<D>();
+  e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)asm_);
+  if (e != cudaSuccess) return e;
+  {
+    HILS_PROFILE("prefill.attend", s);
+    attend_kernel<D><<<(unsigned)ws.max_tiles, kAttThreads, asm_, s>>>(P, ws);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t n = rows * D;
+  {
+    HILS_PROFILE("prefill.finish", s);
+    finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(P, ws.acc, out, n);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace carve-up; with base == nullptr only the size is computed.
+size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
+  const int64_t rows = (int64_t)P.B * P.L * P.Hq;
+  const int64_t n_pairs = rows * P.k;
+  const int64_t n_keys = (int64_t)P.B * P.Hkv * P.max_chunks;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  PrefillWs w{};
+  w.idx = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  w.w = (float*)take(sizeof(float) * n_pairs);
+  w.counts = (int32_t*)take(sizeof(int32_t) * n_keys);
+  w.offsets = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
+  w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  w.acc = (float*)take(sizeof(float) * rows * P.d);
+  w.n_keys = (int)n_keys;
+  w.max_tiles = (n_pairs + kTilePairs - 1) / kTilePairs + n_keys;
+  if (ws) *ws = w;
+  return off;
+}
+
+cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
+                           const PrefillWs& ws_in, cudaStream_t s) {
+  PrefillWs ws = ws_in;
+  if (idx_out) ws.idx = idx_out;
+  if (w_out) ws.w = w_out;
+  if (P.L == 0 || P.B == 0) return cudaSuccess;
+  return P.d == 64 ? run_prefill<64>(P, out, ws, s) : run_prefill<128>(P, out, ws, s);
+}
+
+}  // namespace hils

@@ -220,3 +220,86 @@ def needle_chunks(seed: int, count: int, n_chunks: int) -> np.ndarray:
             out.append(c)
         j += 1
     return np.array(sorted(out), dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads on the device
+# ----------------------------------------------------------------------------
+SPARE_PAGES = 4
+
+
+def device_workload(w: Workload, device="cuda", seed_offset: int = 0) -> dict:
+    """Allocate and fill every input tensor of workload ``w`` on ``device``.
+
+    Recipe (all N(0,1) unless stated; A and B are N(0, 0.02) float32):
+      pages       [P][2][Hkv][S][d], P = B*max_chunks + 4 spare pages, drawn by
+                  physical element index from stream TID_PAGES;
+      block_table sequence b's chunk j -> page perm[b*max_chunks + j], perm a
+                  seeded permutation of the page ids (TID_PERM);
+      landmarks   [B][max_chunks][Hkv][d] (TID_LM);
+      prefill:    q [B][L][Hq][d] (TID_Q);
+      decode:     q_dec [steps][B][Hq][d] (TID_QDEC), k_new and v_new
+                  [steps][B][Hkv][d] (TID_KNEW, TID_VNEW), seq_lens = context.
+    Needles: a prefill workload with ``needles`` plants, per KV head g, one
+    chunk (seeded) whose landmark is sqrt(d) m_g/|m_g|, m_g the mean of the
+    raw queries of g's query heads over all positions; a decode workload plants
+    ``needles`` chunks (seeded depths, shared by the heads) whose landmark for
+    KV head g is 4 q0/|q0|, q0 the raw step-0 query of g's first query head,
+    so its score is about +4 standard deviations above the N(0,1) background.
+    """
+    import torch
+    seed = w.seed + seed_offset
+    B, Hq, Hkv, d, S = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk_size
+    dt = torch.bfloat16 if w.dtype == DT_BF16 else torch.float32
+    max_chunks = w.n_chunks
+    n_pages = B * max_chunks + SPARE_PAGES
+    out = {"workload": w, "max_chunks": max_chunks, "num_pages": n_pages}
+    pages = torch.empty((n_pages, 2, Hkv, S, d), dtype=dt, device=device)
+    normal_device(pages, seed, TID_PAGES)
+    perm = page_permutation(seed, n_pages)
+    out["pages"] = pages
+    out["block_table"] = torch.from_numpy(
+        np.ascontiguousarray(perm[: B * max_chunks].reshape(B, max_chunks))).to(device)
+    lm = torch.empty((B, max_chunks, Hkv, d), dtype=dt, device=device)
+    normal_device(lm, seed, TID_LM)
+    out["A"] = torch.from_numpy(normal(seed, TID_A, 0, d * w.calib_rank, 0.02, DT_F32)
+                                .reshape(d, w.calib_rank)).to(device)
+    out["B"] = torch.from_numpy(normal(seed, TID_B, 0, w.calib_rank * d, 0.02, DT_F32)
+                                .reshape(w.calib_rank, d)).to(device)
+    group = Hq // Hkv
+    if w.mode == "prefill":
+        q = torch.empty((B, w.seq_len, Hq, d), dtype=dt, device=device)
+        normal_device(q, seed, TID_Q)
+        out["q"] = q
+        if w.needles:
+            n_vis = (w.seq_len + S - 1) // S
+            chunks = needle_chunks(seed, Hkv * w.needles, n_vis)
+            m = q.view(B, w.seq_len, Hkv, group, d).sum(dim=(1, 3), dtype=torch.float64)
+            for b in range(B):
+                for g in range(Hkv):
+                    for n in range(w.needles):
+                        c = int(chunks[g * w.needles + n])
+                        v = math.sqrt(d) * m[b, g] / torch.linalg.vector_norm(m[b, g])
+                        lm[b, c, g] = v.float().to(dt)
+            out["needle_chunks"] = chunks.reshape(Hkv, w.needles)
+    else:
+        steps = w.decode_steps
+        qd = torch.empty((steps, B, Hq, d), dtype=dt, device=device)
+        normal_device(qd, seed, TID_QDEC)
+        kn = torch.empty((steps, B, Hkv, d), dtype=dt, device=device)
+        vn = torch.empty((steps, B, Hkv, d), dtype=dt, device=device)
+        normal_device(kn, seed, TID_KNEW)
+        normal_device(vn, seed, TID_VNEW)
+        out.update(q_dec=qd, k_new=kn, v_new=vn)
+        out["seq_lens"] = torch.full((B,), w.seq_len, dtype=torch.int32, device=device)
+        if w.needles:
+            chunks = needle_chunks(seed, w.needles, w.seq_len // S)
+            q0 = qd[0].double()                                    # [B][Hq][d]
+            for b in range(B):
+                for g in range(Hkv):
+                    v = 4.0 * q0[b, g * group] / torch.linalg.vector_norm(q0[b, g * group])
+                    for c in chunks:
+                        lm[b, int(c), g] = v.float().to(dt)
+            out["needle_chunks"] = chunks
+    out["landmarks"] = lm
+    return out

@@ -1,0 +1,158 @@
+/*
+ * hils.h -- C ABI of the HiLS (Hierarchical Landmark Sparse) attention forward
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Hierarchical Sparse Attention Done Right"; ai-feeds.com digest,
+ * section 方法; oopus.info review, section 二; chatpaper abstract):
+ *   a1  low-rank query calibration      q~ = q + (q A) B            (digest, 输入与分块)
+ *   a2  landmark scoring                s_j = q~ . lm_j / sqrt(d)   (digest, 关键模块 item 1)
+ *   a3  selection: own chunk c(i) = floor(i/S) plus the top-(k-1) chunks j < c(i),
+ *       ordered by (score desc, chunk index asc)                    (digest, 关键模块 item 2)
+ *   a4  fusion weights w = softmax(selected scores)                 (digest, item 1 outer softmax)
+ *   a5  per-chunk attention O_j = softmax(q K_j^T / sqrt(d)) V_j with the raw q,
+ *       keys at positions <= i in the own chunk                     (abstract; digest item 2)
+ *   a6  fused output out = sum_j w_j O_j                            (review, 融合; abstract)
+ *   a7  chunk-granular paged KV access: one page = one chunk        (digest, 关键模块 item 3)
+ *   a8  decode step: append k_t, v_t, then row t of the prefill     (digest, 局限: per-step scan)
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor arguments are caller-owned DEVICE pointers, 16-byte aligned,
+ *     densely packed in the layouts below (row-major, last index fastest).
+ *     The library allocates nothing; scratch comes from the caller's workspace.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on that stream; none synchronises the device.
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns an error status and launches nothing.  The message of the
+ *     last failure on the calling thread is available from hils_last_error().
+ *   - Kernels check block-table entries against num_pages and chunk indices
+ *     against max_chunks; an out-of-range entry skips the access and sets a
+ *     device error word that hils_device_status() reports and clears.
+ *   - Inputs are assumed finite.
+ *   - Shapes: head_dim 64 or 128; chunk_size 64; 1 <= top_k <= 32;
+ *     0 <= calib_rank <= 64; n_q_heads a multiple of n_kv_heads.
+ */
+#ifndef HILS_H_
+#define HILS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HILS_OK = 0,
+  HILS_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+  HILS_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96) */
+  HILS_ERR_WORKSPACE = 3,     /* workspace smaller than hils_workspace_size() */
+  HILS_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  HILS_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+  HILS_ERR_DEVICE_CHECK = 6   /* a device-side bounds check fired */
+} hils_status;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+typedef enum { HILS_OP_SCORE = 0, HILS_OP_TOPK = 1, HILS_OP_PREFILL = 2, HILS_OP_DECODE = 3 } hils_op;
+
+typedef struct {
+  int32_t batch;       /* B: sequences */
+  int32_t n_q_heads;   /* Hq */
+  int32_t n_kv_heads;  /* Hkv; query head h reads KV head h / (Hq/Hkv) */
+  int32_t head_dim;    /* d: 64 or 128 */
+  int32_t chunk_size;  /* S: 64 (one chunk = one KV page) */
+  int32_t top_k;       /* k: own chunk + (k-1) retrieved chunks, 1..32 */
+  int32_t calib_rank;  /* r: rank of the calibration A [d][r], B [r][d]; 0 = none */
+  int32_t dtype;       /* hils_dtype of q, K, V, landmarks, k_new, v_new and out */
+} hils_config;
+
+/* Paged, chunk-granular KV cache (all device memory, owned by the caller). */
+typedef struct {
+  void* pages;                /* [num_pages][2][n_kv_heads][chunk_size][head_dim], [.][0] = K, [.][1] = V */
+  int64_t num_pages;
+  const int32_t* block_table; /* [batch][max_chunks]: logical chunk j of sequence b -> page */
+  int32_t max_chunks;
+  const void* landmarks;      /* [batch][max_chunks][n_kv_heads][head_dim]: one landmark key per chunk
+                                 and KV head, supplied by the caller for every chunk in use,
+                                 including a partially filled last chunk */
+  int32_t* seq_lens;          /* [batch] tokens present; read by hils_decode, advanced by it when appending */
+} hils_kv_cache;
+
+/* Bytes of workspace that `op` needs for this configuration.  q_len is the
+ * number of query positions per sequence (prefill; 1 for decode) and
+ * max_chunks the cache's block-table width.  Returns 0 when none is needed or
+ * on a bad argument (then hils_last_error() says which). */
+size_t hils_workspace_size(const hils_config* cfg, int op, int64_t q_len, int32_t max_chunks);
+
+/* a1 + a2 materialised, for tests and small inputs.
+ * q       [B][q_len][Hq][d]  queries at positions q_pos0 .. q_pos0+q_len-1
+ * A, B    float32 [d][r], [r][d] (ignored when calib_rank == 0)
+ * scores  float32 [B][q_len][Hq][n_cols]; column j holds s_j for j <= floor(pos/S)
+ *         and -inf after it.  Requires floor((q_pos0+q_len-1)/S) < n_cols <= max_chunks. */
+int hils_score(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0, const float* A,
+               const float* B, const hils_kv_cache* cache, float* scores, int32_t n_cols,
+               void* stream);
+
+/* a3 + a4 on materialised scores (layout as hils_score writes it).
+ * idx  int32 [B][q_len][Hq][k]: slot 0 = own chunk, then the selected chunks by
+ *      (score desc, index asc); -1 pads when fewer than k chunks are visible.
+ * w    float32, same shape: softmax of the selected scores, 0 in padded slots. */
+int hils_topk(const hils_config* cfg, const float* scores, int64_t q_len, int64_t q_pos0,
+              int32_t n_cols, int32_t* idx, float* w, void* stream);
+
+/* a1..a7: the full prefill forward, without materialising scores.
+ * q       [B][q_len][Hq][d] at positions q_pos0 .. q_pos0+q_len-1 of every sequence;
+ *         the cache must hold tokens 0 .. q_pos0+q_len-1 (seq_lens is not read).
+ * out     [B][q_len][Hq][d] in cfg->dtype.
+ * idx_out, w_out  optional [B][q_len][Hq][k] copies of the selection (may be NULL).
+ * ws      workspace of at least hils_workspace_size(cfg, HILS_OP_PREFILL, q_len, max_chunks) bytes,
+ *         256-byte aligned; its contents need not be initialised. */
+int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
+                 const float* A, const float* B, const hils_kv_cache* cache, void* out,
+                 int32_t* idx_out, float* w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* a8: one decode step for every sequence of the batch.
+ * q             [B][Hq][d]: one query per sequence.
+ * k_new, v_new  [B][Hkv][d] or both NULL.  When given, each sequence's new token is
+ *               written at position t = seq_lens[b] (its chunk's page must be in the
+ *               block table) and seq_lens[b] is advanced to t+1 on the device at the
+ *               end of the step, so repeated calls (or a captured graph) walk forward.
+ *               When NULL, the token at t = seq_lens[b]-1 must already be present.
+ * out           [B][Hq][d] in cfg->dtype; idx_out, w_out optional [B][Hq][k].
+ * ws            at least hils_workspace_size(cfg, HILS_OP_DECODE, 1, max_chunks) bytes,
+ *               256-byte aligned; zero it once before the first call (cudaMemset)
+ *               and keep it for later calls with the same configuration: its
+ *               completion counters return to zero at the end of every step. */
+int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const void* v_new,
+                const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
+                float* w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reports and clears the device error word set by
+ * the kernels' bounds checks: HILS_OK or HILS_ERR_DEVICE_CHECK (HILS_ERR_CUDA if the
+ * synchronisation itself failed). */
+int hils_device_status(void* stream);
+
+/* Kernel timing with CUDA events, for benchmarking (not thread-safe).
+ * hils_profile_enable(1): from now on every kernel the library launches is
+ * bracketed by an event pair recorded on the call's stream.
+ * hils_profile_collect(): waits for the recorded events and adds their
+ * elapsed times to per-phase totals (phase = kernel name, e.g. "prefill.select").
+ * hils_profile_read(i, ...): phase i's name, total milliseconds and launch
+ * count; returns HILS_ERR_INVALID_ARG past the last phase.
+ * hils_profile_reset(): collects pending events, then clears the totals. */
+int hils_profile_enable(int on);
+int hils_profile_collect(void);
+int hils_profile_read(int i, const char** name, double* total_ms, long long* launches);
+int hils_profile_reset(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* hils_last_error(void);
+
+/* Library version, e.g. "hils-b200 0.1.0 sm_100a". */
+const char* hils_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H_ */

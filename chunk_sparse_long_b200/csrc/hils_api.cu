@@ -242,3 +242,8 @@ const char* hils_last_error(void) { return g_last_error.c_str(); }
 const char* hils_version(void) { return "hils-b200 0.1.0 sm_100a"; }
 
 }  // extern "C"
+
+namespace hils {
+// Lets other translation units of the library report through hils_last_error().
+void record_error(const char* msg) { g_last_error = msg; }
+}  // namespace hils

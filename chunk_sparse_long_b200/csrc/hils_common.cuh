@@ -111,6 +111,9 @@ class ProfileScope {
 };
 #define HILS_PROFILE(name, stream) ::hils::ProfileScope _hils_prof_scope_(name, stream)
 
+// Sets the message hils_last_error() returns on this thread.
+void record_error(const char* msg);
+
 // ---- launchers (each returns cudaError_t of its launches) -----------------
 cudaError_t launch_score(const Params& P, float* scores, int n_cols, cudaStream_t s);
 cudaError_t launch_topk(const Params& P, const float* scores, int n_cols, int32_t* idx, float* w,

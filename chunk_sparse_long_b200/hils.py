@@ -25,7 +25,8 @@ STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
 
 EXPORTED = ("hils_workspace_size", "hils_score", "hils_topk", "hils_prefill", "hils_decode",
             "hils_device_status", "hils_last_error", "hils_version", "hils_profile_enable",
-            "hils_profile_collect", "hils_profile_read", "hils_profile_reset")
+            "hils_profile_collect", "hils_profile_read", "hils_profile_reset",
+            "hils_decode_noalloc", "hils_decode_noalloc_capacity")
 
 
 class HilsError(RuntimeError):
@@ -87,6 +88,10 @@ def load(path: str = LIB_PATH):
                                     ctypes.POINTER(ctypes.c_longlong)]
     L.hils_profile_reset.restype = ctypes.c_int
     L.hils_profile_reset.argtypes = []
+    L.hils_decode_noalloc.restype = ctypes.c_int
+    L.hils_decode_noalloc.argtypes = [cfgp, P, P, P, P, P, cachep, P, P, P, P]
+    L.hils_decode_noalloc_capacity.restype = ctypes.c_size_t
+    L.hils_decode_noalloc_capacity.argtypes = []
     _lib = L
     return L
 
@@ -175,6 +180,19 @@ def decode(cfg, q, k_new, v_new, A, B, cache: Cache, out, idx_out, w_out, ws, ws
     _check(load().hils_decode(ctypes.byref(cfg.c()), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(A),
                               _ptr(B), ctypes.byref(cache.c()), _ptr(out), _ptr(idx_out),
                               _ptr(w_out), _ptr(ws), ws_bytes, _stream(stream)), "hils_decode")
+
+
+def decode_noalloc(cfg, q, k_new, v_new, A, B, cache: Cache, out, idx_out, w_out, stream=None):
+    """hils_decode for callers that cannot allocate: scratch is the library's
+    built-in array (see include/hils.h); calls on one device must not overlap."""
+    _check(load().hils_decode_noalloc(ctypes.byref(cfg.c()), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                      _ptr(A), _ptr(B), ctypes.byref(cache.c()), _ptr(out),
+                                      _ptr(idx_out), _ptr(w_out), _stream(stream)),
+           "hils_decode_noalloc")
+
+
+def decode_noalloc_capacity() -> int:
+    return int(load().hils_decode_noalloc_capacity())
 
 
 def device_status(stream=None):

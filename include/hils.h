@@ -127,6 +127,27 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
                 const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, void* stream);
 
+/* The decode step without a workspace argument, for callers that cannot
+ * allocate device memory: plugins run by a host engine that owns every device
+ * allocation and passes kernels only their inputs and outputs, and services
+ * that must not allocate once they are serving (cudaMalloc can synchronise the
+ * device and can fail under memory pressure).  The paper has no counterpart:
+ * this is a deployment convenience around hils_decode.
+ * Arguments and results are those of hils_decode.  Its scratch is one array of
+ * hils_decode_noalloc_capacity() bytes (4 MiB) built into the library, which
+ * every GPU that loads the library holds until the process exits; a
+ * configuration that needs more returns HILS_ERR_WORKSPACE (use hils_decode).
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture.  Each call clears the array's
+ * completion counters (a cudaMemsetAsync on `stream`) and otherwise reuses
+ * what the previous call left there.  All calls on one device share the array:
+ * calls that overlap on the GPU (other streams, other threads) race and give
+ * wrong results, so serialise them.  Allocates no memory. */
+int hils_decode_noalloc(const hils_config* cfg, const void* q, const void* k_new,
+                        const void* v_new, const float* A, const float* B, hils_kv_cache* cache,
+                        void* out, int32_t* idx_out, float* w_out, void* stream);
+size_t hils_decode_noalloc_capacity(void);
+
 /* Synchronises `stream`, then reports and clears the device error word set by
  * the kernels' bounds checks: HILS_OK or HILS_ERR_DEVICE_CHECK (HILS_ERR_CUDA if the
  * synchronisation itself failed). */

@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_KERNELS_PER_STEP = 6   # select, count, scan, scatter, attend, finish
+PREFILL_KERNELS_PER_STEP = 6   # select, count, scan, scatter, attend, merge (bf16 path)
 DECODE_KERNELS_PER_STEP = 2    # scan (+append, selection), attend (+merge)
 
 
@@ -228,7 +228,7 @@ def time_prefill_e2e(hils, torch, wl, steps, warmup):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def time_decode(hils, torch, wl, warmup_steps=8):
+def time_decode(hils, torch, wl, warmup_steps=8, n_steps=0):
     """All decode steps of the workload, one after another (each appends its
     token); L2 is flushed before every step and only the step itself is timed."""
     w = wl["workload"]
@@ -260,7 +260,7 @@ def time_decode(hils, torch, wl, warmup_steps=8):
     run(warmup_steps, False)
     hils.profile_reset()
     hils.profile_enable(True)
-    times = run(w.decode_steps, True)
+    times = run(n_steps if n_steps > 0 else w.decode_steps, True)
     hils.profile_enable(False)
     phases = hils.profile_read()
     hils.device_status(stream)
@@ -339,6 +339,10 @@ def main():
     ap.add_argument("--workload", default="prefill_128k_gqa")
     ap.add_argument("--decode-workload", default="decode_512k")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--skip-prefill", action="store_true",
+                    help="time only the decode workload (for profiling runs)")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="timed decode steps (default: all of the workload's steps)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
@@ -384,6 +388,15 @@ def main():
         build.build()
     barrier()
     hils.load()
+    if args.skip_prefill:
+        dw = hi.WORKLOADS[args.decode_workload]
+        dwl = hi.device_workload(dw, seed_offset=rank)
+        times, dph = time_decode(hils, torch, dwl, n_steps=args.decode_steps)
+        if rank == 0:
+            print(json.dumps({"decode_only": dw.name, "us_per_step": statistics.mean(times) * 1e3,
+                              "kernels_us_per_step": {k: v[0] / max(1, v[1]) * 1e3
+                                                      for k, v in dph.items()}}))
+        return
     wl = hi.device_workload(w, seed_offset=rank)
     torch.cuda.synchronize()
     ms, phases, clocks, _keep = time_prefill(hils, torch, wl, args.steps, args.warmup, barrier,
@@ -394,10 +407,10 @@ def main():
     dom = max(phases.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms_total, dom_launches) = dom
     dom_ms = dom_ms_total / max(1, dom_launches)
-    if dom_name == "prefill.attend":
+    if dom_name.startswith("prefill.attend"):
         work, what = counts["attention_flop"], "useful attention flop (QK^T + PV over selected keys)"
-    elif dom_name == "prefill.select":
-        work, what = counts["score_flop"] + counts["calib_flop"], "landmark scoring + calibration flop"
+    elif dom_name.startswith("prefill.select"):
+        work, what = counts["score_flop"], "useful landmark-scoring flop (q~ . landmark, causal chunks)"
     else:
         work, what = counts["attention_flop"], "useful attention flop"
     achieved = work / (dom_ms / 1e3) / 1e12
@@ -426,9 +439,9 @@ def main():
     if not args.no_decode:
         dw = hi.WORKLOADS[args.decode_workload]
         dwl = hi.device_workload(dw, seed_offset=rank)
-        times, dph = time_decode(hils, torch, dwl)
+        times, dph = time_decode(hils, torch, dwl, n_steps=args.decode_steps)
         us = maxreduce(statistics.mean(times)) * 1e3
-        by = [decode_bytes(dw, s) for s in range(dw.decode_steps)]
+        by = [decode_bytes(dw, s) for s in range(len(times))]
         tot = statistics.mean(b["total"] for b in by)
         kvb = statistics.mean(b["kv_bytes"] for b in by)
         lmb = statistics.mean(b["landmark_bytes"] for b in by)
@@ -437,7 +450,7 @@ def main():
         dms_per = dms / max(1, dl)
         dbytes = lmb if dn == "decode.scan" else kvb
         result["decode"] = {
-            "workload": dw.name, "us_per_step": us, "steps": dw.decode_steps,
+            "workload": dw.name, "us_per_step": us, "steps": len(times),
             "context": dw.seq_len, "bytes_per_step": tot, "landmark_bytes": lmb, "kv_bytes": kvb,
             "step_gbs": tot / (us / 1e6) / 1e9,
             "step_hbm_frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"],
@@ -447,7 +460,7 @@ def main():
                          "frac": dbytes / (dms_per / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
                          "peak_source": f"{pk_src} HBM copy bandwidth"},
             "l2": "flushed (256 MB write) before every step; only the step is timed",
-            "gpu_launches": DECODE_KERNELS_PER_STEP * dw.decode_steps,
+            "gpu_launches": DECODE_KERNELS_PER_STEP * len(times),
         }
         del dwl
     if rank == 0 and nworld == 1 and not args.no_cpu_baseline:

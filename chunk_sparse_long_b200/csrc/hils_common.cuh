@@ -11,6 +11,7 @@
 namespace hils {
 
 constexpr int kChunk = 64;       // chunk_size the kernels are written for
+constexpr int kItemPairs = 512;  // pairs per tensor-core attention work item (4 tiles of 128)
 constexpr int kMaxTopK = 32;
 constexpr int kMaxRank = 64;
 
@@ -127,13 +128,18 @@ struct PrefillWs {
   int32_t* tile_off; // [n_keys + 1] tile offsets
   int32_t* cursor;   // [n_keys]
   int32_t* pairs;    // [rows * k] pair ids (row * k + slot)
-  float* acc;        // [rows][d]
+  float* acc;        // [rows][d] float32 accumulator (CUDA-core attention)
+  void* partial;     // [rows * k][d] bf16 per-pair partial outputs (tensor-core attention)
+  int32_t* queue;    // work-item counter of the persistent attention kernel
   int n_keys;
   int64_t max_tiles;
 };
 size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base);
 cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
                            const PrefillWs& ws, cudaStream_t s);
+cudaError_t launch_select_tc(const Params& P, int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const PrefillWs& ws,
+                           cudaStream_t s);
 
 struct DecodeWs {
   float* cand_s;       // [B][n_split][Hq][k-1]

@@ -169,8 +169,8 @@ __global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int6
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n_keys,
-                                                    int32_t* offsets, int32_t* tile_off,
-                                                    int32_t* cursor) {
+                                                    int tile_pairs, int32_t* offsets,
+                                                    int32_t* tile_off, int32_t* cursor) {
   __shared__ int32_t sp[1024], stl[1024];
   const int t = threadIdx.x;
   const int per = (n_keys + 1023) / 1024;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n
   int32_t ps = 0, ts = 0;
   for (int key = k0; key < k1; ++key) {
     ps += counts[key];
-    ts += (counts[key] + kTilePairs - 1) / kTilePairs;
+    ts += (counts[key] + tile_pairs - 1) / tile_pairs;
   }
   sp[t] = ps;
   stl[t] = ts;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n
     cursor[key] = po;
     tile_off[key] = to;
     po += counts[key];
-    to += (counts[key] + kTilePairs - 1) / kTilePairs;
+    to += (counts[key] + tile_pairs - 1) / tile_pairs;
   }
   if (t == 1023) {
     offsets[n_keys] = sp[1023];
@@ -308,26 +308,34 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
   const int64_t n_pairs = rows * P.k;
   cudaError_t e;
   // a1..a4
-  const size_t ssm = select_smem<D>(P.r);
-  e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
-  if (e != cudaSuccess) return e;
-  dim3 sg((unsigned)((P.L + kSelThreads - 1) / kSelThreads), P.Hq, P.B);
-  {
-    HILS_PROFILE("prefill.select", s);
-    select_kernel<D><<<sg, kSelThreads, ssm, s>>>(P, ws.idx, ws.w);
+  if (P.dtype == HILS_BF16) {
+    if ((e = launch_select_tc(P, ws.idx, ws.w, s)) != cudaSuccess) return e;
+  } else {
+    const size_t ssm = select_smem<D>(P.r);
+    e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ssm);
+    if (e != cudaSuccess) return e;
+    dim3 sg((unsigned)((P.L + kSelThreads - 1) / kSelThreads), P.Hq, P.B);
+    {
+      HILS_PROFILE("prefill.select", s);
+      select_kernel<D><<<sg, kSelThreads, ssm, s>>>(P, ws.idx, ws.w);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // bucket by (sequence, KV head, chunk)
   if ((e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ws.n_keys, s)) != cudaSuccess) return e;
   const unsigned pb = (unsigned)((n_pairs + 255) / 256);
   {
     HILS_PROFILE("prefill.bucket", s);
     count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs);
-    scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, ws.offsets, ws.tile_off, ws.cursor);
+    const int tile_pairs = P.dtype == HILS_BF16 ? kItemPairs : kTilePairs;
+    scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
+                                   ws.cursor);
     scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, n_pairs);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // a5 + a6
+  if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws.idx, ws, s);
   if ((e = cudaMemsetAsync(ws.acc, 0, sizeof(float) * rows * D, s)) != cudaSuccess) return e;
   constexpr size_t asm_ = attend_smem<D>();
   e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -369,7 +377,12 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
   w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
-  w.acc = (float*)take(sizeof(float) * rows * P.d);
+  if (P.dtype == HILS_BF16) {
+    w.partial = take((size_t)2 * n_pairs * P.d);
+  } else {
+    w.acc = (float*)take(sizeof(float) * rows * P.d);
+  }
+  w.queue = (int32_t*)take(sizeof(int32_t));
   w.n_keys = (int)n_keys;
   w.max_tiles = (n_pairs + kTilePairs - 1) / kTilePairs + n_keys;
   if (ws) *ws = w;

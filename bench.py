@@ -257,10 +257,14 @@ def time_decode(hils, torch, wl, warmup_steps=8, n_steps=0):
         torch.cuda.synchronize()
         return [a.elapsed_time(b) for a, b in evs]
 
+    n = n_steps if n_steps > 0 else w.decode_steps
     run(warmup_steps, False)
+    # step times without per-kernel events (they would separate the two kernels)
+    times = run(n, True)
+    # per-kernel times from a second pass over the same steps
     hils.profile_reset()
     hils.profile_enable(True)
-    times = run(n_steps if n_steps > 0 else w.decode_steps, True)
+    run(n, True)
     hils.profile_enable(False)
     phases = hils.profile_read()
     hils.device_status(stream)

@@ -76,11 +76,14 @@ extern "C" int hils_decode_noalloc(const hils_config* cfg, const void* q, const 
   if (st != HILS_OK) return st;
   // The array keeps whatever the previous call left.  The completion counters
   // must start at zero: clear them (their place depends on the configuration).
-  hils::Params P{};
+  hils::Params P{};   // the fields the workspace carve-up reads
   P.B = cfg->batch;
   P.Hq = cfg->n_q_heads;
+  P.Hkv = cfg->n_kv_heads;
   P.d = cfg->head_dim;
   P.k = cfg->top_k;
+  P.r = cfg->calib_rank;
+  P.dtype = cfg->dtype;
   P.max_chunks = cache->max_chunks;
   hils::DecodeWs w{};
   hils::decode_ws_bytes(P, &w, (char*)scratch);

@@ -142,8 +142,10 @@ cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const
                            cudaStream_t s);
 
 struct DecodeWs {
-  float* cand_s;       // [B][n_split][Hq][k-1]
+  float* cand_s;       // [B][n_split][Hq][k-1] each split's best candidates, best first
   int32_t* cand_j;     // same
+  float* best;         // [B][Hq][n_split] each split's best score (-inf if none)
+  float* s_own;        // [B][Hq] the own chunk's score
   int32_t* idx;        // [B][Hq][k]
   float* w;            // [B][Hq][k]
   float* part;         // [B][Hq][k][d]

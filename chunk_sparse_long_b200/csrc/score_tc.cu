@@ -14,13 +14,14 @@
 //       accumulated by 3 x d/16 tcgen05.mma (M=128, N=128) into one of two
 //       TMEM buffers, so the MMAs of block n+1 run while block n is consumed.
 //   a3  thread t reads its 128 scores from TMEM, 32 columns at a time, and keeps
-//       the k-1 best candidates j < own in a min-heap whose root is the worst
-//       kept one.  A lane first builds the bitmask of columns that beat its
-//       root (the same work in every lane), then the warp loops max(popcount)
-//       times, each lane inserting its next set column -- so lanes do not
-//       serialise each other's inserts.  Strict '>' against the root while j
-//       ascends keeps the lower index on ties; the own chunk's score is kept
-//       apart.  The heap is sorted (score desc, index asc) at the end.
+//       the k-1 best candidates j < own in a sorted list held in registers
+//       (worst kept entry first).  A lane first builds the bitmask of columns
+//       that beat its worst entry (the same work in every lane), then the warp
+//       loops max(popcount) times, each lane inserting its next set column
+//       through an unrolled compare-and-shift network -- lanes do not
+//       serialise each other's inserts and nothing waits on memory.  Strict
+//       '>' against the worst entry while j ascends keeps the lower index on
+//       ties; the own chunk's score is kept apart.
 //   a4  softmax of the own and selected scores -> idx, w.
 #include <cfloat>
 
@@ -43,8 +44,8 @@ struct ScoreLayout {
   static constexpr uint32_t kLmB = kBlk * D * 2;              // one landmark block
   static constexpr uint32_t kQ = 0;                           // kTerms tiles
   static constexpr uint32_t kLm = kTerms * kQt;               // kLmBufs blocks
-  static constexpr uint32_t kList = kLm + kLmBufs * kLmB;     // heap [kMaxTopK][128] + ids
-  static constexpr uint32_t kEnd = kList + 2 * kMaxTopK * kThrS * 4;
+  static constexpr uint32_t kScratch = kLm + kLmBufs * kLmB;  // calibration t = qA [r][128]
+  static constexpr uint32_t kEnd = kScratch + kMaxRank * kThrS * 4;
   static constexpr uint32_t kSmem = kEnd + 1024;
 };
 
@@ -68,33 +69,38 @@ __device__ __forceinline__ bool worse(float sa, int ja, float sb, int jb) {
   return sa < sb || (sa == sb && ja > jb);
 }
 
-// Replaces the root of the thread's min-heap (column `tid` of [K][kThrS]; the
-// root is the worst kept entry) by (s, j) and restores the heap order.
-__device__ __noinline__ void heap_replace_root(float* hS, int* hJ, int tid, int K, float s, int j) {
-  int i = 0;
-  for (;;) {
-    const int l = 2 * i + 1;
-    if (l >= K) break;
-    int c = l;
-    float cs = hS[l * kThrS + tid];
-    int cj = hJ[l * kThrS + tid];
-    if (l + 1 < K) {
-      const float rs = hS[(l + 1) * kThrS + tid];
-      const int rj = hJ[(l + 1) * kThrS + tid];
-      if (worse(rs, rj, cs, cj)) {
-        c = l + 1;
-        cs = rs;
-        cj = rj;
-      }
+// The k-1 best candidates of one row, kept in registers in ascending order
+// (index 0 = the worst kept entry, compared against every new candidate).
+// Slots [K, KS) hold +inf sentinels that no candidate beats, slots [0, K)
+// start as -inf sentinels that every candidate beats; KS is a compile-time
+// bound so the insertion network below is fully unrolled (no local memory).
+template <int KS>
+struct RegList {
+  float s[KS];
+  int j[KS];
+
+  __device__ __forceinline__ void init(int K) {
+#pragma unroll
+    for (int p = 0; p < KS; ++p) {
+      s[p] = p < K ? -INFINITY : INFINITY;
+      j[p] = p < K ? INT32_MAX : -1;
     }
-    if (!worse(cs, cj, s, j)) break;
-    hS[i * kThrS + tid] = cs;
-    hJ[i * kThrS + tid] = cj;
-    i = c;
   }
-  hS[i * kThrS + tid] = s;
-  hJ[i * kThrS + tid] = j;
-}
+  // Drops entry 0 and inserts (ns, nj), which must rank above entry 0:
+  // every slot takes its upper neighbour, the new entry, or keeps its value.
+  __device__ __forceinline__ void insert(float ns, int nj) {
+    bool c[KS + 1];
+#pragma unroll
+    for (int p = 0; p < KS; ++p) c[p] = worse(s[p], j[p], ns, nj);
+    c[KS] = false;
+#pragma unroll
+    for (int p = 0; p < KS; ++p) {
+      const bool up = p + 1 < KS && c[p + 1];
+      s[p] = up ? s[p + 1] : (c[p] ? ns : s[p]);
+      j[p] = up ? j[p + 1] : (c[p] ? nj : j[p]);
+    }
+  }
+};
 
 // v[x] for a runtime x in 0..31 without dynamic register indexing (select tree).
 __device__ __forceinline__ uint32_t pick32(const uint32_t (&v)[32], int x) {
@@ -110,7 +116,7 @@ __device__ __forceinline__ uint32_t pick32(const uint32_t (&v)[32], int x) {
   return (x & 1) ? a[1] : a[0];
 }
 
-template <int D>
+template <int D, int KS>
 __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* idx, float* w) {
   using Lay = ScoreLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -143,7 +149,7 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
     tc::tmem_relinquish();
   }
 
-  // ---- a1: q~ in float32 (A and B staged in the landmark buffers) ----------
+  // ---- a1: q~ in float32 (A, B staged in the landmark buffers, qA in scratch) --
   float qt[D];
 #pragma unroll
   for (int e = 0; e < D; e += 8) {
@@ -155,24 +161,43 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
     }
   }
   if (P.r > 0) {
-    float* sA = reinterpret_cast<float*>(smem + Lay::kLm);
-    float* sB = sA + D * P.r;
-    float* sT = reinterpret_cast<float*>(smem + Lay::kList);   // [r][128]
-    for (int x = tid; x < D * P.r; x += kThrS) {
-      sA[x] = P.A[x];
-      sB[x] = P.Bm[x];
+    const int r4 = (P.r + 3) & ~3;                 // A rows padded to a multiple of 4
+    float* sA = reinterpret_cast<float*>(smem + Lay::kLm);        // [D][r4]
+    float* sB = sA + D * r4;                                      // [r][D]
+    float* sT = reinterpret_cast<float*>(smem + Lay::kScratch);   // [r4][128]
+    for (int x = tid; x < D * r4; x += kThrS) {
+      const int e = x / r4, a = x % r4;
+      sA[x] = a < P.r ? P.A[e * P.r + a] : 0.f;
     }
+    for (int x = tid; x < P.r * D; x += kThrS) sB[x] = P.Bm[x];
     __syncthreads();
-    for (int a = 0; a < P.r; ++a) {
-      float acc = 0.f;
+    // t = q A: four independent accumulator chains per pass, 16-byte broadcast loads
+    for (int a = 0; a < r4; a += 4) {
+      float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
 #pragma unroll
-      for (int e = 0; e < D; ++e) acc = fmaf(qt[e], sA[e * P.r + a], acc);
-      sT[a * kThrS + tid] = acc;
+      for (int e = 0; e < D; ++e) {
+        const float4 av = *reinterpret_cast<const float4*>(sA + e * r4 + a);
+        t0 = fmaf(qt[e], av.x, t0);
+        t1 = fmaf(qt[e], av.y, t1);
+        t2 = fmaf(qt[e], av.z, t2);
+        t3 = fmaf(qt[e], av.w, t3);
+      }
+      sT[(a + 0) * kThrS + tid] = t0;
+      sT[(a + 1) * kThrS + tid] = t1;
+      sT[(a + 2) * kThrS + tid] = t2;
+      sT[(a + 3) * kThrS + tid] = t3;
     }
+    // q~ = q + t B
     for (int a = 0; a < P.r; ++a) {
       const float ta = sT[a * kThrS + tid];
 #pragma unroll
-      for (int e = 0; e < D; ++e) qt[e] = fmaf(ta, sB[a * D + e], qt[e]);
+      for (int e = 0; e < D; e += 4) {
+        const float4 bv = *reinterpret_cast<const float4*>(sB + a * D + e);
+        qt[e] = fmaf(ta, bv.x, qt[e]);
+        qt[e + 1] = fmaf(ta, bv.y, qt[e + 1]);
+        qt[e + 2] = fmaf(ta, bv.z, qt[e + 2]);
+        qt[e + 3] = fmaf(ta, bv.w, qt[e + 3]);
+      }
     }
   }
   // three-term bf16 split of q~ into the A tiles
@@ -197,7 +222,7 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
   }
   tc::fence_proxy_async();
   tc::tc_fence_before();
-  __syncthreads();   // A/B/T scratch is dead from here on
+  __syncthreads();   // A, B and t scratch are dead from here on
   tc::tc_fence_after();
   const uint32_t tmem = tmem_sh;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -205,13 +230,8 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
 
   // ---- a2/a3: landmark blocks --------------------------------------------
   const int K = P.k - 1;
-  float* lsS = reinterpret_cast<float*>(smem + Lay::kList);
-  int* lsJ = reinterpret_cast<int*>(lsS + kMaxTopK * kThrS);
-  for (int a = 0; a < K; ++a) {   // sentinels: worse than any real candidate
-    lsS[a * kThrS + tid] = -INFINITY;
-    lsJ[a * kThrS + tid] = INT32_MAX;
-  }
-  float thr = -INFINITY;          // score of the heap root
+  RegList<KS> list;
+  list.init(K);
   float s_own = 0.f;
   uint32_t phase[2] = {0u, 0u};
 
@@ -233,22 +253,20 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
       tc::tmem_ld32(tmem + sb * kBlk + lane_off + c0, sv);
       tc::tmem_ld_wait();
       uint32_t m = 0;
+      const float thr = list.s[0];
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int64_t j = j0 + c0 + x;
         const float s = __uint_as_float(sv[x]) * P.inv_sqrt_d;
         if (j == own) s_own = s;
-        m |= (K > 0 && j < own && s > thr) ? (1u << x) : 0u;
+        m |= (j < own && s > thr) ? (1u << x) : 0u;
       }
       while (__any_sync(0xffffffffu, m != 0)) {
         if (m) {
           const int x = __ffs(m) - 1;
           m &= m - 1;
           const float s = __uint_as_float(pick32(sv, x)) * P.inv_sqrt_d;
-          if (s > thr) {
-            heap_replace_root(lsS, lsJ, tid, K, s, (int)(j0 + c0 + x));
-            thr = lsS[tid];
-          }
+          if (s > list.s[0]) list.insert(s, (int)(j0 + c0 + x));
         }
       }
     }
@@ -291,38 +309,31 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
   }
   consume(n_blk - 1);
 
-  // ---- sort the kept candidates (score desc, index asc); sentinels sink ----
-  for (int a = 1; a < K; ++a) {
-    const float ks = lsS[a * kThrS + tid];
-    const int kj = lsJ[a * kThrS + tid];
-    int p = a;
-    while (p > 0 && worse(lsS[(p - 1) * kThrS + tid], lsJ[(p - 1) * kThrS + tid], ks, kj)) {
-      lsS[p * kThrS + tid] = lsS[(p - 1) * kThrS + tid];
-      lsJ[p * kThrS + tid] = lsJ[(p - 1) * kThrS + tid];
-      --p;
-    }
-    lsS[p * kThrS + tid] = ks;
-    lsJ[p * kThrS + tid] = kj;
-  }
-  int n = 0;
-  while (n < K && lsJ[n * kThrS + tid] != INT32_MAX) ++n;
-
-  // ---- a4: fusion weights ------------------------------------------------
+  // ---- a4: fusion weights; the list is read best-first -------------------
   if (valid) {
     float m = s_own;
-    for (int a = 0; a < n; ++a) m = fmaxf(m, lsS[a * kThrS + tid]);
+#pragma unroll
+    for (int p = 0; p < KS; ++p)
+      if (list.j[p] != INT32_MAX && list.j[p] >= 0) m = fmaxf(m, list.s[p]);
     float z = __expf(s_own - m);
-    for (int a = 0; a < n; ++a) z += __expf(lsS[a * kThrS + tid] - m);
+#pragma unroll
+    for (int p = 0; p < KS; ++p)
+      if (list.j[p] != INT32_MAX && list.j[p] >= 0) z += __expf(list.s[p] - m);
     const float iz = 1.f / z;
     int32_t* ix = idx + r * P.k;
     float* wr = w + r * P.k;
     ix[0] = (int32_t)own;
     wr[0] = __expf(s_own - m) * iz;
-    for (int a = 0; a < n; ++a) {
-      ix[1 + a] = lsJ[a * kThrS + tid];
-      wr[1 + a] = __expf(lsS[a * kThrS + tid] - m) * iz;
+    int n = 1;
+#pragma unroll
+    for (int p = KS - 1; p >= 0; --p) {
+      if (list.j[p] != INT32_MAX && list.j[p] >= 0) {
+        ix[n] = list.j[p];
+        wr[n] = __expf(list.s[p] - m) * iz;
+        ++n;
+      }
     }
-    for (int a = n + 1; a < P.k; ++a) {
+    for (int a = n; a < P.k; ++a) {
       ix[a] = -1;
       wr[a] = 0.f;
     }
@@ -334,22 +345,25 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsS);
 }
 
-template <int D>
+template <int D, int KS>
 cudaError_t run_score_tc(const Params& P, int32_t* idx, float* w, cudaStream_t s) {
   using Lay = ScoreLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D, KS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((P.L + kRowsS - 1) / kRowsS), P.Hq, P.B);
   HILS_PROFILE("prefill.select_tc", s);
-  score_tc_kernel<D><<<grid, kThrS, Lay::kSmem, s>>>(P, idx, w);
+  score_tc_kernel<D, KS><<<grid, kThrS, Lay::kSmem, s>>>(P, idx, w);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_select_tc(const Params& P, int32_t* idx, float* w, cudaStream_t s) {
-  return P.d == 64 ? run_score_tc<64>(P, idx, w, s) : run_score_tc<128>(P, idx, w, s);
+  // the register list holds 16 or 32 slots (k-1 <= 31)
+  if (P.k - 1 <= 16)
+    return P.d == 64 ? run_score_tc<64, 16>(P, idx, w, s) : run_score_tc<128, 16>(P, idx, w, s);
+  return P.d == 64 ? run_score_tc<64, 32>(P, idx, w, s) : run_score_tc<128, 32>(P, idx, w, s);
 }
 
 }  // namespace hils

@@ -194,6 +194,9 @@ WORKLOADS = {
     "prefill_8k": Workload("prefill_8k", 1, 16, 16, 64, 64, 16, 16, DT_BF16, 8192, 2, "prefill"),
     "prefill_128k_gqa": Workload("prefill_128k_gqa", 1, 32, 8, 128, 64, 32, 32, DT_BF16,
                                  131072, 3, "prefill", needles=1),
+    # the 128K GQA shape at 16K tokens: a profiling-size case (a few GB on the device)
+    "prefill_16k_gqa": Workload("prefill_16k_gqa", 1, 32, 8, 128, 64, 32, 32, DT_BF16, 16384, 3,
+                                "prefill"),
     "decode_512k": Workload("decode_512k", 1, 16, 16, 64, 64, 16, 16, DT_BF16, 524288, 4,
                             "decode", decode_steps=256),
     "decode_128k_b32": Workload("decode_128k_b32", 32, 16, 16, 64, 64, 16, 16, DT_BF16, 131072,

@@ -37,6 +37,7 @@ constexpr int kThrS = 128;
 constexpr int kTerms = 3;
 constexpr uint32_t kTmemColsS = 256;  // two S buffers of 128 columns
 constexpr int kLmBufs = 3;            // landmark blocks in flight: prefetch distance 2
+constexpr int kBulkPasses = 12;       // a chunk this dense for some lane is merged in bulk
 
 template <int D>
 struct ScoreLayout {
@@ -86,18 +87,68 @@ struct RegList {
       j[p] = p < K ? INT32_MAX : -1;
     }
   }
-  // Drops entry 0 and inserts (ns, nj), which must rank above entry 0:
-  // every slot takes its upper neighbour, the new entry, or keeps its value.
+  // Drops entry 0 and inserts (ns, nj), which must rank above entry 0.  New
+  // candidates arrive in ascending chunk order, so a kept entry with the same
+  // score always ranks above the new one: comparing scores alone decides.
+  // Every slot takes its upper neighbour, the new entry, or keeps its value.
   __device__ __forceinline__ void insert(float ns, int nj) {
     bool c[KS + 1];
 #pragma unroll
-    for (int p = 0; p < KS; ++p) c[p] = worse(s[p], j[p], ns, nj);
+    for (int p = 0; p < KS; ++p) c[p] = s[p] < ns;
     c[KS] = false;
 #pragma unroll
     for (int p = 0; p < KS; ++p) {
       const bool up = p + 1 < KS && c[p + 1];
       s[p] = up ? s[p + 1] : (c[p] ? ns : s[p]);
       j[p] = up ? j[p + 1] : (c[p] ? nj : j[p]);
+    }
+  }
+  // Merges 32 new candidates (any order; masked ones as (-inf, INT32_MAX)) into
+  // the list: bitonic sort of the 32 (worst first), then the best KS of the
+  // union by one bitonic merge.  The +inf sentinels above slot K are the best
+  // of all, so exactly the best K real entries stay in slots [0, K).
+  __device__ __forceinline__ void merge32(float (&vs)[32], int (&vj)[32]) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+      for (int m = k >> 1; m > 0; m >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int l = i ^ m;
+          if (l > i) {
+            const bool up = (i & k) == 0;          // ascending block: worst first
+            const bool swap = up ? worse(vs[l], vj[l], vs[i], vj[i])
+                                 : worse(vs[i], vj[i], vs[l], vj[l]);
+            if (swap) {
+              const float ts = vs[i]; vs[i] = vs[l]; vs[l] = ts;
+              const int tj = vj[i]; vj[i] = vj[l]; vj[l] = tj;
+            }
+          }
+        }
+      }
+    }
+    // best KS of the list (ascending) and the top KS of vs (ascending): slot p
+    // takes the better of s[p] and the (p+1)-th best of vs, which leaves a
+    // bitonic sequence holding the best KS; a bitonic merge sorts it
+#pragma unroll
+    for (int p = 0; p < KS; ++p) {
+      const float cs = vs[32 - KS + (KS - 1 - p)];
+      const int cj = vj[32 - KS + (KS - 1 - p)];
+      if (worse(s[p], j[p], cs, cj)) {
+        s[p] = cs;
+        j[p] = cj;
+      }
+    }
+#pragma unroll
+    for (int m = KS >> 1; m > 0; m >>= 1) {
+#pragma unroll
+      for (int i = 0; i < KS; ++i) {
+        const int l = i ^ m;
+        if (l > i && worse(s[l], j[l], s[i], j[i])) {
+          const float ts = s[i]; s[i] = s[l]; s[l] = ts;
+          const int tj = j[i]; j[i] = j[l]; j[l] = tj;
+        }
+      }
     }
   }
 };
@@ -260,6 +311,19 @@ __global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, int32_t* i
         const float s = __uint_as_float(sv[x]) * P.inv_sqrt_d;
         if (j == own) s_own = s;
         m |= (j < own && s > thr) ? (1u << x) : 0u;
+      }
+      if (__reduce_max_sync(0xffffffffu, (unsigned)__popc(m)) >= kBulkPasses) {
+        // dense chunk: sort the 32 columns and merge them in one go
+        float vs[32];
+        int vj[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const bool in = (m >> x) & 1u;
+          vs[x] = in ? __uint_as_float(sv[x]) * P.inv_sqrt_d : -INFINITY;
+          vj[x] = in ? (int)(j0 + c0 + x) : INT32_MAX;
+        }
+        list.merge32(vs, vj);
+        m = 0;
       }
       while (__any_sync(0xffffffffu, m != 0)) {
         if (m) {

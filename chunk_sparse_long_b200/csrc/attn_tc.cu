@@ -2,24 +2,30 @@
 // tensor cores (tcgen05, TMEM accumulators), bf16 inputs.
 //
 // Work is key-major: the (row, slot) pairs are bucketed by (sequence, KV head,
-// chunk) and a work item is up to kItemPairs pairs of one bucket, so the
-// chunk's 64 x d K and V tiles are staged in shared memory once per item and
-// shared by up to four 128-row tiles.  Per 128-row tile:
+// query window, chunk) and a work item is up to kItemPairs pairs of one
+// bucket, so the chunk's 64 x d K and V tiles are staged in shared memory once
+// per item and shared by up to four 128-row tiles.  One persistent CTA per SM
+// runs a warp-specialised pipeline over its items' tiles:
 //
-//   gather   every thread copies its pair's query row (cp.async, 16 B) into a
-//            128-byte-swizzled K-major tile; the next tile's rows are
-//            prefetched into the other buffer while this one is computed
-//   S = Q K^T   tcgen05.mma, M=128 N=64, f32 in TMEM
-//   softmax  thread t reads TMEM lane t (its pair's 64 logits), masks keys
-//            after the query in the own chunk, writes P (bf16) over the
-//            consumed Q tile
-//   O = P V  tcgen05.mma, M=128 N=d, V read MN-major from the same tile
-//   epilogue O * (w / l) -> bf16 partial, staged in shared memory and written
-//            row-contiguously to partial[pair] (one 2d-byte row per pair)
+//   warps 0-3 (producers)  take items from a global queue; per item copy K
+//       and V into one of two buffers, per tile gather the 128 pairs' query
+//       rows (cp.async, 16 B; warp w the rows 32w ..) into one of NS
+//       128-byte-swizzled K-major stages and publish the tile (rows, causal
+//       key counts) on the stage's barrier.
+//   warp 4 (MMA)  one thread polls the barriers and issues, as soon as each
+//       is ready, S = Q K^T (M=128, N=64) into the TMEM S buffer of the
+//       tile's group, or O = P V (N=d, V read MN-major) of a tile whose
+//       softmax is done.
+//   warps 5-8, 9-12 (two groups, even / odd tiles)  thread t of a group owns
+//       tile row t (TMEM lane t): softmax of its 64 logits, keys after the
+//       query masked in the own chunk, P (bf16) written over the consumed Q
+//       stage; then O / l -> bf16 into the same stage, and one thread writes
+//       the whole tile with a single bulk copy.
 //
-// merge_kernel then sums each query row's k partials in float32 (slot order,
-// deterministic) and writes the output row.  Partials are rounded to bf16 once
-// each, relative to their own (small) magnitude.
+// Partials are stored in bucket order, one row of d bf16 per pair (16-byte
+// chunk c of the row at chunk slot c ^ (position & 7)); merge_kernel then sums
+// each query row's k partials times the fusion weights in float32, slot order
+// (deterministic), and writes the output row.
 #include <cfloat>
 
 #include "hils_common.cuh"
@@ -29,282 +35,405 @@ namespace hils {
 namespace {
 
 constexpr int kRows = 128;          // pairs per MMA tile (M)
-constexpr int kThreads = 128;       // one thread per tile row / TMEM lane
-constexpr uint32_t kTmemCols = 256; // S (64 cols) + O (d cols)
+constexpr int kProducers = 4;       // producer warps
+constexpr int kMmaWarp = kProducers;
+constexpr int kWarps = kProducers + 1 + 8;  // producers, MMA, two groups of four
+constexpr int kThreads = kWarps * 32;
 
 template <int D>
 struct AttnLayout {
+  static constexpr int NS = 4;                          // query stages
   static constexpr uint32_t kQBytes = kRows * D * 2;   // one query tile
   static constexpr uint32_t kKVBytes = kChunk * D * 2; // one K (or V) tile
-  static constexpr uint32_t kQ0 = 0;
-  static constexpr uint32_t kQ1 = kQBytes;
-  static constexpr uint32_t kK = 2 * kQBytes;
-  static constexpr uint32_t kV = kK + kKVBytes;
-  static constexpr uint32_t kEnd = kV + kKVBytes;
-  // + slack for 1024-byte alignment; at least the d=128 footprint so that no more
-  // than two CTAs share an SM (two CTAs x 256 TMEM columns = the SM's 512)
-  static constexpr uint32_t kSmem = (kEnd + 1024 > 99328u) ? kEnd + 1024 : 99328u;
+  static constexpr uint32_t kQ = 0;                    // NS stages
+  static constexpr uint32_t kK = NS * kQBytes;         // two K buffers
+  static constexpr uint32_t kV = kK + 2 * kKVBytes;    // two V buffers
+  static constexpr uint32_t kEnd = kV + 2 * kKVBytes;
+  static constexpr uint32_t kSmem = kEnd + 1024;       // + slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
+  static constexpr uint32_t kTmemS = 0;                // two S buffers of 64 columns
+  static constexpr uint32_t kTmemO = 2 * kChunk;       // two O buffers of D columns
 };
 
-__device__ __forceinline__ int find_key(const int32_t* tile_off, int n_keys, int item) {
-  int lo = 0, hi = n_keys - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (tile_off[mid] <= item) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// Copy one query row (pair id pid, or zeros when pid < 0) into tile buffer q_smem.
-template <int D>
-__device__ __forceinline__ void gather_q_row(const Params& P, uint32_t q_smem, int row, int32_t pid) {
-  const int64_t r = pid >= 0 ? pid / P.k : 0;
-  const uint16_t* src = reinterpret_cast<const uint16_t*>(P.q) + r * D;
-  const uint32_t bytes = pid >= 0 ? 16u : 0u;
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint32_t dst = q_smem + (uint32_t)(c >> 3) * (kRows * 128) + tc::swz(row, c & 7);
-    tc::cp_async16(dst, src + c * 8, bytes);
-  }
-}
+struct TileDesc {
+  int32_t tile_base;  // bucket position of the tile's row 0
+  int32_t n_valid;    // rows in use
+  int32_t kb;         // K/V buffer
+  int32_t kv_phase;   // parity of that buffer's fill
+  int32_t first, last, end;
+};
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(Params P, PrefillWs ws) {
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillWs ws) {
   using Lay = AttnLayout<D>;
+  constexpr int NS = Lay::NS;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_s, bar_o;
+  __shared__ uint64_t q_full[NS], q_empty[NS], kv_full[2], kv_empty[2];
+  __shared__ uint64_t s_full[2], sm_done[2], o_full[2], o_free[2];
+  __shared__ TileDesc desc[NS];
+  __shared__ int32_t meta_r[NS][kRows];   // query row of each tile row (-1: unused)
+  __shared__ uint8_t meta_nk[NS][kRows];  // keys visible to it (64, or fewer in the own chunk)
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int item_sh;
+  __shared__ int item_sh[2];
   __shared__ int abort_sh;
-  __shared__ int32_t pid_sh[kRows];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t sbase = tc::smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    tc::mbar_init(&bar_s, 1);
-    tc::mbar_init(&bar_o, 1);
+    for (int x = 0; x < NS; ++x) {
+      tc::mbar_init(&q_full[x], 64 * kProducers);   // a cp.async and a plain arrival per producer
+      tc::mbar_init(&q_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(&kv_full[x], 32 * kProducers);
+      tc::mbar_init(&kv_empty[x], 1);
+      tc::mbar_init(&s_full[x], 1);
+      tc::mbar_init(&sm_done[x], 128);
+      tc::mbar_init(&o_full[x], 1);
+      tc::mbar_init(&o_free[x], 128);
+    }
     tc::fence_mbar_init();
     abort_sh = 0;
   }
-  if (warp == 0) {
-    tc::tmem_alloc(&tmem_base_sh, kTmemCols);
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(&tmem_base_sh, Lay::kTmemCols);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tmem_s = tmem;          // columns [0, 64)
-  const uint32_t tmem_o = tmem + 64;     // columns [64, 64 + D)
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  constexpr uint32_t kIdS = tc::idesc_bf16(kRows, kChunk, 0);
-  constexpr uint32_t kIdO = tc::idesc_bf16(kRows, D, 1);
-  const float scale_log2 = P.inv_sqrt_d * 1.4426950408889634f;
-
-  uint32_t phase_s = 0, phase_o = 0;
   const int n_items = ws.tile_off[ws.n_keys];
-  int prev_key = -1;
 
-  for (;;) {
-    if (tid == 0) item_sh = atomicAdd(ws.queue, 1);
-    __syncthreads();
-    const int item = item_sh;
-    if (item >= n_items || abort_sh) break;
-    const int key = find_key(ws.tile_off, ws.n_keys, item);
-    const int j = key % P.max_chunks;
-    const int bg = key / P.max_chunks;
-    const int g = bg % P.Hkv, b = bg / P.Hkv;
-    const int p0 = ws.offsets[key] + (item - ws.tile_off[key]) * kItemPairs;
-    const int p1 = min(p0 + kItemPairs, ws.offsets[key + 1]);
-    const int n_tiles = (p1 - p0 + kRows - 1) / kRows;
-
-    // K and V of this chunk (only when the chunk changes)
-    if (key != prev_key) {
-      const int64_t page = page_of(P, b, j);
-      const uint16_t* kp = reinterpret_cast<const uint16_t*>(P.pages) +
-                           (page >= 0 ? page_offset(P, page, 0, g, 0) : 0);
-      const uint16_t* vp = reinterpret_cast<const uint16_t*>(P.pages) +
-                           (page >= 0 ? page_offset(P, page, 1, g, 0) : 0);
-      const uint32_t bytes = page >= 0 ? 16u : 0u;
-      for (int x = tid; x < kChunk * (D / 8); x += kThreads) {
-        const int s = x / (D / 8), c = x % (D / 8);
-        const uint32_t off = (uint32_t)(c >> 3) * (kChunk * 128) + tc::swz(s, c & 7);
-        tc::cp_async16(sbase + Lay::kK + off, kp + s * D + c * 8, bytes);
-        tc::cp_async16(sbase + Lay::kV + off, vp + s * D + c * 8, bytes);
+  if (warp < kProducers) {
+    // --------------------------------------------------------------- producers
+    constexpr int CPR = D / 8;       // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;    // rows per warp-wide copy instruction
+    const int ptid = tid;            // 0 .. 32 * kProducers - 1
+    int n = 0, item_idx = 0;
+    bool ok = true;
+    for (;; ++item_idx) {
+      if (ptid == 0) item_sh[item_idx & 1] = atomicAdd(ws.queue, 1);
+      // every producer thread takes the same decision here
+      if (tc::named_barrier_or(3, 32 * kProducers, !ok || abort_sh != 0)) {
+        ok = false;
+        break;
       }
-      prev_key = key;
-    }
-    // first tile's query rows (pair id and weight of this thread's row are
-    // fetched one tile ahead, so no dependent global load sits on the tile's path)
-    int buf = 0;
-    int32_t pid = p0 + tid < p1 ? ws.pairs[p0 + tid] : -1;
-    gather_q_row<D>(P, sbase + Lay::kQ0, tid, pid);
-    tc::cp_async_commit();
-    float w_next = pid >= 0 ? ws.w[pid] : 0.f;
-
-    for (int t = 0; t < n_tiles; ++t) {
-      const uint32_t q_cur = sbase + (buf ? Lay::kQ1 : Lay::kQ0);
-      const uint32_t q_nxt = sbase + (buf ? Lay::kQ0 : Lay::kQ1);
-      tc::cp_async_wait<0>();
-      tc::fence_proxy_async();
-      tc::tc_fence_before();
-      __syncthreads();
-      // S = Q K^T
-      if (tid == 0) {
-        tc::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(q_cur + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc(sbase + Lay::kK + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem_s, a, bd, kIdS, kk > 0);
-        }
-        tc::mma_commit(&bar_s);
+      const int item = item_sh[item_idx & 1];
+      if (item >= n_items) break;
+      const int key = ws.item_key[item];
+      const int j = key % P.max_chunks;
+      const int bg = key / P.max_chunks / ws.n_win;
+      const int g = bg % P.Hkv, b = bg / P.Hkv;
+      const int p0 = ws.offsets[key] + (item - ws.tile_off[key]) * kItemPairs;
+      const int p1 = min(p0 + kItemPairs, ws.offsets[key + 1]);
+      const int nt = (p1 - p0 + kRows - 1) / kRows;
+      const int kb = item_idx & 1;
+      if (item_idx >= 2 && !tc::mbar_wait(&kv_empty[kb], ((item_idx >> 1) - 1) & 1)) {
+        ok = false;
+        continue;
       }
-      // this thread's pair for the current tile
-      const int32_t my_pid = pid;
-      const float wj = w_next;
-      int nk = kChunk;
-      if (my_pid >= 0) {
-        const int64_t r = my_pid / P.k;
-        const int64_t pos = P.pos0 + (r / P.Hq) % P.L;
-        if (pos / kChunk == j) nk = (int)(pos - (int64_t)j * kChunk + 1);
-      }
-      pid_sh[tid] = my_pid;
-      // prefetch the next tile's query rows into the other buffer
-      if (t + 1 < n_tiles) {
-        const int pn = p0 + (t + 1) * kRows + tid;
-        pid = pn < p1 ? ws.pairs[pn] : -1;
-        gather_q_row<D>(P, q_nxt, tid, pid);
-        tc::cp_async_commit();
-        w_next = pid >= 0 ? ws.w[pid] : 0.f;
-      }
-      if (!tc::mbar_wait(&bar_s, phase_s)) abort_sh = 1;
-      phase_s ^= 1;
-      tc::tc_fence_after();
-      // softmax of this thread's row (TMEM lane tid), P -> bf16 over the Q tile
-      uint32_t sr[64];
       {
-        uint32_t a[32], c[32];
-        tc::tmem_ld32(tmem_s + lane_off, a);
-        tc::tmem_ld32(tmem_s + lane_off + 32, c);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          sr[x] = a[x];
-          sr[32 + x] = c[x];
+        const int64_t page = page_of(P, b, j);
+        const uint16_t* kp = reinterpret_cast<const uint16_t*>(P.pages) +
+                             (page >= 0 ? page_offset(P, page, 0, g, 0) : 0);
+        const uint16_t* vp = reinterpret_cast<const uint16_t*>(P.pages) +
+                             (page >= 0 ? page_offset(P, page, 1, g, 0) : 0);
+        const uint32_t bytes = page >= 0 ? 16u : 0u;
+        const uint32_t kdst = sbase + Lay::kK + kb * Lay::kKVBytes;
+        const uint32_t vdst = sbase + Lay::kV + kb * Lay::kKVBytes;
+        for (int x = ptid; x < kChunk * CPR; x += 32 * kProducers) {
+          const int s = x / CPR, c = x % CPR;
+          const uint32_t off = (uint32_t)(c >> 3) * (kChunk * 128) + tc::swz(s, c & 7);
+          tc::cp_async16(kdst + off, kp + s * D + c * 8, bytes);
+          tc::cp_async16(vdst + off, vp + s * D + c * 8, bytes);
         }
+        tc::cp_async_mbar_arrive(&kv_full[kb]);
       }
-      float m = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < 64; ++x)
-        if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
-      float l = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int x = 0; x < 64; x += 2) {
-        const float e0 = x < nk ? exp2f((__uint_as_float(sr[x]) - m) * scale_log2) : 0.f;
-        const float e1 = x + 1 < nk ? exp2f((__uint_as_float(sr[x + 1]) - m) * scale_log2) : 0.f;
-        const uint32_t pp = tc::pack_bf16x2(e0, e1);
-        pk[x >> 1] = pp;
-        l += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
-      }
-      uint8_t* prow = smem + (q_cur - sbase);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + tc::swz(tid, c)) = v;
-      }
-      tc::fence_proxy_async();
-      tc::tc_fence_before();
-      __syncthreads();
-      // O = P V
-      if (tid == 0) {
-        tc::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(q_cur + kk * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc(sbase + Lay::kV + kk * 2048, kChunk * 128, 1024);
-          tc::mma_bf16(tmem_o, a, bd, kIdO, kk > 0);
+      for (int t = 0; t < nt && ok; ++t, ++n) {
+        const int st = n % NS;
+        if (n >= NS && !tc::mbar_wait(&q_empty[st], ((n / NS) - 1) & 1)) {
+          ok = false;
+          break;
         }
-        tc::mma_commit(&bar_o);
-      }
-      if (!tc::mbar_wait(&bar_o, phase_o)) abort_sh = 1;
-      phase_o ^= 1;
-      tc::tc_fence_after();
-      // epilogue: O * (w / l) -> bf16 row staged over the P/Q tile (16-byte chunk c
-      // of row r at chunk slot c ^ (r & 7): conflict-free), then coalesced stores
-      const float sc = (my_pid >= 0 && l > 0.f) ? wj / l : 0.f;
-      uint8_t* orow = smem + (q_cur - sbase) + tid * (D * 2);
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tc::tmem_ld32(tmem_o + lane_off + c0, o);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            w4[u] = tc::pack_bf16x2(__uint_as_float(o[q4 * 8 + 2 * u]) * sc,
-                                    __uint_as_float(o[q4 * 8 + 2 * u + 1]) * sc);
-          const int c = (c0 >> 3) + q4;
-          *reinterpret_cast<uint4*>(orow + ((c ^ (tid & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
-      // the staged rows are written by whole warps: lane x stores 4-byte word x (+32...)
-      __syncthreads();
-      {
         const int tile_base = p0 + t * kRows;
-        const uint32_t* stg = reinterpret_cast<const uint32_t*>(smem + (q_cur - sbase));
-        for (int rr = warp; rr < kRows; rr += kThreads / 32) {
-          const int pi = tile_base + rr;
-          if (pi >= p1) break;
-          const int32_t rp = pid_sh[rr];
-          uint32_t* dst = reinterpret_cast<uint32_t*>(ws.partial) + (int64_t)rp * (D / 2);
+        const int nv = min(kRows, p1 - tile_base);
+        {
+          const int row = warp * 32 + lane;
+          int32_t r = -1;
+          int nk = kChunk;
+          if (row < nv) {
+            const int32_t pid = ws.pairs[tile_base + row];
+            r = pid / P.k;
+            const int64_t pos = P.pos0 + ((int64_t)r / P.Hq) % P.L;
+            if (pos / kChunk == j) nk = (int)(pos - (int64_t)j * kChunk + 1);
+          }
+          meta_r[st][row] = r;
+          meta_nk[st][row] = (uint8_t)nk;
+        }
+        __syncwarp();
+        const uint32_t qdst = sbase + Lay::kQ + st * Lay::kQBytes;
 #pragma unroll
-          for (int x = tid & 31; x < D / 2; x += 32)
-            dst[x] = stg[rr * (D / 2) + ((((x >> 2) ^ (rr & 7)) << 2) | (x & 3))];
+        for (int it = 0; it < 32 / RPI; ++it) {
+          const int row = warp * 32 + it * RPI + lane / CPR, c = lane % CPR;
+          const int32_t r = meta_r[st][row];
+          const uint16_t* src =
+              reinterpret_cast<const uint16_t*>(P.q) + (int64_t)(r >= 0 ? r : 0) * D + c * 8;
+          tc::cp_async16(qdst + (uint32_t)(c >> 3) * (kRows * 128) + tc::swz(row, c & 7), src,
+                         r >= 0 ? 16u : 0u);
+        }
+        if (ptid == 0) {
+          TileDesc d;
+          d.tile_base = tile_base;
+          d.n_valid = nv;
+          d.kb = kb;
+          d.kv_phase = (item_idx >> 1) & 1;
+          d.first = t == 0;
+          d.last = t == nt - 1;
+          d.end = 0;
+          desc[st] = d;
+        }
+        tc::cp_async_mbar_arrive(&q_full[st]);
+        tc::mbar_arrive(&q_full[st]);
+      }
+    }
+    // two end markers: one for each group
+    for (int e = 0; e < 2 && ok; ++e, ++n) {
+      const int st = n % NS;
+      if (n >= NS && !tc::mbar_wait(&q_empty[st], ((n / NS) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      if (ptid == 0) {
+        TileDesc d{};
+        d.end = 1;
+        desc[st] = d;
+      }
+      tc::cp_async_mbar_arrive(&q_full[st]);
+      tc::mbar_arrive(&q_full[st]);
+    }
+    if (!ok) abort_sh = 1;
+    tc::cp_async_wait<0>();
+  } else if (warp == kMmaWarp) {
+    // -------------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdS = tc::idesc_bf16(kRows, kChunk, 0);
+      constexpr uint32_t kIdO = tc::idesc_bf16(kRows, D, 1);
+      int ns = 0, np = 0;        // next tile to issue S for / P V for
+      bool s_done = false;
+      uint64_t t_idle = 0;
+      uint32_t idle = 0;
+      for (;;) {
+        bool progress = false;
+        // O = P V of tile np once its softmax is done and its O buffer is free
+        if (np < ns) {
+          const int wg = np & 1;
+          if (tc::mbar_try_wait(&sm_done[wg], (np >> 1) & 1) &&
+              (np < 2 || tc::mbar_try_wait(&o_free[wg], ((np >> 1) - 1) & 1))) {
+            tc::tc_fence_after();
+            const TileDesc dm = desc[np % NS];
+            const uint32_t pst = sbase + Lay::kQ + (np % NS) * Lay::kQBytes;
+            const uint32_t vb = sbase + Lay::kV + dm.kb * Lay::kKVBytes;
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk) {
+              const uint64_t a = tc::smem_desc(pst + kk * 32, 16, 1024);
+              const uint64_t bd = tc::smem_desc(vb + kk * 2048, kChunk * 128, 1024);
+              tc::mma_bf16(tmem + Lay::kTmemO + wg * D, a, bd, kIdO, kk > 0);
+            }
+            tc::mma_commit(&o_full[wg]);
+            if (dm.last) tc::mma_commit(&kv_empty[dm.kb]);
+            ++np;
+            progress = true;
+          }
+        }
+        // S = Q K^T of tile ns once it is gathered and its S buffer is free
+        if (!s_done) {
+          const int st = ns % NS, wg = ns & 1;
+          if (tc::mbar_try_wait(&q_full[st], (ns / NS) & 1)) {
+            const TileDesc d = desc[st];
+            if (d.end) {
+              s_done = true;
+            } else if ((!d.first || tc::mbar_try_wait(&kv_full[d.kb], d.kv_phase)) &&
+                       (ns < 2 || tc::mbar_try_wait(&sm_done[wg], ((ns >> 1) - 1) & 1))) {
+              tc::tc_fence_after();
+              const uint32_t qst = sbase + Lay::kQ + st * Lay::kQBytes;
+              const uint32_t kbuf = sbase + Lay::kK + d.kb * Lay::kKVBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::smem_desc(qst + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = tc::smem_desc(kbuf + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
+                tc::mma_bf16(tmem + Lay::kTmemS + wg * kChunk, a, bd, kIdS, kk > 0);
+              }
+              tc::mma_commit(&s_full[wg]);
+              ++ns;
+              progress = true;
+            }
+          }
+        }
+        if (s_done && np == ns) break;
+        if (progress || abort_sh) {
+          idle = 0;
+          if (abort_sh) break;
+        } else if ((++idle & 255u) == 0) {
+          const uint64_t now = tc::globaltimer_ns();
+          if (idle == 256) t_idle = now;
+          else if (now - t_idle > 2000000000ull) {
+            abort_sh = 1;
+            break;
+          }
         }
       }
-      buf ^= 1;
     }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------- softmax + epilogue groups
+    const int wg = (warp - kMmaWarp - 1) >> 2;
+    const int row = ((warp & 3) << 5) + lane;            // TMEM lane of this warp's quarter
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float scale_log2 = P.inv_sqrt_d * 1.4426950408889634f;
+    bool ok = true;
+    for (int n = wg, u = 0;; n += 2, ++u) {
+      const int st = n % NS;
+      bool bad = !tc::warp_wait(&q_full[st], (n / NS) & 1);
+      const TileDesc d = desc[st];
+      // the group leaves together or not at all (its named barrier below)
+      if (tc::named_barrier_or(1 + wg, 128, bad)) {
+        ok = false;
+        break;
+      }
+      if (d.end) break;
+      const int nk = meta_nk[st][row];
+      uint8_t* stage = smem + Lay::kQ + st * Lay::kQBytes;
+      bad = !tc::warp_wait(&s_full[wg], u & 1);
+      float linv = 0.f;
+      if (!bad) {
+        tc::tc_fence_after();
+        uint32_t sr[64];
+        {
+          uint32_t a[32], c[32];
+          tc::tmem_ld32(tmem + lane_off + Lay::kTmemS + wg * kChunk, a);
+          tc::tmem_ld32(tmem + lane_off + Lay::kTmemS + wg * kChunk + 32, c);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            sr[x] = a[x];
+            sr[32 + x] = c[x];
+          }
+        }
+        float m = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
+        float l = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int x = 0; x < 64; x += 2) {
+          const float e0 = x < nk ? exp2f((__uint_as_float(sr[x]) - m) * scale_log2) : 0.f;
+          const float e1 = x + 1 < nk ? exp2f((__uint_as_float(sr[x + 1]) - m) * scale_log2) : 0.f;
+          const uint32_t pp = tc::pack_bf16x2(e0, e1);
+          pk[x >> 1] = pp;
+          l += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(stage + tc::swz(row, c)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        tc::fence_proxy_async();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm_done[wg]);
+        linv = l > 0.f ? 1.f / l : 0.f;
+        bad = !tc::warp_wait(&o_full[wg], u & 1);
+      }
+      if (!bad) {
+        tc::tc_fence_after();
+        // O / l -> bf16, row `row` of the stage, 16-byte chunk c at slot c ^ (position & 7)
+        const int key7 = (d.tile_base + row) & 7;
+        uint8_t* orow = stage + row * (D * 2);
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tc::tmem_ld32(tmem + lane_off + Lay::kTmemO + wg * D + c0, o);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w4[e] = tc::pack_bf16x2(__uint_as_float(o[q4 * 8 + 2 * e]) * linv,
+                                      __uint_as_float(o[q4 * 8 + 2 * e + 1]) * linv);
+            const int c = (c0 >> 3) + q4;
+            *reinterpret_cast<uint4*>(orow + ((c ^ key7) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&o_free[wg]);
+        tc::fence_proxy_async();
+      }
+      if (tc::named_barrier_or(1 + wg, 128, bad || abort_sh != 0)) {
+        ok = false;
+        break;
+      }
+      if (row == 0) {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(ws.partial) + (int64_t)d.tile_base * (D * 2);
+        tc::bulk_s2g(dst, sbase + Lay::kQ + st * Lay::kQBytes, (uint32_t)d.n_valid * (D * 2));
+        tc::bulk_commit();
+        tc::bulk_wait_read();
+        tc::mbar_arrive(&q_empty[st]);
+      }
+    }
+    if (!ok) abort_sh = 1;
+    if (row == 0) tc::bulk_wait_all();
   }
+
   if (abort_sh && tid == 0) set_device_error(kErrTimeout);
-  tc::cp_async_wait<0>();
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tc::tmem_dealloc(tmem, Lay::kTmemCols);
 }
 
-// out[row] = sum over valid slots of partial[row * k + slot]  (float32, slot order)
+// out[row] = sum over valid slots of w[row, slot] * partial[inv[row * k + slot]]
+// (float32, slot order); one warp per row, lane x owns elements x*E .. x*E+E-1.
 template <int D>
-__global__ void merge_kernel(Params P, PrefillWs ws, const int32_t* idx, void* out, int64_t rows) {
+__global__ void merge_kernel(Params P, PrefillWs ws, const int32_t* idx, const float* wts,
+                             void* out, int64_t rows) {
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
   constexpr int E = D / 32;  // elements per lane
+  const int e0 = lane * E;
+  const int c = e0 >> 3, within = e0 & 7;
+  // this row's slots, one per lane
+  int32_t my_pos = -1;
+  float my_w = 0.f;
+  if (lane < P.k && idx[r * P.k + lane] >= 0) {
+    my_pos = ws.inv[r * P.k + lane];
+    my_w = wts[r * P.k + lane];
+  }
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   for (int s = 0; s < P.k; ++s) {
-    if (idx[r * P.k + s] < 0) continue;
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(ws.partial) + (r * P.k + s) * D + lane * E;
+    const int32_t pos = __shfl_sync(0xffffffffu, my_pos, s);
+    const float w = __shfl_sync(0xffffffffu, my_w, s);
+    if (pos < 0) continue;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(ws.partial) + (int64_t)pos * D +
+                          ((c ^ (pos & 7)) << 3) + within;
     if (E == 4) {
       const uint2 v = *reinterpret_cast<const uint2*>(src);
-      acc[0] += __uint_as_float(v.x << 16);
-      acc[1] += __uint_as_float(v.x & 0xFFFF0000u);
-      acc[2] += __uint_as_float(v.y << 16);
-      acc[3] += __uint_as_float(v.y & 0xFFFF0000u);
+      acc[0] = fmaf(w, __uint_as_float(v.x << 16), acc[0]);
+      acc[1] = fmaf(w, __uint_as_float(v.x & 0xFFFF0000u), acc[1]);
+      acc[2] = fmaf(w, __uint_as_float(v.y << 16), acc[2]);
+      acc[3] = fmaf(w, __uint_as_float(v.y & 0xFFFF0000u), acc[3]);
     } else {
       const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
-      acc[0] += __uint_as_float(v << 16);
-      acc[1] += __uint_as_float(v & 0xFFFF0000u);
+      acc[0] = fmaf(w, __uint_as_float(v << 16), acc[0]);
+      acc[1] = fmaf(w, __uint_as_float(v & 0xFFFF0000u), acc[1]);
     }
   }
-  uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * D + lane * E;
+  uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * D + e0;
   if (E == 4) {
     *reinterpret_cast<uint2*>(o) = make_uint2(tc::pack_bf16x2(acc[0], acc[1]),
                                               tc::pack_bf16x2(acc[2], acc[3]));
@@ -314,34 +443,39 @@ __global__ void merge_kernel(Params P, PrefillWs ws, const int32_t* idx, void* o
 }
 
 template <int D>
-cudaError_t run_attn_tc(const Params& P, void* out, const int32_t* idx, const PrefillWs& ws,
-                        cudaStream_t s) {
+cudaError_t run_attn_tc(const Params& P, void* out, const int32_t* idx, const float* w,
+                        const PrefillWs& ws, cudaStream_t s) {
   using Lay = AttnLayout<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Lay::kSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int dev = 0, sms = 148, per_sm = 1;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel<D>, kThreads,
+                                                         Lay::kSmem)) != cudaSuccess)
+    return e;
   if ((e = cudaMemsetAsync(ws.queue, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
   {
     HILS_PROFILE("prefill.attend_tc", s);
-    attn_tc_kernel<D><<<2 * sms, kThreads, Lay::kSmem, s>>>(P, ws);
+    attn_tc_kernel<D><<<sms * max(1, per_sm), kThreads, Lay::kSmem, s>>>(P, ws);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = (int64_t)P.B * P.L * P.Hq;
   {
     HILS_PROFILE("prefill.merge", s);
-    merge_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(P, ws, idx, out, rows);
+    merge_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(P, ws, idx, w, out, rows);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const PrefillWs& ws,
-                           cudaStream_t s) {
-  return P.d == 64 ? run_attn_tc<64>(P, out, idx, ws, s) : run_attn_tc<128>(P, out, idx, ws, s);
+cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const float* w,
+                           const PrefillWs& ws, cudaStream_t s) {
+  return P.d == 64 ? run_attn_tc<64>(P, out, idx, w, ws, s)
+                   : run_attn_tc<128>(P, out, idx, w, ws, s);
 }
 
 }  // namespace hils

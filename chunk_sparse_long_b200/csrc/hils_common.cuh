@@ -148,18 +148,22 @@ cudaError_t launch_topk(const Params& P, const float* scores, int n_cols, int32_
 struct PrefillWs {
   int32_t* idx;      // [rows][k]
   float* w;          // [rows][k]
-  int32_t* counts;   // [n_keys]
+  int32_t* counts;   // [n_keys]; key = ((b * Hkv + g) * n_win + window) * max_chunks + chunk
   int32_t* offsets;  // [n_keys + 1] pair offsets
   int32_t* tile_off; // [n_keys + 1] tile offsets
   int32_t* cursor;   // [n_keys]
-  int32_t* pairs;    // [rows * k] pair ids (row * k + slot)
+  int32_t* pairs;    // [rows * k] pair ids (row * k + slot) in bucket order
+  int32_t* inv;      // [rows * k] bucket position of each pair id
   float* acc;        // [rows][d] float32 accumulator (CUDA-core attention)
-  void* partial;     // [rows * k][d] bf16 per-pair partial outputs (tensor-core attention)
+  void* partial;     // [rows * k][d] bf16 per-pair O / l in bucket order (tensor-core attention)
   int32_t* queue;    // work-item counter of the persistent attention kernel
   void* qimg;        // bf16: per 128-row tile the three q~ term tiles (shared-memory images)
   float* scores;     // bf16: landmark scores, score_cols columns per (sequence, head)
   int64_t score_cols;
+  int32_t* item_key; // [max_tiles] key of every work item
   int n_keys;
+  int n_win;         // query windows per sequence
+  int64_t win_rows;  // query positions per window
   int64_t max_tiles;
 };
 size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base);
@@ -167,8 +171,8 @@ cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* 
                            const PrefillWs& ws, cudaStream_t s);
 cudaError_t launch_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, float* w,
                              cudaStream_t s);
-cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const PrefillWs& ws,
-                           cudaStream_t s);
+cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const float* w,
+                           const PrefillWs& ws, cudaStream_t s);
 
 struct DecodeWs {
   float* cand_s;       // [B][n_split][Hq][k-1] each split's best candidates, best first

@@ -24,6 +24,10 @@ constexpr int kLmTile = 32;
 constexpr int kTilePairs = 128;
 constexpr int kAttThreads = 256;
 constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kBucketWindow = 8192;   // query positions per bucketing window
+constexpr int kBucketRows = 1024;     // query positions per bucketing CTA
+constexpr int kHistMax = 24576;       // chunk bins a bucketing CTA keeps in shared memory
+constexpr int64_t kMaxKeys = 1 << 26; // bucket keys above which windows are dropped
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -150,13 +154,100 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Params P, int32_t* 
 }
 
 // ---- bucketing ------------------------------------------------------------
-__device__ __forceinline__ int64_t pair_key(const Params& P, int64_t r, int32_t j) {
-  const int h = (int)(r % P.Hq);
-  const int b = (int)(r / ((int64_t)P.L * P.Hq));
-  return ((int64_t)b * P.Hkv + h / P.group) * P.max_chunks + j;
+// Keys are (sequence, KV head, query window, chunk): the attention kernels take
+// work items in key order, so the items running at the same time read the
+// query rows of one window of kBucketWindow positions, which stay in L2.
+struct Windows {
+  int n;            // windows per sequence
+  int64_t rows;     // query positions per window (a multiple of kBucketRows)
+};
+
+__device__ __forceinline__ int64_t bucket_key(const Params& P, Windows W, int b, int g, int64_t i,
+                                              int32_t j) {
+  return (((int64_t)b * P.Hkv + g) * W.n + i / W.rows) * P.max_chunks + j;
 }
 
-__global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int64_t n_pairs) {
+// Pair p = row * k + slot of row (b, i, h) -> its key (global-atomic fallback path).
+__device__ __forceinline__ int64_t pair_key(const Params& P, Windows W, int64_t p, int32_t j) {
+  const int64_t r = p / P.k;
+  const int h = (int)(r % P.Hq);
+  const int64_t bi = r / P.Hq;
+  return bucket_key(P, W, (int)(bi / P.L), h / P.group, bi % P.L, j);
+}
+
+// One CTA per (sequence b, KV head g, block of kBucketRows query positions):
+// the block's pairs are counted into a shared-memory histogram over the chunks
+// its rows can see, then added to the global counts once per nonzero bin.
+// Every pair of a position i of the group's heads is one run of group * k
+// consecutive idx entries.
+__device__ __forceinline__ void block_hist(const Params& P, const int32_t* idx, int32_t* hist,
+                                           int nvis, int64_t i0, int64_t i1, int b, int g,
+                                           bool check) {
+  const int per_i = P.group * P.k;
+  const int n = (int)(i1 - i0) * per_i;
+  for (int f = threadIdx.x; f < n; f += blockDim.x) {
+    const int64_t i = i0 + f / per_i;
+    const int32_t j = idx[(((int64_t)b * P.L + i) * P.Hq + g * P.group) * P.k + f % per_i];
+    if (j < 0) continue;
+    if (j >= nvis) {
+      if (check) set_device_error(kErrChunk);
+      continue;
+    }
+    atomicAdd(&hist[j], 1);
+  }
+}
+
+__global__ void __launch_bounds__(256) bucket_count_kernel(Params P, const int32_t* idx,
+                                                           int32_t* counts, Windows W) {
+  extern __shared__ int32_t hist[];
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int64_t i0 = (int64_t)blockIdx.x * kBucketRows, i1 = min(i0 + kBucketRows, P.L);
+  const int nvis = (int)min((int64_t)P.max_chunks, (P.pos0 + i1 - 1) / kChunk + 1);
+  for (int x = threadIdx.x; x < nvis; x += blockDim.x) hist[x] = 0;
+  __syncthreads();
+  block_hist(P, idx, hist, nvis, i0, i1, b, g, true);
+  __syncthreads();
+  const int64_t kb = bucket_key(P, W, b, g, i0, 0);
+  for (int x = threadIdx.x; x < nvis; x += blockDim.x)
+    if (hist[x]) atomicAdd(&counts[kb + x], hist[x]);
+}
+
+// Same blocks: one global atomic per nonzero bin reserves the block's range of
+// each bucket, shared-memory atomics place the pairs inside it.
+__global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int32_t* idx,
+                                                             int32_t* cursor, int32_t* pairs,
+                                                             int32_t* inv, Windows W) {
+  extern __shared__ int32_t hist[];
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int64_t i0 = (int64_t)blockIdx.x * kBucketRows, i1 = min(i0 + kBucketRows, P.L);
+  const int nvis = (int)min((int64_t)P.max_chunks, (P.pos0 + i1 - 1) / kChunk + 1);
+  int32_t* base = hist + nvis;
+  for (int x = threadIdx.x; x < nvis; x += blockDim.x) hist[x] = 0;
+  __syncthreads();
+  block_hist(P, idx, hist, nvis, i0, i1, b, g, false);
+  __syncthreads();
+  const int64_t kb = bucket_key(P, W, b, g, i0, 0);
+  for (int x = threadIdx.x; x < nvis; x += blockDim.x) {
+    const int32_t c = hist[x];
+    base[x] = c ? atomicAdd(&cursor[kb + x], c) : 0;
+    hist[x] = 0;
+  }
+  __syncthreads();
+  const int per_i = P.group * P.k;
+  const int n = (int)(i1 - i0) * per_i;
+  for (int f = threadIdx.x; f < n; f += blockDim.x) {
+    const int64_t p = (((int64_t)b * P.L + i0 + f / per_i) * P.Hq + g * P.group) * P.k + f % per_i;
+    const int32_t j = idx[p];
+    if (j < 0 || j >= nvis) continue;
+    const int32_t at = base[j] + atomicAdd(&hist[j], 1);
+    pairs[at] = (int32_t)p;
+    inv[p] = at;
+  }
+}
+
+// Fallback when a block's visible chunks do not fit in shared memory.
+__global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int64_t n_pairs,
+                             Windows W) {
   const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= n_pairs) return;
   const int32_t j = idx[p];
@@ -165,12 +256,26 @@ __global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int6
     set_device_error(kErrChunk);
     return;
   }
-  atomicAdd(&counts[pair_key(P, p / P.k, j)], 1);
+  atomicAdd(&counts[pair_key(P, W, p, j)], 1);
 }
 
+__global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, int32_t* pairs,
+                               int32_t* inv, int64_t n_pairs, Windows W) {
+  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n_pairs) return;
+  const int32_t j = idx[p];
+  if (j < 0 || j >= P.max_chunks) return;
+  const int32_t at = atomicAdd(&cursor[pair_key(P, W, p, j)], 1);
+  pairs[at] = (int32_t)p;
+  inv[p] = at;
+}
+
+// Exclusive scans of the bucket sizes (pair offsets) and of their work items
+// (ceil(count / tile_pairs) each), and the key of every work item.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n_keys,
                                                     int tile_pairs, int32_t* offsets,
-                                                    int32_t* tile_off, int32_t* cursor) {
+                                                    int32_t* tile_off, int32_t* cursor,
+                                                    int32_t* item_key) {
   __shared__ int32_t sp[1024], stl[1024];
   const int t = threadIdx.x;
   const int per = (n_keys + 1023) / 1024;
@@ -192,26 +297,19 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n
   }
   int32_t po = sp[t] - ps, to = stl[t] - ts;
   for (int key = k0; key < k1; ++key) {
+    const int32_t c = counts[key];
+    const int32_t nt = (c + tile_pairs - 1) / tile_pairs;
     offsets[key] = po;
     cursor[key] = po;
     tile_off[key] = to;
-    po += counts[key];
-    to += (counts[key] + tile_pairs - 1) / tile_pairs;
+    for (int u = 0; u < nt; ++u) item_key[to + u] = key;
+    po += c;
+    to += nt;
   }
   if (t == 1023) {
     offsets[n_keys] = sp[1023];
     tile_off[n_keys] = stl[1023];
   }
-}
-
-__global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, int32_t* pairs,
-                               int64_t n_pairs) {
-  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (p >= n_pairs) return;
-  const int32_t j = idx[p];
-  if (j < 0 || j >= P.max_chunks) return;
-  const int32_t at = atomicAdd(&cursor[pair_key(P, p / P.k, j)], 1);
-  pairs[at] = (int32_t)p;
 }
 
 // ---- attention over key-major tiles ------------------------------------
@@ -225,14 +323,9 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(Params P, PrefillWs
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x;
   if (tile >= ws.tile_off[ws.n_keys]) return;
-  int lo = 0, hi = ws.n_keys - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (ws.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int key = lo;
+  const int key = ws.item_key[tile];
   const int j = key % P.max_chunks;
-  const int bg = key / P.max_chunks;
+  const int bg = key / P.max_chunks / ws.n_win;
   const int g = bg % P.Hkv, b = bg / P.Hkv;
   const int64_t page = page_of(P, b, j);
   if (page < 0) return;
@@ -324,18 +417,38 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
   }
   // bucket by (sequence, KV head, chunk)
   if ((e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ws.n_keys, s)) != cudaSuccess) return e;
-  const unsigned pb = (unsigned)((n_pairs + 255) / 256);
   {
     HILS_PROFILE("prefill.bucket", s);
-    count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs);
     const int tile_pairs = P.dtype == HILS_BF16 ? kItemPairs : kTilePairs;
-    scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
-                                   ws.cursor);
-    scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, n_pairs);
+    const int64_t nvis_max = min((int64_t)P.max_chunks, (P.pos0 + P.L - 1) / kChunk + 1);
+    const size_t hsm = sizeof(int32_t) * 2 * (size_t)nvis_max;
+    if (nvis_max <= kHistMax) {
+      if ((e = cudaFuncSetAttribute(bucket_scatter_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm)) !=
+          cudaSuccess)
+        return e;
+      if ((e = cudaFuncSetAttribute(bucket_count_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm)) !=
+          cudaSuccess)
+        return e;
+      const dim3 bgrid((unsigned)((P.L + kBucketRows - 1) / kBucketRows), P.Hkv, P.B);
+      const Windows W{ws.n_win, ws.win_rows};
+      bucket_count_kernel<<<bgrid, 256, hsm / 2, s>>>(P, ws.idx, ws.counts, W);
+      scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
+                                     ws.cursor, ws.item_key);
+      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, W);
+    } else {
+      const unsigned pb = (unsigned)((n_pairs + 255) / 256);
+      const Windows W{ws.n_win, ws.win_rows};
+      count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs, W);
+      scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
+                                     ws.cursor, ws.item_key);
+      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, n_pairs, W);
+    }
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // a5 + a6
-  if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws.idx, ws, s);
+  if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws.idx, ws.w, ws, s);
   if ((e = cudaMemsetAsync(ws.acc, 0, sizeof(float) * rows * D, s)) != cudaSuccess) return e;
   constexpr size_t asm_ = attend_smem<D>();
   e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -362,7 +475,14 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   const int64_t rows = (int64_t)P.B * P.L * P.Hq;
   const int64_t n_pairs = rows * P.k;
-  const int64_t n_keys = (int64_t)P.B * P.Hkv * P.max_chunks;
+  // query windows, unless the key space would grow past kMaxKeys
+  int n_win = (int)((P.L + kBucketWindow - 1) / kBucketWindow);
+  int64_t win_rows = kBucketWindow;
+  if ((int64_t)P.B * P.Hkv * n_win * P.max_chunks > kMaxKeys) {
+    n_win = 1;
+    win_rows = P.L > 0 ? P.L : 1;
+  }
+  const int64_t n_keys = (int64_t)P.B * P.Hkv * n_win * P.max_chunks;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
@@ -377,6 +497,7 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
   w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  w.inv = (int32_t*)take(sizeof(int32_t) * n_pairs);
   if (P.dtype == HILS_BF16) {
     // the landmark scores and q~ images are dead before the attention writes
     // its partials, so all three share one region
@@ -399,7 +520,10 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   }
   w.queue = (int32_t*)take(sizeof(int32_t));
   w.n_keys = (int)n_keys;
+  w.n_win = n_win;
+  w.win_rows = win_rows;
   w.max_tiles = (n_pairs + kTilePairs - 1) / kTilePairs + n_keys;
+  w.item_key = (int32_t*)take(sizeof(int32_t) * w.max_tiles);
   if (ws) *ws = w;
   return off;
 }

@@ -55,7 +55,9 @@ struct ScoreLayout {
 
 // ---- a1: calibration ------------------------------------------------------
 // RP = calibration rank rounded up (A staged as [D][RP] with zero columns).
-template <int D, int RP>
+// Each thread computes NR rows (row tid of NR consecutive tiles), so every
+// 16-byte broadcast load of A or B feeds NR x 4 FMAs.
+template <int D, int RP, int NR>
 __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, int T,
                                                       int64_t n_tiles) {
   using Lay = ScoreLayout<D>;
@@ -70,82 +72,107 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
   for (int x = tid; x < RP * D; x += kThrS) sB[x] = x < P.r * D ? P.Bm[x] : 0.f;
   __syncthreads();
 
-  for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x) {
-    const int t = (int)(g % T);
-    const int64_t bh = g / T;
-    const int h = (int)(bh % P.Hq), b = (int)(bh / P.Hq);
-    const int64_t i = (int64_t)t * kRowsS + tid;
-    const bool valid = i < P.L;
-    const int64_t qoff = (((int64_t)b * P.L + (valid ? i : 0)) * P.Hq + h) * D;
+  const int64_t n_groups = (n_tiles + NR - 1) / NR;
+  for (int64_t gg = blockIdx.x; gg < n_groups; gg += gridDim.x) {
+    int64_t qoff[NR];
+    bool valid[NR];
+#pragma unroll
+    for (int v = 0; v < NR; ++v) {
+      const int64_t g = gg * NR + v;
+      const int t = (int)(g % T);
+      const int64_t bh = g / T;
+      const int h = (int)(bh % P.Hq), b = (int)(bh / P.Hq);
+      const int64_t i = (int64_t)t * kRowsS + tid;
+      valid[v] = g < n_tiles && i < P.L;
+      qoff[v] = valid[v] ? (((int64_t)b * P.L + i) * P.Hq + h) * D : 0;
+    }
     // t = q A: one accumulator chain per rank column, summed over e in order
-    float ta[RP];
+    float ta[NR][RP];
 #pragma unroll
-    for (int a = 0; a < RP; ++a) ta[a] = 0.f;
+    for (int v = 0; v < NR; ++v)
+#pragma unroll
+      for (int a = 0; a < RP; ++a) ta[v][a] = 0.f;
     if (P.r > 0) {
-#pragma unroll 2
+#pragma unroll 1
       for (int e0 = 0; e0 < D; e0 += 8) {
-        float qv[8];
-        if (valid) {
-          load8(P.q, HILS_BF16, qoff + e0, qv);
-        } else {
+        float qv[NR][8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) qv[u] = 0.f;
+        for (int v = 0; v < NR; ++v) {
+          if (valid[v]) {
+            load8(P.q, HILS_BF16, qoff[v] + e0, qv[v]);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) qv[v][u] = 0.f;
+          }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
 #pragma unroll
           for (int a = 0; a < RP; a += 4) {
             const float4 av = *reinterpret_cast<const float4*>(sA + (e0 + u) * RP + a);
-            ta[a] = fmaf(qv[u], av.x, ta[a]);
-            ta[a + 1] = fmaf(qv[u], av.y, ta[a + 1]);
-            ta[a + 2] = fmaf(qv[u], av.z, ta[a + 2]);
-            ta[a + 3] = fmaf(qv[u], av.w, ta[a + 3]);
+#pragma unroll
+            for (int v = 0; v < NR; ++v) {
+              ta[v][a] = fmaf(qv[v][u], av.x, ta[v][a]);
+              ta[v][a + 1] = fmaf(qv[v][u], av.y, ta[v][a + 1]);
+              ta[v][a + 2] = fmaf(qv[v][u], av.z, ta[v][a + 2]);
+              ta[v][a + 3] = fmaf(qv[v][u], av.w, ta[v][a + 3]);
+            }
           }
         }
       }
     }
     // q~ = q + t B (a ascending), then the three-term split, 8 elements at a time
-    uint8_t* img = qimg + g * Lay::kQimg;
 #pragma unroll 1
     for (int c = 0; c < D / 8; ++c) {
-      float x[8];
-      if (valid) {
-        load8(P.q, HILS_BF16, qoff + c * 8, x);
-      } else {
+      float x[NR][8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = 0.f;
+      for (int v = 0; v < NR; ++v) {
+        if (valid[v]) {
+          load8(P.q, HILS_BF16, qoff[v] + c * 8, x[v]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[v][u] = 0.f;
+        }
       }
 #pragma unroll
       for (int a = 0; a < RP; ++a) {
         if (a < P.r) {
           const float4 b0 = *reinterpret_cast<const float4*>(sB + a * D + c * 8);
           const float4 b1 = *reinterpret_cast<const float4*>(sB + a * D + c * 8 + 4);
-          x[0] = fmaf(ta[a], b0.x, x[0]);
-          x[1] = fmaf(ta[a], b0.y, x[1]);
-          x[2] = fmaf(ta[a], b0.z, x[2]);
-          x[3] = fmaf(ta[a], b0.w, x[3]);
-          x[4] = fmaf(ta[a], b1.x, x[4]);
-          x[5] = fmaf(ta[a], b1.y, x[5]);
-          x[6] = fmaf(ta[a], b1.z, x[6]);
-          x[7] = fmaf(ta[a], b1.w, x[7]);
+#pragma unroll
+          for (int v = 0; v < NR; ++v) {
+            x[v][0] = fmaf(ta[v][a], b0.x, x[v][0]);
+            x[v][1] = fmaf(ta[v][a], b0.y, x[v][1]);
+            x[v][2] = fmaf(ta[v][a], b0.z, x[v][2]);
+            x[v][3] = fmaf(ta[v][a], b0.w, x[v][3]);
+            x[v][4] = fmaf(ta[v][a], b1.x, x[v][4]);
+            x[v][5] = fmaf(ta[v][a], b1.y, x[v][5]);
+            x[v][6] = fmaf(ta[v][a], b1.z, x[v][6]);
+            x[v][7] = fmaf(ta[v][a], b1.w, x[v][7]);
+          }
         }
       }
-      uint32_t hw[4], mw[4], lw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float x0 = x[2 * u], x1 = x[2 * u + 1];
-        hw[u] = tc::pack_bf16x2(x0, x1);
-        x0 -= __uint_as_float(hw[u] << 16);
-        x1 -= __uint_as_float(hw[u] & 0xFFFF0000u);
-        mw[u] = tc::pack_bf16x2(x0, x1);
-        x0 -= __uint_as_float(mw[u] << 16);
-        x1 -= __uint_as_float(mw[u] & 0xFFFF0000u);
-        lw[u] = tc::pack_bf16x2(x0, x1);
-      }
       const uint32_t off = (uint32_t)(c >> 3) * (kRowsS * 128) + tc::swz(tid, c & 7);
-      *reinterpret_cast<uint4*>(img + 0 * Lay::kQt + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(img + 1 * Lay::kQt + off) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
-      *reinterpret_cast<uint4*>(img + 2 * Lay::kQt + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+#pragma unroll
+      for (int v = 0; v < NR; ++v) {
+        if (gg * NR + v >= n_tiles) continue;
+        uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float x0 = x[v][2 * u], x1 = x[v][2 * u + 1];
+          hw[u] = tc::pack_bf16x2(x0, x1);
+          x0 -= __uint_as_float(hw[u] << 16);
+          x1 -= __uint_as_float(hw[u] & 0xFFFF0000u);
+          mw[u] = tc::pack_bf16x2(x0, x1);
+          x0 -= __uint_as_float(mw[u] << 16);
+          x1 -= __uint_as_float(mw[u] & 0xFFFF0000u);
+          lw[u] = tc::pack_bf16x2(x0, x1);
+        }
+        uint8_t* img = qimg + (gg * NR + v) * Lay::kQimg;
+        *reinterpret_cast<uint4*>(img + 0 * Lay::kQt + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(img + 1 * Lay::kQt + off) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+        *reinterpret_cast<uint4*>(img + 2 * Lay::kQt + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
     }
   }
 }
@@ -395,7 +422,7 @@ __device__ __forceinline__ float pick32(const float (&v)[32], int x) {
   return (x & 1) ? a[1] : a[0];
 }
 
-__global__ void __launch_bounds__(kThrS) select_kernel(Params P, const float* scores, int T,
+__global__ void __launch_bounds__(kThrS, 6) select_kernel(Params P, const float* scores, int T,
                                                        int64_t cols_per_head, int32_t* idx,
                                                        float* w) {
   extern __shared__ uint64_t heap_sh[];   // [k-1][kThrS]
@@ -476,16 +503,17 @@ __global__ void __launch_bounds__(kThrS) select_kernel(Params P, const float* sc
 template <int D, int RP>
 cudaError_t run_calib(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, int n_sm,
                       cudaStream_t s) {
+  constexpr int NR = RP <= 32 ? 2 : 1;
   const size_t sm = sizeof(float) * 2 * D * RP;
-  cudaError_t e = cudaFuncSetAttribute(calib_kernel<D, RP>,
+  cudaError_t e = cudaFuncSetAttribute(calib_kernel<D, RP, NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_kernel<D, RP>, kThrS, sm);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_kernel<D, RP, NR>, kThrS, sm);
   if (e != cudaSuccess) return e;
-  const int64_t grid = min(n_tiles, (int64_t)n_sm * max(1, per_sm));
+  const int64_t grid = min((n_tiles + NR - 1) / NR, (int64_t)n_sm * max(1, per_sm));
   HILS_PROFILE("prefill.calib", s);
-  calib_kernel<D, RP><<<(unsigned)grid, kThrS, sm, s>>>(P, qimg, T, n_tiles);
+  calib_kernel<D, RP, NR><<<(unsigned)grid, kThrS, sm, s>>>(P, qimg, T, n_tiles);
   return cudaGetLastError();
 }
 

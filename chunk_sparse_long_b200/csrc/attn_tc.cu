@@ -7,15 +7,17 @@
 // per item and shared by up to four 128-row tiles.  One persistent CTA per SM
 // runs a warp-specialised pipeline over its items' tiles:
 //
-//   warps 0-3 (producers)  take items from a global queue; per item copy K
+//   warps 0-3 (producers)  take items in a fixed order; per item copy K
 //       and V into one of two buffers, per tile gather the 128 pairs' query
 //       rows (cp.async, 16 B; warp w the rows 32w ..) into one of NS
 //       128-byte-swizzled K-major stages and publish the tile (rows, causal
 //       key counts) on the stage's barrier.
 //   warp 4 (MMA)  one thread polls the barriers and issues, as soon as each
 //       is ready, S = Q K^T (M=128, N=64) into the TMEM S buffer of the
-//       tile's group, or O = P V (N=d, V read MN-major) of a tile whose
-//       softmax is done.
+//       tile's group, or O = P V of a tile whose softmax is done.  V is read
+//       MN-major with one extra 64-column block whose first column is all
+//       ones (N = d + 16), so column d of O is l = sum of the bf16 P row,
+//       summed by the tensor core in float32.
 //   warps 5-8, 9-12 (two groups, even / odd tiles)  thread t of a group owns
 //       tile row t (TMEM lane t): softmax of its 64 logits, keys after the
 //       query masked in the own chunk, P (bf16) written over the consumed Q
@@ -45,14 +47,17 @@ struct AttnLayout {
   static constexpr int NS = 4;                          // query stages
   static constexpr uint32_t kQBytes = kRows * D * 2;   // one query tile
   static constexpr uint32_t kKVBytes = kChunk * D * 2; // one K (or V) tile
+  static constexpr uint32_t kBlkBytes = kChunk * 128;  // one 64-column block of a K/V tile
+  static constexpr uint32_t kVBuf = kKVBytes + kBlkBytes;  // V tile + the ones block
   static constexpr uint32_t kQ = 0;                    // NS stages
   static constexpr uint32_t kK = NS * kQBytes;         // two K buffers
-  static constexpr uint32_t kV = kK + 2 * kKVBytes;    // two V buffers
-  static constexpr uint32_t kEnd = kV + 2 * kKVBytes;
+  static constexpr uint32_t kV = kK + 2 * kKVBytes;    // two V buffers (+ ones blocks)
+  static constexpr uint32_t kEnd = kV + 2 * kVBuf;
   static constexpr uint32_t kSmem = kEnd + 1024;       // + slack for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
+  static constexpr int kNO = D + 16;                   // O columns: d values and l
+  static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS = 0;                // two S buffers of 64 columns
-  static constexpr uint32_t kTmemO = 2 * kChunk;       // two O buffers of D columns
+  static constexpr uint32_t kTmemO = 2 * kChunk;       // two O buffers of kNO columns
 };
 
 struct TileDesc {
@@ -74,7 +79,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
   __shared__ int32_t meta_r[NS][kRows];   // query row of each tile row (-1: unused)
   __shared__ uint8_t meta_nk[NS][kRows];  // keys visible to it (64, or fewer in the own chunk)
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int item_sh[2];
   __shared__ int abort_sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -101,6 +105,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
     tc::tmem_alloc(&tmem_base_sh, Lay::kTmemCols);
     tc::tmem_relinquish();
   }
+  // the ones block after each V tile: element 0 of every key row is 1.0 (bf16)
+  for (int x = tid; x < 2 * (int)Lay::kBlkBytes / 16; x += kThreads) {
+    const int buf = x / (Lay::kBlkBytes / 16), y = x % (Lay::kBlkBytes / 16);
+    const int s = y >> 3, c = y & 7;
+    uint8_t* blk = smem + Lay::kV + buf * Lay::kVBuf + Lay::kKVBytes;
+    *reinterpret_cast<uint4*>(blk + tc::swz(s, c)) = make_uint4(c == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+  }
+  tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -109,26 +121,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
 
   if (warp < kProducers) {
     // --------------------------------------------------------------- producers
+    // Items are taken in a fixed order (blockIdx.x, + gridDim.x, ...), so the
+    // dependent loads are issued ahead of their use: the (key, pair range) of
+    // the item after next, the page of the next item's chunk, and the pair id
+    // of this thread's row in the next tile.
     constexpr int CPR = D / 8;       // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;    // rows per warp-wide copy instruction
     const int ptid = tid;            // 0 .. 32 * kProducers - 1
-    int n = 0, item_idx = 0;
+    const int my_row = warp * 32 + lane;
+    const int stride = gridDim.x;
+    auto item_info = [&](int it) {
+      return it < n_items ? ws.items[it] : make_int4(0, 0, 0, 0);
+    };
+    // block-table entry of the chunk of item `it` (raw; checked when used)
+    auto raw_page = [&](int it, const int4& inf) -> int32_t {
+      if (it >= n_items) return -1;
+      const int j = inf.x % P.max_chunks;
+      const int b = inf.x / P.max_chunks / ws.n_win / P.Hkv;
+      return P.block_table[(int64_t)b * P.max_chunks + j];
+    };
+    int item = blockIdx.x;
+    int4 info = item_info(item);
+    int4 info_next = item_info(item + stride);
+    int32_t page_raw = raw_page(item, info);
+    int32_t pid_next = (item < n_items && info.y + my_row < info.z) ? ws.pairs[info.y + my_row] : -1;
+    int n = 0;
     bool ok = true;
-    for (;; ++item_idx) {
-      if (ptid == 0) item_sh[item_idx & 1] = atomicAdd(ws.queue, 1);
+    for (int item_idx = 0;; ++item_idx) {
       // every producer thread takes the same decision here
       if (tc::named_barrier_or(3, 32 * kProducers, !ok || abort_sh != 0)) {
         ok = false;
         break;
       }
-      const int item = item_sh[item_idx & 1];
       if (item >= n_items) break;
-      const int key = ws.item_key[item];
+      const int next_item = item + stride;
+      const int4 info_after = item_info(next_item + stride);
+      const int32_t page_raw_next = raw_page(next_item, info_next);
+      const int key = info.x;
       const int j = key % P.max_chunks;
       const int bg = key / P.max_chunks / ws.n_win;
-      const int g = bg % P.Hkv, b = bg / P.Hkv;
-      const int p0 = ws.offsets[key] + (item - ws.tile_off[key]) * kItemPairs;
-      const int p1 = min(p0 + kItemPairs, ws.offsets[key + 1]);
+      const int g = bg % P.Hkv;
+      const int p0 = info.y, p1 = info.z;
       const int nt = (p1 - p0 + kRows - 1) / kRows;
       const int kb = item_idx & 1;
       if (item_idx >= 2 && !tc::mbar_wait(&kv_empty[kb], ((item_idx >> 1) - 1) & 1)) {
@@ -136,14 +169,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         continue;
       }
       {
-        const int64_t page = page_of(P, b, j);
+        int64_t page = page_raw;
+        if (page < 0 || page >= P.num_pages) {
+          set_device_error(kErrPage);
+          page = -1;
+        }
         const uint16_t* kp = reinterpret_cast<const uint16_t*>(P.pages) +
                              (page >= 0 ? page_offset(P, page, 0, g, 0) : 0);
         const uint16_t* vp = reinterpret_cast<const uint16_t*>(P.pages) +
                              (page >= 0 ? page_offset(P, page, 1, g, 0) : 0);
         const uint32_t bytes = page >= 0 ? 16u : 0u;
         const uint32_t kdst = sbase + Lay::kK + kb * Lay::kKVBytes;
-        const uint32_t vdst = sbase + Lay::kV + kb * Lay::kKVBytes;
+        const uint32_t vdst = sbase + Lay::kV + kb * Lay::kVBuf;
         for (int x = ptid; x < kChunk * CPR; x += 32 * kProducers) {
           const int s = x / CPR, c = x % CPR;
           const uint32_t off = (uint32_t)(c >> 3) * (kChunk * 128) + tc::swz(s, c & 7);
@@ -160,18 +197,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         }
         const int tile_base = p0 + t * kRows;
         const int nv = min(kRows, p1 - tile_base);
+        const int32_t pid = pid_next;
+        // this row's pair in the next tile: of this item, or the first tile of the next
         {
-          const int row = warp * 32 + lane;
+          int pn, pend;
+          if (t + 1 < nt) {
+            pn = tile_base + kRows + my_row;
+            pend = p1;
+          } else {
+            pn = info_next.y + my_row;
+            pend = next_item < n_items ? info_next.z : 0;
+          }
+          pid_next = pn < pend ? ws.pairs[pn] : -1;
+        }
+        {
           int32_t r = -1;
           int nk = kChunk;
-          if (row < nv) {
-            const int32_t pid = ws.pairs[tile_base + row];
+          if (pid >= 0) {
             r = pid / P.k;
             const int64_t pos = P.pos0 + ((int64_t)r / P.Hq) % P.L;
             if (pos / kChunk == j) nk = (int)(pos - (int64_t)j * kChunk + 1);
           }
-          meta_r[st][row] = r;
-          meta_nk[st][row] = (uint8_t)nk;
+          meta_r[st][my_row] = r;
+          meta_nk[st][my_row] = (uint8_t)nk;
         }
         __syncwarp();
         const uint32_t qdst = sbase + Lay::kQ + st * Lay::kQBytes;
@@ -198,6 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         tc::cp_async_mbar_arrive(&q_full[st]);
         tc::mbar_arrive(&q_full[st]);
       }
+      item = next_item;
+      info = info_next;
+      info_next = info_after;
+      page_raw = page_raw_next;
     }
     // two end markers: one for each group
     for (int e = 0; e < 2 && ok; ++e, ++n) {
@@ -220,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
     // -------------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_bf16(kRows, kChunk, 0);
-      constexpr uint32_t kIdO = tc::idesc_bf16(kRows, D, 1);
+      constexpr uint32_t kIdO = tc::idesc_bf16(kRows, Lay::kNO, 1);
       int ns = 0, np = 0;        // next tile to issue S for / P V for
       bool s_done = false;
       uint64_t t_idle = 0;
@@ -235,12 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
             tc::tc_fence_after();
             const TileDesc dm = desc[np % NS];
             const uint32_t pst = sbase + Lay::kQ + (np % NS) * Lay::kQBytes;
-            const uint32_t vb = sbase + Lay::kV + dm.kb * Lay::kKVBytes;
+            const uint32_t vb = sbase + Lay::kV + dm.kb * Lay::kVBuf;
 #pragma unroll
             for (int kk = 0; kk < kChunk / 16; ++kk) {
               const uint64_t a = tc::smem_desc(pst + kk * 32, 16, 1024);
               const uint64_t bd = tc::smem_desc(vb + kk * 2048, kChunk * 128, 1024);
-              tc::mma_bf16(tmem + Lay::kTmemO + wg * D, a, bd, kIdO, kk > 0);
+              tc::mma_bf16(tmem + Lay::kTmemO + wg * Lay::kNO, a, bd, kIdO, kk > 0);
             }
             tc::mma_commit(&o_full[wg]);
             if (dm.last) tc::mma_commit(&kv_empty[dm.kb]);
@@ -307,7 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
       const int nk = meta_nk[st][row];
       uint8_t* stage = smem + Lay::kQ + st * Lay::kQBytes;
       bad = !tc::warp_wait(&s_full[wg], u & 1);
-      float linv = 0.f;
       if (!bad) {
         tc::tc_fence_after();
         uint32_t sr[64];
@@ -322,19 +373,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
             sr[32 + x] = c[x];
           }
         }
+        // keys after the query exist only in the own chunk: a warp-uniform branch
+        const bool masked = !__all_sync(0xffffffffu, nk == kChunk);
         float m = -INFINITY;
+        if (!masked) {
 #pragma unroll
-        for (int x = 0; x < 64; ++x)
-          if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
-        float l = 0.f;
+          for (int x = 0; x < 64; ++x) m = fmaxf(m, __uint_as_float(sr[x]));
+        } else {
+#pragma unroll
+          for (int x = 0; x < 64; ++x)
+            if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
+        }
+        const float mb = m * scale_log2;
         uint32_t pk[32];
+        if (!masked) {
 #pragma unroll
-        for (int x = 0; x < 64; x += 2) {
-          const float e0 = x < nk ? exp2f((__uint_as_float(sr[x]) - m) * scale_log2) : 0.f;
-          const float e1 = x + 1 < nk ? exp2f((__uint_as_float(sr[x + 1]) - m) * scale_log2) : 0.f;
-          const uint32_t pp = tc::pack_bf16x2(e0, e1);
-          pk[x >> 1] = pp;
-          l += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
+          for (int x = 0; x < 64; x += 2)
+            pk[x >> 1] = tc::pack_bf16x2(
+                tc::ex2_approx(fmaf(__uint_as_float(sr[x]), scale_log2, -mb)),
+                tc::ex2_approx(fmaf(__uint_as_float(sr[x + 1]), scale_log2, -mb)));
+        } else {
+#pragma unroll
+          for (int x = 0; x < 64; x += 2)
+            pk[x >> 1] = tc::pack_bf16x2(
+                x < nk ? tc::ex2_approx(fmaf(__uint_as_float(sr[x]), scale_log2, -mb)) : 0.f,
+                x + 1 < nk ? tc::ex2_approx(fmaf(__uint_as_float(sr[x + 1]), scale_log2, -mb))
+                           : 0.f);
         }
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -343,18 +407,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         tc::fence_proxy_async();
         tc::tc_fence_before();
         tc::mbar_arrive(&sm_done[wg]);
-        linv = l > 0.f ? 1.f / l : 0.f;
         bad = !tc::warp_wait(&o_full[wg], u & 1);
       }
       if (!bad) {
         tc::tc_fence_after();
+        // l = column d of O (the ones block)
+        float linv;
+        {
+          uint32_t lv[16];
+          tc::tmem_ld16(tmem + lane_off + Lay::kTmemO + wg * Lay::kNO + D, lv);
+          tc::tmem_ld_wait();
+          const float l = __uint_as_float(lv[0]);
+          linv = l > 0.f ? 1.f / l : 0.f;
+        }
         // O / l -> bf16, row `row` of the stage, 16-byte chunk c at slot c ^ (position & 7)
         const int key7 = (d.tile_base + row) & 7;
         uint8_t* orow = stage + row * (D * 2);
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
-          tc::tmem_ld32(tmem + lane_off + Lay::kTmemO + wg * D + c0, o);
+          tc::tmem_ld32(tmem + lane_off + Lay::kTmemO + wg * Lay::kNO + c0, o);
           tc::tmem_ld_wait();
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -456,7 +528,6 @@ cudaError_t run_attn_tc(const Params& P, void* out, const int32_t* idx, const fl
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel<D>, kThreads,
                                                          Lay::kSmem)) != cudaSuccess)
     return e;
-  if ((e = cudaMemsetAsync(ws.queue, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
   {
     HILS_PROFILE("prefill.attend_tc", s);
     attn_tc_kernel<D><<<sms * max(1, per_sm), kThreads, Lay::kSmem, s>>>(P, ws);

@@ -160,7 +160,7 @@ struct PrefillWs {
   void* qimg;        // bf16: per 128-row tile the three q~ term tiles (shared-memory images)
   float* scores;     // bf16: landmark scores, score_cols columns per (sequence, head)
   int64_t score_cols;
-  int32_t* item_key; // [max_tiles] key of every work item
+  int4* items;       // [max_tiles] (key, first pair, end pair, 0) of every work item
   int n_keys;
   int n_win;         // query windows per sequence
   int64_t win_rows;  // query positions per window

@@ -25,7 +25,7 @@ constexpr int kTilePairs = 128;
 constexpr int kAttThreads = 256;
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kBucketWindow = 8192;   // query positions per bucketing window
-constexpr int kBucketRows = 1024;     // query positions per bucketing CTA
+constexpr int kBucketRows = 256;      // query positions per bucketing CTA
 constexpr int kHistMax = 24576;       // chunk bins a bucketing CTA keeps in shared memory
 constexpr int64_t kMaxKeys = 1 << 26; // bucket keys above which windows are dropped
 
@@ -271,11 +271,12 @@ __global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, in
 }
 
 // Exclusive scans of the bucket sizes (pair offsets) and of their work items
-// (ceil(count / tile_pairs) each), and the key of every work item.
+// (ceil(count / tile_pairs) each), and (key, first pair, end pair) of every
+// work item.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n_keys,
                                                     int tile_pairs, int32_t* offsets,
                                                     int32_t* tile_off, int32_t* cursor,
-                                                    int32_t* item_key) {
+                                                    int4* items) {
   __shared__ int32_t sp[1024], stl[1024];
   const int t = threadIdx.x;
   const int per = (n_keys + 1023) / 1024;
@@ -302,7 +303,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n
     offsets[key] = po;
     cursor[key] = po;
     tile_off[key] = to;
-    for (int u = 0; u < nt; ++u) item_key[to + u] = key;
+    for (int u = 0; u < nt; ++u)
+      items[to + u] = make_int4(key, po + u * tile_pairs, min(po + (u + 1) * tile_pairs, po + c), 0);
     po += c;
     to += nt;
   }
@@ -323,7 +325,8 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(Params P, PrefillWs
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x;
   if (tile >= ws.tile_off[ws.n_keys]) return;
-  const int key = ws.item_key[tile];
+  const int4 item = ws.items[tile];
+  const int key = item.x;
   const int j = key % P.max_chunks;
   const int bg = key / P.max_chunks / ws.n_win;
   const int g = bg % P.Hkv, b = bg / P.Hkv;
@@ -340,8 +343,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(Params P, PrefillWs
     for (int u = 0; u < 8; ++u) sV[s * LD + e8 + u] = v[u];
   }
   __syncthreads();
-  const int p0 = ws.offsets[key] + (tile - ws.tile_off[key]) * kTilePairs;
-  const int p1 = min(p0 + kTilePairs, ws.offsets[key + 1]);
+  const int p0 = item.y, p1 = item.z;
   float* q = sQ + warp * D;
   for (int p = p0 + warp; p < p1; p += kAttWarps) {
     const int32_t pid = ws.pairs[p];
@@ -435,14 +437,14 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
       const Windows W{ws.n_win, ws.win_rows};
       bucket_count_kernel<<<bgrid, 256, hsm / 2, s>>>(P, ws.idx, ws.counts, W);
       scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
-                                     ws.cursor, ws.item_key);
+                                     ws.cursor, ws.items);
       bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, W);
     } else {
       const unsigned pb = (unsigned)((n_pairs + 255) / 256);
       const Windows W{ws.n_win, ws.win_rows};
       count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs, W);
       scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
-                                     ws.cursor, ws.item_key);
+                                     ws.cursor, ws.items);
       scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, n_pairs, W);
     }
   }
@@ -523,7 +525,7 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.n_win = n_win;
   w.win_rows = win_rows;
   w.max_tiles = (n_pairs + kTilePairs - 1) / kTilePairs + n_keys;
-  w.item_key = (int32_t*)take(sizeof(int32_t) * w.max_tiles);
+  w.items = (int4*)take(sizeof(int4) * w.max_tiles);
   if (ws) *ws = w;
   return off;
 }

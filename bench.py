@@ -35,8 +35,8 @@ sys.path.insert(0, ROOT)
 import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_KERNELS_PER_STEP = 6   # select, count, scan, scatter, attend, merge (bf16 path)
-DECODE_KERNELS_PER_STEP = 2    # scan (+append, selection), attend (+merge)
+PREFILL_KERNELS_PER_STEP = 8   # calib, score, select, bucket count, scan, scatter, attend, merge (bf16)
+DECODE_KERNELS_PER_STEP = 3    # prep (append, calibration), scan (+selection), attend (+merge)
 
 
 def peaks():
@@ -230,7 +230,12 @@ def time_prefill_e2e(hils, torch, wl, steps, warmup):
 
 def time_decode(hils, torch, wl, warmup_steps=8, n_steps=0):
     """All decode steps of the workload, one after another (each appends its
-    token); L2 is flushed before every step and only the step itself is timed."""
+    token).  The step is captured once as a CUDA graph (its three kernels keep
+    their programmatic-launch overlap) and replayed per step: that step's
+    inputs are staged into the graph's buffers and L2 is flushed before it, and
+    only the replay is timed, so host launch cost never shows up as GPU time.
+    A second, eager pass with per-kernel events gives the kernel split (events
+    between the kernels serialise them, so that split over-counts)."""
     w = wl["workload"]
     cfg = cfg_of(hils, w)
     cache = make_cache(hils, wl)
@@ -239,32 +244,59 @@ def time_decode(hils, torch, wl, warmup_steps=8, n_steps=0):
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=dt, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
     seq0 = wl["seq_lens"].clone()
+    sq = torch.empty_like(wl["q_dec"][0])
+    sk = torch.empty_like(wl["k_new"][0])
+    sv = torch.empty_like(wl["v_new"][0])
 
-    def run(n, timed):
-        wl["seq_lens"].copy_(seq0)
-        evs = []
-        for s in range(n):
-            flush.zero_()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            hils.decode(cfg, wl["q_dec"][s], wl["k_new"][s], wl["v_new"][s], wl["A"], wl["B"], cache,
-                        out, None, None, ws, nbytes, stream)
-            b.record(stream)
-            evs.append((a, b))
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) for a, b in evs]
+    def stage(s):
+        sq.copy_(wl["q_dec"][s])
+        sk.copy_(wl["k_new"][s])
+        sv.copy_(wl["v_new"][s])
+
+    def call(stream):
+        hils.decode(cfg, sq, sk, sv, wl["A"], wl["B"], cache, out, None, None, ws, nbytes, stream)
 
     n = n_steps if n_steps > 0 else w.decode_steps
-    run(warmup_steps, False)
-    # step times without per-kernel events (they would separate the two kernels)
-    times = run(n, True)
-    # per-kernel times from a second pass over the same steps
+    # eager warm-up (also sets the kernels' shared-memory limits), then capture
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for s in range(warmup_steps):
+            stage(s % n)
+            call(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(torch.cuda.current_stream())
+    stream = torch.cuda.current_stream()
+
+    wl["seq_lens"].copy_(seq0)
+    evs = []
+    for s in range(n):
+        stage(s)
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    hils.device_status(stream)
+    del graph
+
+    # per-kernel split: eager steps with the event profiler
+    wl["seq_lens"].copy_(seq0)
     hils.profile_reset()
     hils.profile_enable(True)
-    run(n, True)
+    for s in range(n):
+        stage(s)
+        flush.zero_()
+        call(stream)
+    torch.cuda.synchronize()
     hils.profile_enable(False)
     phases = hils.profile_read()
     hils.device_status(stream)
@@ -398,8 +430,9 @@ def main():
         times, dph = time_decode(hils, torch, dwl, n_steps=args.decode_steps)
         if rank == 0:
             print(json.dumps({"decode_only": dw.name, "us_per_step": statistics.mean(times) * 1e3,
-                              "kernels_us_per_step": {k: v[0] / max(1, v[1]) * 1e3
-                                                      for k, v in dph.items()}}))
+                              "us_per_step_median": statistics.median(times) * 1e3,
+                              "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3
+                                                                 for k, v in dph.items()}}))
         return
     wl = hi.device_workload(w, seed_offset=rank)
     torch.cuda.synchronize()
@@ -449,21 +482,19 @@ def main():
         tot = statistics.mean(b["total"] for b in by)
         kvb = statistics.mean(b["kv_bytes"] for b in by)
         lmb = statistics.mean(b["landmark_bytes"] for b in by)
-        dom_d = max(dph.items(), key=lambda kv: kv[1][0])
-        dn, (dms, dl) = dom_d
-        dms_per = dms / max(1, dl)
-        dbytes = lmb if dn == "decode.scan" else kvb
         result["decode"] = {
             "workload": dw.name, "us_per_step": us, "steps": len(times),
             "context": dw.seq_len, "bytes_per_step": tot, "landmark_bytes": lmb, "kv_bytes": kvb,
             "step_gbs": tot / (us / 1e6) / 1e9,
             "step_hbm_frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"],
-            "kernels_us_per_step": {k: v[0] / max(1, v[1]) * 1e3 for k, v in dph.items()},
-            "roofline": {"bound": "hbm", "kernel": dn, "achieved": dbytes / (dms_per / 1e3) / 1e9,
-                         "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": dbytes / (dms_per / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+            "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3 for k, v in dph.items()},
+            # the step's kernels overlap (programmatic dependent launch), so the
+            # roofline is taken over the whole step: its algorithmic bytes / step time
+            "roofline": {"bound": "hbm", "kernel": "decode step (prep + scan + attend, overlapped)",
+                         "achieved": tot / (us / 1e6) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"], "traffic": None,
                          "peak_source": f"{pk_src} HBM copy bandwidth"},
-            "l2": "flushed (256 MB write) before every step; only the step is timed",
+            "timing": "CUDA graph replay of one step; inputs staged and L2 flushed (256 MB write) before it; only the replay is timed",
             "gpu_launches": DECODE_KERNELS_PER_STEP * len(times),
         }
         del dwl

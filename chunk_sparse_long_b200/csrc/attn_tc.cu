@@ -518,8 +518,7 @@ template <int D>
 cudaError_t run_attn_tc(const Params& P, void* out, const int32_t* idx, const float* w,
                         const PrefillWs& ws, cudaStream_t s) {
   using Lay = AttnLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Lay::kSmem);
+  cudaError_t e = set_smem(attn_tc_kernel<D>, Lay::kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, per_sm = 1;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;

@@ -1,31 +1,30 @@
-// Decode step (a8): append, landmark scan, selection, split-k chunk attention.
+// Decode step (a8): append, calibration, landmark scan, selection, split-k
+// chunk attention, as two kernels; the second is launched as a programmatic
+// dependent of the first (it may start early and waits for it before reading
+// its results).
 //
-//   scan    grid (n_split, B), 256 threads.  A CTA owns a contiguous range of
-//           chunks of one sequence.  Each thread first issues all its 16-byte
-//           landmark loads (a 256-byte slice covering whole heads) together
-//           with the calibration matrices; q~ is computed for every query head
-//           while they land, then the slice is scored.  Each head's best k-1
-//           candidates of the range are found by a warp bitonic sort and
-//           written out, best first, with the range's best score; the first
-//           CTA also writes every head's own-chunk score.  The last CTA of a
-//           sequence (one ticket per CTA) advances seq_lens.  No CTA waits.
-//   attend  grid (k, Hq, B), 128 threads, launched as a programmatic
-//           dependent of the scan.  Every CTA of a (sequence, head) merges that
-//           head's ranges itself (the k CTAs of a head do the same merge in
-//           parallel rather than one CTA serially):
-//             tau = the (k-1)-th largest of the threads' maxima of the ranges'
-//                   best scores -- a lower bound of the (k-1)-th best
-//                   candidate, since that many distinct candidates reach it;
-//             every range's list (sorted) is read only down to tau;
-//             the survivors are reduced to the best k-1 by bitonic merges.
-//           The own chunk joins them, the fusion weights follow, and the CTA
-//           attends to its slot's chunk (K and V staged in shared memory):
-//           softmax, P.V, the weighted partial to the workspace; the last CTA
-//           of a (sequence, head) sums the k partials in slot order
-//           (deterministic).
+//   scan    grid (n_split, Hkv, B), 256 threads.  A CTA owns one KV head and a
+//           contiguous range of chunks of one sequence.  Every thread first
+//           issues its 256 bytes of landmark loads and the loads of A, B and
+//           the group's queries; q~ = q + (q A) B of the group's query heads is
+//           computed while the landmarks land, then every chunk of the range is
+//           scored.  Per query head, each warp sorts its part of the range
+//           (warp bitonic sort and merges) and warp 0 merges the warps' lists
+//           into the range's best k-1, written out best first.  The last CTA of
+//           a (sequence, KV head) -- one ticket per CTA -- merges the ranges'
+//           lists into the head's best k-1, adds the own chunk (its score from
+//           the own landmark), and writes the selection and the fusion weights.
+//           The first CTA of a (sequence, KV head) appends k_t and v_t.
+//   attend  grid (k, Hq, B), 128 threads.  The CTA of a (sequence, head, slot)
+//           attends to the slot's chunk: K and V staged in shared memory,
+//           softmax (keys after the query masked in the own chunk), P.V, the
+//           weighted partial to the workspace.  The last CTA of a (sequence,
+//           head) sums the k partials in slot order (deterministic); the last
+//           head of a sequence advances seq_lens.
 #include <cfloat>
 
 #include "hils_common.cuh"
+#include "tc_common.cuh"
 
 namespace hils {
 namespace {
@@ -33,87 +32,96 @@ namespace {
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kAttThreads = 128;
-constexpr int kMergeCap = 512;    // survivors a merging warp can hold
-constexpr int kMergeGroup = 8;    // ranges a lane reads per round of loads
 constexpr unsigned kFull = 0xffffffffu;
 
-// (sa, ja) ranks above (sb, jb): score descending, then chunk index ascending.
-__device__ __forceinline__ bool better(float sa, int ja, float sb, int jb) {
-  return sa > sb || (sa == sb && ja < jb);
+// Selection keys.  A score maps to an unsigned key that orders like the score
+// (-0 taken as +0); key 0 means "no entry" and lies below every real score, and
+// -inf (a chunk that is not a candidate) maps to it as well.  Among equal keys
+// the lower chunk index ranks higher.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  if (s == -INFINITY) return 0u;
+  const uint32_t u = __float_as_uint(s + 0.f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t u) {
+  return u == 0u ? -INFINITY : __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Sorts one (s, j) per lane across the warp, best first (lane 0 = best).
-__device__ __forceinline__ void warp_sort(float& s, int& j) {
+// The best (key, chunk) offered by the warp's lanes: the largest key, and among
+// lanes holding it the lowest chunk.  Two warp reductions.
+__device__ __forceinline__ void warp_best(uint32_t u, int j, uint32_t& bu, int& bj) {
+  bu = __reduce_max_sync(kFull, u);
+  bj = (int)__reduce_min_sync(kFull, u == bu ? (uint32_t)j : 0xFFFFFFFFu);
+}
+
+// Best k (<= 32) of the V entries each lane holds, by rounds of extraction;
+// lane a of the result holds the a-th best (key 0: none).  The entries are
+// consumed.
+template <int V>
+__device__ __forceinline__ void warp_topk(uint32_t (&u)[V], int (&j)[V], int k, uint32_t& ou,
+                                          int& oj) {
   const int lane = threadIdx.x & 31;
+  ou = 0u;
+  oj = INT32_MAX;
+  for (int it = 0; it < k; ++it) {
+    uint32_t cu = 0u;
+    int cj = INT32_MAX;
 #pragma unroll
-  for (int k = 2; k <= 32; k <<= 1) {
+    for (int q = 0; q < V; ++q)
+      if (u[q] > cu || (u[q] == cu && j[q] < cj)) {
+        cu = u[q];
+        cj = j[q];
+      }
+    uint32_t bu;
+    int bj;
+    warp_best(cu, cj, bu, bj);
+    if (bu == 0u) break;
+    if (lane == it) {
+      ou = bu;
+      oj = bj;
+    }
 #pragma unroll
-    for (int m = k >> 1; m > 0; m >>= 1) {
-      const float os = __shfl_xor_sync(kFull, s, m);
-      const int oj = __shfl_xor_sync(kFull, j, m);
-      const bool lower = (lane & m) == 0;
-      const bool desc = (lane & k) == 0;        // this block sorts best first
-      const bool keep_better = lower == desc;
-      const bool take = keep_better ? better(os, oj, s, j) : better(s, j, os, oj);
-      if (take) {
-        s = os;
-        j = oj;
+    for (int q = 0; q < V; ++q)
+      if (u[q] == bu && j[q] == bj) u[q] = 0u;
+  }
+}
+
+// Best k (<= 32) of n lists sorted best first, each of length k, in shared
+// memory (list l at lu[l * k], lj[l * k]); lane a of the result holds the a-th
+// best.  Lane x follows lists x, x + 32, ...; hp[] holds the lists' read
+// positions (shared memory, n entries, reset here).
+__device__ __forceinline__ void warp_merge_lists(const uint32_t* lu, const int* lj, int n, int k,
+                                                 int* hp, uint32_t& ou, int& oj) {
+  const int lane = threadIdx.x & 31;
+  for (int l = lane; l < n; l += 32) hp[l] = 0;
+  __syncwarp();
+  ou = 0u;
+  oj = INT32_MAX;
+  for (int it = 0; it < k; ++it) {
+    uint32_t cu = 0u;
+    int cj = INT32_MAX, cl = -1;
+    for (int l = lane; l < n; l += 32) {
+      const int p = hp[l];
+      if (p >= k) continue;
+      const uint32_t u = lu[l * k + p];
+      const int j = lj[l * k + p];
+      if (u > cu || (u == cu && j < cj)) {
+        cu = u;
+        cj = j;
+        cl = l;
       }
     }
-  }
-}
-
-// a (sorted best first across lanes) := best 32 of a and b (b sorted best first).
-__device__ __forceinline__ void warp_merge(float& as, int& aj, float bs, int bj) {
-  const int lane = threadIdx.x & 31;
-  const float rs = __shfl_sync(kFull, bs, 31 - lane);
-  const int rj = __shfl_sync(kFull, bj, 31 - lane);
-  if (better(rs, rj, as, aj)) {   // the elementwise winners form a bitonic sequence
-    as = rs;
-    aj = rj;
-  }
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) {
-    const float os = __shfl_xor_sync(kFull, as, m);
-    const int oj = __shfl_xor_sync(kFull, aj, m);
-    const bool lower = (lane & m) == 0;
-    const bool take = lower ? better(os, oj, as, aj) : better(as, aj, os, oj);
-    if (take) {
-      as = os;
-      aj = oj;
-    }
-  }
-}
-
-// Best 32 of n (s, j) entries in shared memory, sorted best first across lanes.
-__device__ void warp_top32(const float* s, const int* j, int n, float& os, int& oj) {
-  const int lane = threadIdx.x & 31;
-  os = -INFINITY;
-  oj = INT32_MAX;
-  for (int x0 = 0; x0 < n; x0 += 32) {
-    float bs = x0 + lane < n ? s[x0 + lane] : -INFINITY;
-    int bj = x0 + lane < n ? j[x0 + lane] : INT32_MAX;
-    warp_sort(bs, bj);
-    if (x0 == 0) {
-      os = bs;
+    uint32_t bu;
+    int bj;
+    warp_best(cu, cj, bu, bj);
+    if (bu == 0u) break;
+    if (lane == it) {
+      ou = bu;
       oj = bj;
-    } else {
-      warp_merge(os, oj, bs, bj);
     }
+    if (cl >= 0 && cu == bu && cj == bj) hp[cl] += 1;   // the owner moves past its entry
+    __syncwarp();
   }
-}
-
-// Appends (s, j) for lanes with keep to a warp-private list; returns the new count.
-__device__ __forceinline__ int warp_append(bool keep, float s, int j, float* ls, int* lj, int count,
-                                           int cap) {
-  const int lane = threadIdx.x & 31;
-  const unsigned bal = __ballot_sync(kFull, keep);
-  const int at = count + __popc(bal & ((1u << lane) - 1u));
-  if (keep && at < cap) {
-    ls[at] = s;
-    lj[at] = j;
-  }
-  return count + __popc(bal);
 }
 
 template <int EB>
@@ -133,96 +141,159 @@ __device__ __forceinline__ void unpack16(const uint4& u, float* v) {
   }
 }
 
-// D: head dim; EB: element bytes; SLICE: elements per thread (a multiple or a
-// divisor of D, and a divisor of Hkv*D).
-template <int D, int EB, int SLICE>
-__global__ void __launch_bounds__(kScanThreads, 2)
-    scan_kernel(Params P, const void* k_new, const void* v_new, DecodeWs ws) {
-  constexpr int U = SLICE * EB / 16;               // 16-byte loads per thread
-  constexpr int EPU = 16 / EB;                     // elements per 16-byte load
-  constexpr int QS = D + 4;                        // padded q~ row (conflict-free float4 reads)
-  extern __shared__ float sm[];
-  float* sA = sm;                                  // [D][r] calibration A
-  float* sB = sA + D * P.r;                        // [r][D] calibration B
-  float* sq = sB + P.r * D;                        // [Hq][D] raw q
-  float* sqt = sq + P.Hq * D;                      // [Hq][QS] q~
-  float* sT = sqt + P.Hq * QS;                     // [Hq][kMaxRank] q A
-  float* sS = sT + P.Hq * kMaxRank;                // [chunks_per_split][Hq] scores
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, b = blockIdx.y;
-  const bool append = k_new != nullptr;
+// Decode position of sequence b: seq_lens[b] when appending, else the last
+// token; clamped (and flagged) if it falls outside the block table.
+__device__ __forceinline__ int64_t decode_pos(const Params& P, int b, bool append, bool report) {
   int64_t t = append ? (int64_t)P.seq_lens[b] : (int64_t)P.seq_lens[b] - 1;
-  if (t < 0 || t >= (int64_t)P.max_chunks * kChunk) {  // position outside the block table
-    if (tid == 0 && split == 0) set_device_error(kErrChunk);
+  if (t < 0 || t >= (int64_t)P.max_chunks * kChunk) {
+    if (report) set_device_error(kErrChunk);
     t = t < 0 ? 0 : (int64_t)P.max_chunks * kChunk - 1;
   }
-  const int64_t own = t / kChunk;
-  const int K = P.k - 1;
-  const int row = P.Hkv * D;                       // elements of one chunk's landmarks
-  const int64_t c0 = (int64_t)split * ws.chunks_per_split;
-  const int64_t c1 = min(c0 + ws.chunks_per_split, own);   // candidates j < own
-  const int nloc = c1 > c0 ? (int)(c1 - c0) : 0;
+  return t;
+}
 
-  // ---- every load first: landmark slice, calibration matrices, queries -----
-  const int64_t s0 = (int64_t)tid * SLICE;          // element offset inside the range
-  const bool have = s0 < (int64_t)nloc * row;
-  uint4 lm[U];
-  {
+// Landmark work of one scan thread: 256 bytes of one KV head's landmark rows.
+template <int D, int EB>
+struct ScanGeo {
+  static constexpr int SLICE = 256 / EB;                  // landmark elements per thread
+  static constexpr int CPT = SLICE >= D ? SLICE / D : 1;  // chunks per thread
+  static constexpr int TPC = SLICE >= D ? 1 : D / SLICE;  // threads per chunk
+  static constexpr int EPT = SLICE >= D ? D : SLICE;      // elements per (thread, chunk)
+  static constexpr int CPS = kScanThreads * CPT / TPC;    // chunks per CTA
+  static constexpr int EPU = 16 / EB;                     // elements per 16-byte load
+  static constexpr int UPC = EPT / EPU;                   // 16-byte loads per (thread, chunk)
+  static constexpr int SEG = CPS / kScanWarps;            // chunks a warp sorts
+};
+
+template <int D>
+struct ScanSmem {
+  // the last part stages the ranges' lists of one query head for the last CTA:
+  // keys, chunks and read positions
+  static size_t bytes(int r, int group, int cps, int n_split, int k1) {
+    return sizeof(float) * (size_t)(2 * D * r + group * D + group * (D + 4) + group * kMaxRank +
+                                    cps * group + 2 * kScanWarps * 32 + D +
+                                    n_split * (2 * k1 + 1));
+  }
+};
+
+template <int D, int EB>
+__global__ void __launch_bounds__(kScanThreads, 2)
+    scan_kernel(Params P, const void* k_new, const void* v_new, DecodeWs ws, int32_t* idx_out,
+                float* w_out) {
+  using G = ScanGeo<D, EB>;
+  // the attention grid may be scheduled now; it waits for this one before its reads
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int QS = D + 4;                        // padded q~ row
+  const int group = P.group, K = P.k - 1;
+  extern __shared__ float sm[];
+  float* sA = sm;                                  // [D][r]
+  float* sB = sA + D * P.r;                        // [r][D]
+  float* sq = sB + P.r * D;                        // [group][D] raw q
+  float* sqt = sq + group * D;                     // [group][QS] q~
+  float* sT = sqt + group * QS;                    // [group][kMaxRank] q A
+  float* sS = sT + group * kMaxRank;               // [CPS][group] scores
+  uint32_t* lu = reinterpret_cast<uint32_t*>(sS + G::CPS * group);  // [kScanWarps][k-1] warp lists
+  int* lj = reinterpret_cast<int*>(lu + kScanWarps * 32);           // chunks of those
+  float* slm = reinterpret_cast<float*>(lj + kScanWarps * 32);      // [D] own chunk's landmark
+  uint32_t* mu = reinterpret_cast<uint32_t*>(slm + D);  // [n_split][k-1] ranges' lists (last CTA)
+  int* mj = reinterpret_cast<int*>(mu + ws.n_split * K);
+  int* mhp = mj + ws.n_split * K;                       // [max(n_split, warps)] read positions
+  __shared__ int last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const bool append = ws.append != 0;
+  const int64_t t = decode_pos(P, b, append, tid == 0 && split == 0 && g == 0);
+  const int64_t own = t / kChunk;
+  const int64_t c0 = (int64_t)split * G::CPS;
+  const int cl0 = G::TPC == 1 ? tid * G::CPT : tid / G::TPC;   // first local chunk
+  const int part = G::TPC == 1 ? 0 : tid % G::TPC;              // element part of the row
+
+  // ---- every load first ---------------------------------------------------------
+  uint4 lm[G::CPT][G::UPC];
+#pragma unroll
+  for (int ci = 0; ci < G::CPT; ++ci) {
+    const int64_t j = c0 + cl0 + ci;
+    const bool cand = j < own;
     const uint4* src = reinterpret_cast<const uint4*>(
         reinterpret_cast<const uint8_t*>(P.landmarks) +
-        (((int64_t)b * P.max_chunks + c0) * row + (have ? s0 : 0)) * EB);
+        ((((int64_t)b * P.max_chunks + (cand ? j : 0)) * P.Hkv + g) * D + part * G::EPT) * EB);
 #pragma unroll
-    for (int u = 0; u < U; ++u) lm[u] = have ? __ldcs(src + u) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < G::UPC; ++u) lm[ci][u] = cand ? __ldcs(src + u) : make_uint4(0, 0, 0, 0);
   }
-  // the own chunk's landmarks (first CTA of the sequence), one 16-byte unit per thread
-  const bool own_unit = split == 0 && tid * EPU < row;
-  uint4 own_lm = make_uint4(0, 0, 0, 0);
-  if (own_unit)
-    own_lm = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(P.landmarks) +
-                                                  (((int64_t)b * P.max_chunks + own) * row +
-                                                   tid * EPU) * EB));
-  for (int x = tid; x < D * P.r; x += kScanThreads) {
-    sA[x] = __ldg(P.A + x);
-    sB[x] = __ldg(P.Bm + x);
-  }
-  for (int x = tid; x < P.Hq * D; x += kScanThreads)
-    sq[x] = load_elem(P.q, EB == 2 ? HILS_BF16 : HILS_F32, (int64_t)b * P.Hq * D + x);
-
-  if (append && split == 0) {
-    const int64_t page = page_of(P, b, own);
-    if (page >= 0) {
-      const int slot = (int)(t % kChunk);
-      for (int x = tid; x < P.Hkv * D; x += kScanThreads) {
-        const int g = x / D, e = x % D;
-        const int64_t ko = page_offset(P, page, 0, g, slot) + e;
-        const int64_t vo = page_offset(P, page, 1, g, slot) + e;
-        const int64_t src = ((int64_t)b * P.Hkv + g) * D + e;
-        if (EB == 4) {
-          ((float*)P.pages)[ko] = ((const float*)k_new)[src];
-          ((float*)P.pages)[vo] = ((const float*)v_new)[src];
-        } else {
-          ((uint16_t*)P.pages)[ko] = ((const uint16_t*)k_new)[src];
-          ((uint16_t*)P.pages)[vo] = ((const uint16_t*)v_new)[src];
-        }
+  {
+    constexpr int NQ = (64 * D / G::EPU + kScanThreads - 1) / kScanThreads;
+    const int na = D * P.r / 4, nq = group * D / G::EPU;
+    uint4 rq[NQ], rl = make_uint4(0, 0, 0, 0);
+    // A and B straight into shared memory (asynchronous copies, no registers)
+    for (int x = tid; x < na; x += kScanThreads) {
+      tc::cp_async16(tc::smem_u32(sA + 4 * x), reinterpret_cast<const float4*>(P.A) + x, 16u);
+      tc::cp_async16(tc::smem_u32(sB + 4 * x), reinterpret_cast<const float4*>(P.Bm) + x, 16u);
+    }
+    tc::cp_async_commit();
+    const uint4* qsrc = reinterpret_cast<const uint4*>(
+        reinterpret_cast<const uint8_t*>(P.q) + ((int64_t)b * P.Hq + (int64_t)g * group) * D * EB);
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int x = u * kScanThreads + tid;
+      if (x < nq) rq[u] = __ldg(qsrc + x);
+    }
+    if (tid < D / G::EPU)
+      rl = __ldg(reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint8_t*>(P.landmarks) +
+          (((int64_t)b * P.max_chunks + own) * P.Hkv + g) * D * EB) + tid);
+    // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
+    if (append && split == 0 && tid < 2 * (D / G::EPU)) {
+      const int64_t page = page_of(P, b, own);
+      if (page >= 0) {
+        const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x;
+        uint4* dst = reinterpret_cast<uint4*>(
+            reinterpret_cast<uint8_t*>(const_cast<void*>(P.pages)) +
+            page_offset(P, page, kind, g, (int)(t % kChunk)) * EB) + x;
+        *dst = __ldg(src);
       }
     }
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int x = u * kScanThreads + tid;
+      if (x < nq) {
+        float v[G::EPU];
+        unpack16<EB>(rq[u], v);
+#pragma unroll
+        for (int e = 0; e < G::EPU; ++e) sq[x * G::EPU + e] = v[e];
+      }
+    }
+    if (tid < D / G::EPU) {
+      float v[G::EPU];
+      unpack16<EB>(rl, v);
+#pragma unroll
+      for (int e = 0; e < G::EPU; ++e) slm[tid * G::EPU + e] = v[e];
+    }
+    tc::cp_async_wait<0>();
   }
-  if (split == 0 && tid == 0) ws.tpos[b] = (int32_t)t;
   __syncthreads();
 
-  // ---- a1: q~ = q + (q A) B for every query head -----------------------------
-  for (int x = tid; x < P.Hq * P.r; x += kScanThreads) {
-    const int h = x / P.r, a = x % P.r;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};   // four independent chains
-#pragma unroll
-    for (int e = 0; e < D; e += 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(sq[h * D + e + u], sA[(e + u) * P.r + a], acc[u]);
+  // ---- a1: q~ = q + (q A) B of the group's heads --------------------------------
+  if (P.r > 0) {
+    // t[h][a]: LP lanes per (h, a) pair, each summing a strided part over e
+    const int pairs = group * P.r;
+    int LP = 32;
+    while (LP > 1 && LP * pairs > kScanThreads) LP >>= 1;
+    for (int base = 0; base < pairs * LP; base += kScanThreads) {
+      const int x = base + tid;
+      const int pr = x / LP, sub = x % LP;
+      float acc = 0.f;
+      if (pr < pairs) {
+        const int h = pr / P.r, a = pr % P.r;
+        for (int e = sub; e < D; e += LP) acc = fmaf(sq[h * D + e], sA[e * P.r + a], acc);
+      }
+      for (int o = LP >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+      if (pr < pairs && sub == 0) sT[(pr / P.r) * kMaxRank + pr % P.r] = acc;
     }
-    sT[h * kMaxRank + a] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    __syncthreads();
   }
-  __syncthreads();
-  for (int x = tid; x < P.Hq * D; x += kScanThreads) {
+  for (int x = tid; x < group * D; x += kScanThreads) {
     const int h = x / D, e = x % D;
     float acc = sq[x];
     for (int a = 0; a < P.r; ++a) acc = fmaf(sT[h * kMaxRank + a], sB[a * D + e], acc);
@@ -230,264 +301,111 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   }
   __syncthreads();
 
-  // ---- a2: scores of this thread's slice -------------------------------------
-  {
-    const int jj = (int)(s0 / row);
-    const int off = (int)(s0 % row);
-    constexpr int HPS = SLICE >= D ? SLICE / D : 1;   // heads in the slice
-    constexpr int TPH = SLICE >= D ? 1 : D / SLICE;   // threads sharing one head
-    constexpr int EPH = SLICE >= D ? D : SLICE;       // elements of one head in the slice
+  // ---- a2: scores of the range ----------------------------------------------------
 #pragma unroll
-    for (int hs = 0; hs < HPS; ++hs) {
-      const int g = off / D + hs;
-      const int e0 = SLICE >= D ? 0 : off % D;
-      for (int hh = 0; hh < P.group; ++hh) {
-        const int h = (have ? g : 0) * P.group + hh;
-        const float* qt = sqt + h * QS + e0;
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < EPH / EPU; ++u) {
-          float lv[EPU];
-          unpack16<EB>(lm[hs * (EPH / EPU) + u], lv);
-#pragma unroll
-          for (int e = 0; e < EPU; e += 4) {
-            const float4 q4 = *reinterpret_cast<const float4*>(qt + u * EPU + e);
-            acc = fmaf(q4.x, lv[e], acc);
-            acc = fmaf(q4.y, lv[e + 1], acc);
-            acc = fmaf(q4.z, lv[e + 2], acc);
-            acc = fmaf(q4.w, lv[e + 3], acc);
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < TPH; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        if (have && (tid % TPH) == 0) sS[jj * P.Hq + h] = acc * P.inv_sqrt_d;
-      }
-    }
-  }
-  // own chunk scores: one 16-byte unit per thread, partial dots gathered in shared memory
-  if (split == 0) {
-    float* part = sS + ws.chunks_per_split * P.Hq;   // [Hq][D / EPU] partial dots
-    for (int x = tid; x < row / EPU; x += kScanThreads) {
-      const uint4 u = x == tid ? own_lm
-                               : __ldg(reinterpret_cast<const uint4*>(
-                                     reinterpret_cast<const uint8_t*>(P.landmarks) +
-                                     (((int64_t)b * P.max_chunks + own) * row + x * EPU) * EB));
-      float lv[EPU];
-      unpack16<EB>(u, lv);
-      const int g = (x * EPU) / D, e0 = (x * EPU) % D;
-      for (int hh = 0; hh < P.group; ++hh) {
-        const int h = g * P.group + hh;
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPU; ++e) acc = fmaf(sqt[h * QS + e0 + e], lv[e], acc);
-        part[h * (D / EPU) + e0 / EPU] = acc;
-      }
-    }
-    __syncthreads();
-    for (int h = warp; h < P.Hq; h += kScanWarps) {
+  for (int ci = 0; ci < G::CPT; ++ci) {
+    const int64_t j = c0 + cl0 + ci;
+    for (int hh = 0; hh < group; ++hh) {
+      const float* qt = sqt + hh * QS + part * G::EPT;
       float acc = 0.f;
-      for (int u = lane; u < D / EPU; u += 32) acc += part[h * (D / EPU) + u];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-      if (lane == 0) ws.s_own[(int64_t)b * P.Hq + h] = acc * P.inv_sqrt_d;
+      for (int u = 0; u < G::UPC; ++u) {
+        float lv[G::EPU];
+        unpack16<EB>(lm[ci][u], lv);
+#pragma unroll
+        for (int e = 0; e < G::EPU; e += 4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(qt + u * G::EPU + e);
+          acc = fmaf(q4.x, lv[e], acc);
+          acc = fmaf(q4.y, lv[e + 1], acc);
+          acc = fmaf(q4.z, lv[e + 2], acc);
+          acc = fmaf(q4.w, lv[e + 3], acc);
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < G::TPC; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+      if (part == 0) sS[(cl0 + ci) * group + hh] = j < own ? acc * P.inv_sqrt_d : -INFINITY;
     }
   }
   __syncthreads();
 
-  // ---- a3 (local): best k-1 candidates of the range per head ----------------
-  if (K > 0) {
-    float* cs = ws.cand_s + ((int64_t)b * ws.n_split + split) * P.Hq * K;
-    int32_t* cj = ws.cand_j + ((int64_t)b * ws.n_split + split) * P.Hq * K;
-    for (int h = warp; h < P.Hq; h += kScanWarps) {
-      float bs = -INFINITY;
-      int bj = INT32_MAX;
-      for (int x0 = 0; x0 < nloc; x0 += 32) {
-        float s = x0 + lane < nloc ? sS[(x0 + lane) * P.Hq + h] : -INFINITY;
-        int j = x0 + lane < nloc ? (int)(c0 + x0 + lane) : INT32_MAX;
-        warp_sort(s, j);
-        if (x0 == 0) {
-          bs = s;
-          bj = j;
-        } else {
-          warp_merge(bs, bj, s, j);
-        }
-      }
+  // ---- a3 (range): best k-1 of the range per query head ---------------------------
+  // each warp extracts the best k-1 of its part of the range, warp 0 merges the
+  // warps' lists
+  for (int hh = 0; hh < group && K > 0; ++hh) {
+    const int h = g * group + hh;
+    constexpr int V = G::SEG >= 32 ? G::SEG / 32 : 1;
+    uint32_t u[V];
+    int jj[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const int x = q * 32 + lane;
+      const int cl = warp * G::SEG + x;
+      u[q] = x < G::SEG ? score_key(sS[cl * group + hh]) : 0u;
+      jj[q] = (int)(c0 + cl);
+    }
+    uint32_t ou;
+    int oj;
+    warp_topk<V>(u, jj, K, ou, oj);
+    if (lane < K) {
+      lu[warp * K + lane] = ou;
+      lj[warp * K + lane] = oj;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      warp_merge_lists(lu, lj, kScanWarps, K, mhp, ou, oj);
       if (lane < K) {
-        cs[h * K + lane] = bs;
-        cj[h * K + lane] = bj == INT32_MAX ? -1 : bj;
+        const int64_t o = (((int64_t)b * P.Hq + h) * ws.n_split + split) * K + lane;
+        ws.cand_s[o] = key_score(ou);
+        ws.cand_j[o] = ou == 0u ? -1 : oj;
       }
-      if (lane == 0) ws.best[((int64_t)b * P.Hq + h) * ws.n_split + split] = bs;
-    }
-  }
-
-  // ---- the last CTA of the sequence advances seq_lens ---------------------
-  if (append) {
-    __syncthreads();
-    if (tid == 0) {
-      int32_t* cnt = ws.tickets + 2 * P.B * P.Hq + b;
-      const int old = atomicAdd(cnt, 1);
-      if (old == ws.n_split - 1) {
-        P.seq_lens[b] = (int32_t)(t + 1);
-        *cnt = 0;
-      }
-    }
-  }
-}
-
-template <int D, int EB>
-__global__ void __launch_bounds__(kAttThreads)
-    attend_kernel(Params P, DecodeWs ws, void* out, int32_t* idx_out, float* w_out) {
-  constexpr int EPU = 16 / EB;                 // elements per 16-byte load
-  constexpr int KL = D + (EB == 2 ? 8 : 4);    // padded shared-memory row (elements)
-  constexpr int NW = kAttThreads / 32;
-  extern __shared__ __align__(16) uint8_t kv_raw[];   // [2][kChunk][KL] elements
-  __shared__ float ms[kMergeCap];
-  __shared__ int mj[kMergeCap];
-  __shared__ float wmax_s[NW][32];
-  __shared__ int mcount;
-  __shared__ float tau_sh;
-  __shared__ int sel_j[kMaxTopK];
-  __shared__ float sel_w[kMaxTopK];
-  __shared__ float sq[D];
-  __shared__ float sp[kChunk];
-  __shared__ float red[8];
-  __shared__ float half_o[kAttThreads];
-  __shared__ int last;
-  // wait for the scan (programmatic dependent launch: this grid may start early)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
-  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / P.group;
-  const int64_t bh = (int64_t)b * P.Hq + h;
-  const int K = P.k - 1;
-  // independent loads first: position, own score, this head's query
-  const int64_t t = __ldcg(ws.tpos + b);
-  const float s_own = __ldcg(ws.s_own + bh);
-  for (int e = tid; e < D; e += kAttThreads)
-    sq[e] = load_elem(P.q, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e);
-  const int64_t own = t / kChunk;
-
-  // ---- a3: merge this head's ranges (every CTA of the head does the same) ----
-  if (tid == 0) mcount = 0;
-  if (K > 0) {
-    const float* bests = ws.best + bh * ws.n_split;
-    const float* all_s = ws.cand_s + (int64_t)b * ws.n_split * P.Hq * K + (int64_t)h * K;
-    const int32_t* all_j = ws.cand_j + (int64_t)b * ws.n_split * P.Hq * K + (int64_t)h * K;
-    const int64_t sstride = (int64_t)P.Hq * K;
-    float tmax = -INFINITY;
-    for (int sp0 = 0; sp0 < ws.n_split; sp0 += kAttThreads * kMergeGroup) {
-      float bv[kMergeGroup];
-#pragma unroll
-      for (int u = 0; u < kMergeGroup; ++u) {
-        const int spl = sp0 + u * kAttThreads + tid;
-        bv[u] = spl < ws.n_split ? __ldcg(bests + spl) : -INFINITY;
-      }
-#pragma unroll
-      for (int u = 0; u < kMergeGroup; ++u) tmax = fmaxf(tmax, bv[u]);
-    }
-    float ts = tmax;
-    int tj = tid;
-    warp_sort(ts, tj);
-    wmax_s[wrp][lane] = ts;
-    __syncthreads();
-    if (wrp == 0) {
-      float as = wmax_s[0][lane];
-      int aj = lane;
-      for (int w2 = 1; w2 < NW; ++w2) warp_merge(as, aj, wmax_s[w2][lane], 32 * w2 + lane);
-      const float tau = __shfl_sync(kFull, as, K - 1);
-      if (lane == 0) tau_sh = tau;
     }
     __syncthreads();
-    const float tau = tau_sh;
-    // survivors: each range's sorted list down to tau
-    for (int sp0 = 0; sp0 < ws.n_split; sp0 += kAttThreads * kMergeGroup) {
-      float bv[kMergeGroup];
-#pragma unroll
-      for (int u = 0; u < kMergeGroup; ++u) {
-        const int spl = sp0 + u * kAttThreads + tid;
-        bv[u] = spl < ws.n_split ? __ldcg(bests + spl) : -INFINITY;
-      }
-#pragma unroll
-      for (int u = 0; u < kMergeGroup; ++u) {
-        const int spl = sp0 + u * kAttThreads + tid;
-        if (spl >= ws.n_split || !(bv[u] >= tau)) continue;
-        for (int a0 = 0; a0 < K; a0 += 4) {
-          float v4[4];
-          int j4[4];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            v4[a] = a0 + a < K ? __ldcg(all_s + spl * sstride + a0 + a) : -INFINITY;
-            j4[a] = a0 + a < K ? __ldcg(all_j + spl * sstride + a0 + a) : -1;
-          }
-          bool more = true;
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            if (more && j4[a] >= 0 && v4[a] >= tau) {
-              const int at = atomicAdd(&mcount, 1);
-              if (at < kMergeCap) {
-                ms[at] = v4[a];
-                mj[at] = j4[a];
-              }
-            } else {
-              more = false;
-            }
-          }
-          if (!more) break;
-        }
-      }
-    }
   }
+
+  // ---- a3/a4: the last CTA of the (sequence, KV head) merges the ranges -----------
+  __threadfence();
   __syncthreads();
-  if (wrp == 0) {
-    float os = -INFINITY;
-    int oj = INT32_MAX;
-    if (K > 0) {
-      const int cnt = mcount;
-      if (cnt <= kMergeCap) {
-        warp_top32(ms, mj, cnt, os, oj);
-      } else {
-        // heavily tied scores: every range's list in full, 32 entries at a time
-        const int total = ws.n_split * K;
-        const float* all_s = ws.cand_s + (int64_t)b * ws.n_split * P.Hq * K + (int64_t)h * K;
-        const int32_t* all_j = ws.cand_j + (int64_t)b * ws.n_split * P.Hq * K + (int64_t)h * K;
-        const int64_t sstride = (int64_t)P.Hq * K;
-        for (int x0 = 0; x0 < total; x0 += 32) {
-          const int x = x0 + lane;
-          float v = x < total ? __ldcg(all_s + (x / K) * sstride + x % K) : -INFINITY;
-          int vj = x < total ? __ldcg(all_j + (x / K) * sstride + x % K) : -1;
-          if (vj < 0) {
-            v = -INFINITY;
-            vj = INT32_MAX;
-          }
-          warp_sort(v, vj);
-          if (x0 == 0) {
-            os = v;
-            oj = vj;
-          } else {
-            warp_merge(os, oj, v, vj);
-          }
-        }
-      }
+  if (tid == 0) last = atomicAdd(&ws.tickets[b * P.Hkv + g], 1) == ws.n_split - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int hh = 0; hh < group; ++hh) {
+    const int h = g * group + hh;
+    const int64_t bh = (int64_t)b * P.Hq + h;
+    // the ranges' lists of this head into shared memory
+    for (int x = tid; x < ws.n_split * K; x += kScanThreads) {
+      const float v = __ldcg(ws.cand_s + bh * ws.n_split * K + x);
+      const int vj = __ldcg(ws.cand_j + bh * ws.n_split * K + x);
+      mu[x] = vj < 0 ? 0u : score_key(v);
+      mj[x] = vj < 0 ? INT32_MAX : vj;
     }
-    // a4: slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
-    const float sh_s = __shfl_sync(kFull, os, (lane + 31) & 31);
-    const int sh_j = __shfl_sync(kFull, oj, (lane + 31) & 31);
-    const float my_s = lane == 0 ? s_own : sh_s;
-    const int my_j = lane == 0 ? (int)own : (sh_j == INT32_MAX ? -1 : sh_j);
-    const bool live = lane < P.k && my_j >= 0;
-    float m = live ? my_s : -INFINITY;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t ou = 0u;
+      int oj = INT32_MAX;
+      if (K > 0) warp_merge_lists(mu, mj, ws.n_split, K, mhp, ou, oj);
+      // the own chunk's score
+      float so = 0.f;
+      for (int e = lane; e < D; e += 32) so = fmaf(sqt[hh * QS + e], slm[e], so);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    const float ex = live ? __expf(my_s - m) : 0.f;
-    float z = ex;
+      for (int o = 16; o > 0; o >>= 1) so += __shfl_xor_sync(kFull, so, o);
+      so *= P.inv_sqrt_d;
+      // a4: slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
+      const uint32_t sh_u = __shfl_sync(kFull, ou, (lane + 31) & 31);
+      const int sh_j = __shfl_sync(kFull, oj, (lane + 31) & 31);
+      const float my_s = lane == 0 ? so : key_score(sh_u);
+      const int my_j = lane == 0 ? (int)own : (sh_u == 0u ? -1 : sh_j);
+      const bool live = lane < P.k && my_j >= 0;
+      float m = live ? my_s : -INFINITY;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-    if (lane < P.k) {
-      const int jv = live ? my_j : -1;
-      const float wv = live ? ex / z : 0.f;
-      sel_j[lane] = jv;
-      sel_w[lane] = wv;
-      if (slot == 0) {
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+      const float ex = live ? __expf(my_s - m) : 0.f;
+      float z = ex;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+      if (lane < P.k) {
+        const int jv = live ? my_j : -1;
+        const float wv = live ? ex / z : 0.f;
         const int64_t o = bh * P.k + lane;
         ws.idx[o] = jv;
         ws.w[o] = wv;
@@ -495,14 +413,39 @@ __global__ void __launch_bounds__(kAttThreads)
         if (w_out) w_out[o] = wv;
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
+  if (tid == 0) ws.tickets[b * P.Hkv + g] = 0;
+}
+
+template <int D, int EB>
+__global__ void __launch_bounds__(kAttThreads)
+    attend_kernel(Params P, DecodeWs ws, void* out) {
+  constexpr int EPU = 16 / EB;                 // elements per 16-byte load
+  constexpr int KL = D + (EB == 2 ? 8 : 4);    // padded shared-memory row (elements)
+  extern __shared__ __align__(16) uint8_t kv_raw[];   // [2][kChunk][KL] elements
+  __shared__ float sq[D];
+  __shared__ float sp[kChunk];
+  __shared__ float red[8];
+  __shared__ float half_o[kAttThreads];
+  __shared__ int last;
+  const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
+  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / P.group;
+  const int64_t bh = (int64_t)b * P.Hq + h;
+  // this head's query does not depend on the scan
+  for (int e = tid; e < D; e += kAttThreads)
+    sq[e] = load_elem(P.q, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e);
+  // wait for the scan (programmatic dependent launch: this grid may start early)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t t = decode_pos(P, b, ws.append != 0, false);
+  const int64_t own = t / kChunk;
+  const int32_t j = __ldcg(ws.idx + bh * P.k + slot);
+  const float wj = __ldcg(ws.w + bh * P.k + slot);
+  const int64_t page = j >= 0 ? page_of(P, b, j) : -1;
 
   // ---- a5: attention to this slot's chunk ----------------------------------
-  const int32_t j = sel_j[slot];
-  const float wj = sel_w[slot];
   float* part = ws.part + (bh * P.k + slot) * D;
-  const int64_t page = j >= 0 ? page_of(P, b, j) : -1;
   if (page >= 0) {
     // K and V tiles of the chunk into shared memory: every 16-byte load in flight at once
     const uint8_t* kp = reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 0, g, 0) * EB;
@@ -588,82 +531,80 @@ __global__ void __launch_bounds__(kAttThreads)
     for (int a = 0; a < P.k; ++a) acc += __ldcg(ws.part + (bh * P.k + a) * D + e);
     store_elem(out, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e, acc);
   }
-  if (tid == 0) ws.tickets[P.B * P.Hq + bh] = 0;
-}
-
-size_t scan_smem(const Params& P, const DecodeWs& ws, int D) {
-  const int epu = P.dtype == HILS_BF16 ? 8 : 4;
-  const size_t own_part = (size_t)P.Hq * (D / epu);
-  return (size_t)(2 * D * P.r + P.Hq * D + P.Hq * (D + 4) + P.Hq * kMaxRank +
-                  ws.chunks_per_split * P.Hq + own_part) * 4;
-}
-
-template <int D, int EB, int SLICE>
-cudaError_t run_decode_t(const Params& P, const void* k_new, const void* v_new, void* out,
-                         int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s) {
-  const size_t smem = scan_smem(P, ws, D);
-  cudaError_t e = cudaFuncSetAttribute(scan_kernel<D, EB, SLICE>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  {
-    HILS_PROFILE("decode.scan", s);
-    scan_kernel<D, EB, SLICE><<<dim3(ws.n_split, P.B), kScanThreads, smem, s>>>(P, k_new, v_new, ws);
+  if (tid == 0) {
+    ws.tickets[P.B * P.Hq + bh] = 0;
+    // every kernel of the step has read seq_lens: the last head of the sequence advances it
+    if (ws.append) {
+      int32_t* done = ws.tickets + 2 * P.B * P.Hq + b;
+      if (atomicAdd(done, 1) == P.Hq - 1) {
+        P.seq_lens[b] = (int32_t)(t + 1);
+        *done = 0;
+      }
+    }
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
-    HILS_PROFILE("decode.attend", s);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(P.k, P.Hq, P.B);
-    cfg.blockDim = dim3(kAttThreads);
-    const size_t kv_bytes = (size_t)2 * kChunk * (D + (EB == 2 ? 8 : 4)) * EB;
-    e = cudaFuncSetAttribute(attend_kernel<D, EB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kv_bytes);
-    if (e != cudaSuccess) return e;
-    cfg.dynamicSmemBytes = kv_bytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, attend_kernel<D, EB>, P, ws, out, idx_out, w_out);
-  }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
 }
 
-// Elements per thread slice: 256 bytes when a chunk's landmark row splits into
-// whole slices of that size, else 128 bytes (float32) / 64 elements.
-int slice_elems(const Params& P) {
-  const int eb = P.dtype == HILS_BF16 ? 2 : 4;
-  return (eb == 2 && (P.Hkv * P.d) % 128 == 0) ? 128 : 64;
+size_t scan_smem(const Params& P, int D, int cps, int n_split) {
+  const int k1 = P.k - 1, ns = n_split > kScanWarps ? n_split : kScanWarps;
+  return D == 64 ? ScanSmem<64>::bytes(P.r, P.group, cps, ns, k1)
+                 : ScanSmem<128>::bytes(P.r, P.group, cps, ns, k1);
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous one in the stream is still running.
+template <typename... Args, typename... Actual>
+cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Actual... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 template <int D, int EB>
 cudaError_t run_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                        int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s) {
-  if (slice_elems(P) == 128)
-    return run_decode_t<D, EB, 128>(P, k_new, v_new, out, idx_out, w_out, ws, s);
-  return run_decode_t<D, EB, 64>(P, k_new, v_new, out, idx_out, w_out, ws, s);
+  cudaError_t e;
+  {
+    const size_t smem = scan_smem(P, D, ScanGeo<D, EB>::CPS, ws.n_split);
+    if ((e = set_smem(scan_kernel<D, EB>, smem)) != cudaSuccess) return e;
+    HILS_PROFILE("decode.scan", s);
+    scan_kernel<D, EB><<<dim3(ws.n_split, P.Hkv, P.B), kScanThreads, smem, s>>>(
+        P, k_new, v_new, ws, idx_out, w_out);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    const size_t kv_bytes = (size_t)2 * kChunk * (D + (EB == 2 ? 8 : 4)) * EB;
+    if ((e = set_smem(attend_kernel<D, EB>, kv_bytes)) != cudaSuccess) return e;
+    HILS_PROFILE("decode.attend", s);
+    e = launch_pdl(attend_kernel<D, EB>, dim3(P.k, P.Hq, P.B), dim3(kAttThreads), kv_bytes, s, P,
+                   ws, out);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+int chunks_per_split(const Params& P) {
+  if (P.dtype == HILS_BF16) return P.d == 64 ? ScanGeo<64, 2>::CPS : ScanGeo<128, 2>::CPS;
+  return P.d == 64 ? ScanGeo<64, 4>::CPS : ScanGeo<128, 4>::CPS;
 }
 
 }  // namespace
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// One CTA scans 256 thread slices, i.e. chunks_per_split chunks.
-static void pick_split(const Params& P, DecodeWs* w) {
-  const int row = P.Hkv * P.d;
-  int cps = row > 0 ? kScanThreads * slice_elems(P) / row : 1;
-  if (cps < 1) cps = 1;
-  w->chunks_per_split = cps;
-  w->n_split = (P.max_chunks + cps - 1) / cps;
-  if (w->n_split < 1) w->n_split = 1;
-}
-
 size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
   DecodeWs w{};
-  pick_split(P, &w);
+  w.chunks_per_split = chunks_per_split(P);
+  w.n_split = (P.max_chunks + w.chunks_per_split - 1) / w.chunks_per_split;
+  if (w.n_split < 1) w.n_split = 1;
   const int K = P.k - 1 > 0 ? P.k - 1 : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -671,28 +612,22 @@ size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
     off += align256(bytes);
     return p;
   };
-  const int64_t nc = (int64_t)P.B * w.n_split * P.Hq * K;
+  const int64_t nc = (int64_t)P.B * P.Hq * w.n_split * K;
   w.cand_s = (float*)take(sizeof(float) * nc);
   w.cand_j = (int32_t*)take(sizeof(int32_t) * nc);
-  w.best = (float*)take(sizeof(float) * (int64_t)P.B * P.Hq * w.n_split);
-  w.s_own = (float*)take(sizeof(float) * (int64_t)P.B * P.Hq);
   w.idx = (int32_t*)take(sizeof(int32_t) * P.B * P.Hq * P.k);
   w.w = (float*)take(sizeof(float) * P.B * P.Hq * P.k);
   w.part = (float*)take(sizeof(float) * P.B * P.Hq * P.k * P.d);
   w.tickets = (int32_t*)take(sizeof(int32_t) * (2 * P.B * P.Hq + P.B));
-  w.tpos = (int32_t*)take(sizeof(int32_t) * P.B);
   if (out) *out = w;
   return off;
 }
 
-size_t decode_scan_smem_bytes(const Params& P) {
-  DecodeWs w{};
-  pick_split(P, &w);
-  return scan_smem(P, w, P.d);
-}
 
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,
-                          int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s) {
+                          int32_t* idx_out, float* w_out, const DecodeWs& ws_in, cudaStream_t s) {
+  DecodeWs ws = ws_in;
+  ws.append = k_new != nullptr;
   if (P.dtype == HILS_BF16)
     return P.d == 64 ? run_decode<64, 2>(P, k_new, v_new, out, idx_out, w_out, ws, s)
                      : run_decode<128, 2>(P, k_new, v_new, out, idx_out, w_out, ws, s);

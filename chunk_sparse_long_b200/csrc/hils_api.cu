@@ -6,6 +6,10 @@
 #include <cstring>
 #include <string>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "hils_common.cuh"
 
 namespace {
@@ -63,6 +67,8 @@ int check_config(const hils_config* c, hils::Params* P) {
 int check_calib(const hils_config* c, const float* A, const float* B, hils::Params* P) {
   if (c->calib_rank > 0 && (!A || !B))
     return fail(HILS_ERR_INVALID_ARG, "calib_rank %d needs A and B", c->calib_rank);
+  if (c->calib_rank > 0 && (!aligned16(A) || !aligned16(B)))
+    return fail(HILS_ERR_INVALID_ARG, "A and B must be 16-byte aligned");
   P->A = A;
   P->Bm = B;
   return HILS_OK;
@@ -212,6 +218,9 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
   P.pos0 = 0;
   hils::DecodeWs w{};
   const size_t need = hils::decode_ws_bytes(P, &w, nullptr);
+  if (w.n_split > hils::kMaxSplitLists)
+    return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
+                hils::kMaxSplitLists, P.max_chunks, w.n_split);
   if (!ws || ws_bytes < need)
     return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
   if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
@@ -246,4 +255,18 @@ const char* hils_version(void) { return "hils-b200 0.1.0 sm_100a"; }
 namespace hils {
 // Lets other translation units of the library report through hils_last_error().
 void record_error(const char* msg) { g_last_error = msg; }
+
+cudaError_t set_smem_impl(const void* func, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& have = done[{func, dev}];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
 }  // namespace hils

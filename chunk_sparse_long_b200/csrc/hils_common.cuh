@@ -14,6 +14,7 @@ constexpr int kChunk = 64;       // chunk_size the kernels are written for
 constexpr int kItemPairs = 512;  // pairs per tensor-core attention work item (4 tiles of 128)
 constexpr int kMaxTopK = 32;
 constexpr int kMaxRank = 64;
+constexpr int kMaxSplitLists = 512;  // decode: chunk ranges per (sequence, KV head), at most
 constexpr int kScoreTileRows = 128;  // query rows per landmark-scoring tile
 constexpr int kScoreBlock = 128;     // landmark chunks per scoring block
 
@@ -140,6 +141,14 @@ class ProfileScope {
 // Sets the message hils_last_error() returns on this thread.
 void record_error(const char* msg);
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, calling the runtime only the first time a larger value is needed.
+cudaError_t set_smem_impl(const void* func, size_t bytes);
+template <typename F>
+cudaError_t set_smem(F* func, size_t bytes) {
+  return set_smem_impl(reinterpret_cast<const void*>(func), bytes);
+}
+
 // ---- launchers (each returns cudaError_t of its launches) -----------------
 cudaError_t launch_score(const Params& P, float* scores, int n_cols, cudaStream_t s);
 cudaError_t launch_topk(const Params& P, const float* scores, int n_cols, int32_t* idx, float* w,
@@ -175,16 +184,15 @@ cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const
                            const PrefillWs& ws, cudaStream_t s);
 
 struct DecodeWs {
-  float* cand_s;       // [B][n_split][Hq][k-1] each split's best candidates, best first
-  int32_t* cand_j;     // same
-  float* best;         // [B][Hq][n_split] each split's best score (-inf if none)
-  float* s_own;        // [B][Hq] the own chunk's score
-  int32_t* idx;        // [B][Hq][k]
-  float* w;            // [B][Hq][k]
-  float* part;         // [B][Hq][k][d]
-  int32_t* tickets;    // [B][Hq] scan tickets, [B][Hq] attention tickets, [B] head-done
-  int32_t* tpos;       // [B] position of this step's query
+  float* cand_s;       // [B][Hq][n_split][k-1] each range's best candidates, best first
+  int32_t* cand_j;     // same (-1: none)
+  int32_t* idx;        // [B][Hq][k] selected chunks (slot 0 = own)
+  float* w;            // [B][Hq][k] fusion weights
+  float* part;         // [B][Hq][k][d] weighted per-slot outputs
+  int32_t* tickets;    // [B][Hkv] scan tickets, at B*Hq: [B][Hq] attention tickets, at
+                       // 2*B*Hq: [B] heads done; all return to zero after each step
   int n_split, chunks_per_split;
+  int append;          // k_new / v_new given
 };
 size_t decode_ws_bytes(const Params& P, DecodeWs* ws, char* base);
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,

@@ -407,8 +407,7 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
     if ((e = launch_select_tc(P, ws, ws.idx, ws.w, s)) != cudaSuccess) return e;
   } else {
     const size_t ssm = select_smem<D>(P.r);
-    e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)ssm);
+    e = set_smem(select_kernel<D>, ssm);
     if (e != cudaSuccess) return e;
     dim3 sg((unsigned)((P.L + kSelThreads - 1) / kSelThreads), P.Hq, P.B);
     {
@@ -425,12 +424,10 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
     const int64_t nvis_max = min((int64_t)P.max_chunks, (P.pos0 + P.L - 1) / kChunk + 1);
     const size_t hsm = sizeof(int32_t) * 2 * (size_t)nvis_max;
     if (nvis_max <= kHistMax) {
-      if ((e = cudaFuncSetAttribute(bucket_scatter_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm)) !=
+      if ((e = set_smem(bucket_scatter_kernel, hsm)) !=
           cudaSuccess)
         return e;
-      if ((e = cudaFuncSetAttribute(bucket_count_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm)) !=
+      if ((e = set_smem(bucket_count_kernel, hsm)) !=
           cudaSuccess)
         return e;
       const dim3 bgrid((unsigned)((P.L + kBucketRows - 1) / kBucketRows), P.Hkv, P.B);
@@ -453,8 +450,7 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
   if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws.idx, ws.w, ws, s);
   if ((e = cudaMemsetAsync(ws.acc, 0, sizeof(float) * rows * D, s)) != cudaSuccess) return e;
   constexpr size_t asm_ = attend_smem<D>();
-  e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)asm_);
+  e = set_smem(attend_kernel<D>, asm_);
   if (e != cudaSuccess) return e;
   {
     HILS_PROFILE("prefill.attend", s);

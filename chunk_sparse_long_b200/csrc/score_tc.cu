@@ -505,8 +505,7 @@ cudaError_t run_calib(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, in
                       cudaStream_t s) {
   constexpr int NR = RP <= 32 ? 2 : 1;
   const size_t sm = sizeof(float) * 2 * D * RP;
-  cudaError_t e = cudaFuncSetAttribute(calib_kernel<D, RP, NR>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  cudaError_t e = set_smem(calib_kernel<D, RP, NR>, sm);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_kernel<D, RP, NR>, kThrS, sm);
@@ -539,8 +538,7 @@ cudaError_t run_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, fl
   }
   if (e != cudaSuccess) return e;
 
-  e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)Lay::kSmem);
+  e = set_smem(score_tc_kernel<D>, Lay::kSmem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<D>, kThrS,

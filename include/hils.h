@@ -86,7 +86,7 @@ size_t hils_workspace_size(const hils_config* cfg, int op, int64_t q_len, int32_
 
 /* a1 + a2 materialised, for tests and small inputs.
  * q       [B][q_len][Hq][d]  queries at positions q_pos0 .. q_pos0+q_len-1
- * A, B    float32 [d][r], [r][d] (ignored when calib_rank == 0)
+ * A, B    float32 [d][r], [r][d], 16-byte aligned (ignored when calib_rank == 0)
  * scores  float32 [B][q_len][Hq][n_cols]; column j holds s_j for j <= floor(pos/S)
  *         and -inf after it.  Requires floor((q_pos0+q_len-1)/S) < n_cols <= max_chunks. */
 int hils_score(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0, const float* A,

@@ -101,6 +101,9 @@ def test_decode_argument_checks(lib):
     assert status_of(hils.decode, c, FAKE, None, None, FAKE, FAKE, cache(seq_lens=None), FAKE, None, None, FAKE, ws, 0)[0] == 1
     assert status_of(hils.decode, c, FAKE, None, None, FAKE, FAKE, cache(), FAKE, None, None, FAKE, ws - 1, 0)[0] == 3
     assert status_of(hils.decode, cfg(n_q_heads=128, n_kv_heads=2), FAKE, None, None, FAKE, FAKE, cache(), FAKE, None, None, FAKE, 1 << 30, 0)[0] == 2
+    # the calibration matrices are read in 16-byte units
+    st, msg = status_of(hils.decode, c, FAKE, None, None, FAKE + 4, FAKE, cache(), FAKE, None, None, FAKE, ws, 0)
+    assert st == 1 and "aligned" in msg
 
 
 def test_score_and_topk_argument_checks(lib):

@@ -48,6 +48,25 @@ def peaks():
 
 
 # ----------------------------------------------------------------- work counts
+# DRAM traffic of the attention kernel from one ncu capture on prefill_16k_gqa
+# (dram__bytes_read.sum + dram__bytes_write.sum = 4.316 GB for 15.76M pairs),
+# per (row, slot) pair; it grows with the pairs.  Valid only for the kernel
+# source it was taken on (sha256 below); otherwise the bench reports null.
+ATTN_TRAFFIC = {"file": "chunk_sparse_long_b200/csrc/attn_tc.cu",
+                "sha256": "8c50e4198e4cc5ff65c6ff9e218bdd09c7e13c08adb339667bf9bc9261b98bb9",
+                "bytes_per_pair": 4.316e9 / 15.76e6}
+
+
+def attn_traffic(pairs: float):
+    import hashlib
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), ATTN_TRAFFIC["file"])
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return ATTN_TRAFFIC["bytes_per_pair"] * pairs if digest == ATTN_TRAFFIC["sha256"] else None
+
+
 def prefill_counts(w: hi.Workload) -> dict:
     """Algorithmic work of one prefill step (all rows of all sequences)."""
     S, k, d, r = w.chunk_size, w.top_k, w.head_dim, w.calib_rank
@@ -451,9 +470,12 @@ def main():
     else:
         work, what = counts["attention_flop"], "useful attention flop"
     achieved = work / (dom_ms / 1e3) / 1e12
+    traffic = attn_traffic(counts["pairs"]) if dom_name == "prefill.attend_tc" else None
     roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
                 "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                "frac": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,
+                "traffic_source": "ncu dram bytes on prefill_16k_gqa scaled by (row, slot) pairs"
+                                  if traffic else None,
                 "work_per_launch": work, "work": what,
                 "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)"}
     result = {

@@ -170,6 +170,7 @@ struct PrefillWs {
   float* scores;     // bf16: landmark scores, score_cols columns per (sequence, head)
   int64_t score_cols;
   int4* items;       // [max_tiles] (key, first pair, end pair, 0) of every work item
+  int2* scan_totals; // [ceil(n_keys / 1024)] (pairs, items) of each block of keys
   int n_keys;
   int n_win;         // query windows per sequence
   int64_t win_rows;  // query positions per window

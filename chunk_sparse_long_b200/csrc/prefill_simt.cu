@@ -272,45 +272,99 @@ __global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, in
 
 // Exclusive scans of the bucket sizes (pair offsets) and of their work items
 // (ceil(count / tile_pairs) each), and (key, first pair, end pair) of every
-// work item.
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int n_keys,
-                                                    int tile_pairs, int32_t* offsets,
-                                                    int32_t* tile_off, int32_t* cursor,
-                                                    int4* items) {
-  __shared__ int32_t sp[1024], stl[1024];
-  const int t = threadIdx.x;
-  const int per = (n_keys + 1023) / 1024;
-  const int k0 = min(t * per, n_keys), k1 = min(k0 + per, n_keys);
-  int32_t ps = 0, ts = 0;
-  for (int key = k0; key < k1; ++key) {
-    ps += counts[key];
-    ts += (counts[key] + tile_pairs - 1) / tile_pairs;
+// work item: two passes over blocks of kScanBlock keys.  Pass 1 writes every
+// block's pair and item totals; pass 2 gives each block its prefix (the sum
+// of the earlier blocks' totals) and scans inside the block.
+constexpr int kScanBlock = 1024;
+
+__device__ __forceinline__ int2 block_sum_pairs_items(int2 v, int2* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
   }
-  sp[t] = ps;
-  stl[t] = ts;
+  if (lane == 0) red[warp] = v;
   __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {
-    int32_t a = t >= o ? sp[t - o] : 0, c = t >= o ? stl[t - o] : 0;
-    __syncthreads();
-    sp[t] += a;
-    stl[t] += c;
-    __syncthreads();
+  int2 t = make_int2(0, 0);
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : make_int2(0, 0);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      t.x += __shfl_xor_sync(0xffffffffu, t.x, o);
+      t.y += __shfl_xor_sync(0xffffffffu, t.y, o);
+    }
   }
-  int32_t po = sp[t] - ps, to = stl[t] - ts;
-  for (int key = k0; key < k1; ++key) {
-    const int32_t c = counts[key];
-    const int32_t nt = (c + tile_pairs - 1) / tile_pairs;
+  return t;   // valid in warp 0
+}
+
+__global__ void __launch_bounds__(kScanBlock) scan_totals_kernel(const int32_t* counts, int n_keys,
+                                                                 int tile_pairs, int2* totals) {
+  __shared__ int2 red[32];
+  const int key = blockIdx.x * kScanBlock + threadIdx.x;
+  const int c = key < n_keys ? counts[key] : 0;
+  const int2 t = block_sum_pairs_items(make_int2(c, (c + tile_pairs - 1) / tile_pairs), red);
+  if (threadIdx.x == 0) totals[blockIdx.x] = t;
+}
+
+__global__ void __launch_bounds__(kScanBlock) scan_kernel(const int32_t* counts, int n_keys,
+                                                          int tile_pairs, const int2* totals,
+                                                          int32_t* offsets, int32_t* tile_off,
+                                                          int32_t* cursor, int4* items) {
+  __shared__ int2 red[32];
+  __shared__ int2 base_sh;
+  __shared__ int2 wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // prefix of this block: the totals of the blocks before it
+  int2 pre = make_int2(0, 0);
+  for (int x = tid; x < (int)blockIdx.x; x += kScanBlock) {
+    const int2 t = totals[x];
+    pre.x += t.x;
+    pre.y += t.y;
+  }
+  const int2 bt = block_sum_pairs_items(pre, red);
+  if (tid == 0) base_sh = bt;
+  // inclusive scan of (pairs, items) inside the block
+  const int key = blockIdx.x * kScanBlock + tid;
+  const int c = key < n_keys ? counts[key] : 0;
+  const int nt = (c + tile_pairs - 1) / tile_pairs;
+  int2 v = make_int2(c, nt);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ax = __shfl_up_sync(0xffffffffu, v.x, o), ay = __shfl_up_sync(0xffffffffu, v.y, o);
+    if (lane >= o) {
+      v.x += ax;
+      v.y += ay;
+    }
+  }
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int2 w = lane < (kScanBlock >> 5) ? wsum[lane] : make_int2(0, 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ax = __shfl_up_sync(0xffffffffu, w.x, o), ay = __shfl_up_sync(0xffffffffu, w.y, o);
+      if (lane >= o) {
+        w.x += ax;
+        w.y += ay;
+      }
+    }
+    wsum[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  const int2 wp = warp > 0 ? wsum[warp - 1] : make_int2(0, 0);
+  const int po = base_sh.x + wp.x + v.x - c;    // exclusive pair offset
+  const int to = base_sh.y + wp.y + v.y - nt;   // exclusive item offset
+  if (key < n_keys) {
     offsets[key] = po;
     cursor[key] = po;
     tile_off[key] = to;
     for (int u = 0; u < nt; ++u)
       items[to + u] = make_int4(key, po + u * tile_pairs, min(po + (u + 1) * tile_pairs, po + c), 0);
-    po += c;
-    to += nt;
-  }
-  if (t == 1023) {
-    offsets[n_keys] = sp[1023];
-    tile_off[n_keys] = stl[1023];
+    if (key == n_keys - 1) {
+      offsets[n_keys] = po + c;
+      tile_off[n_keys] = to + nt;
+    }
   }
 }
 
@@ -433,15 +487,23 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
       const dim3 bgrid((unsigned)((P.L + kBucketRows - 1) / kBucketRows), P.Hkv, P.B);
       const Windows W{ws.n_win, ws.win_rows};
       bucket_count_kernel<<<bgrid, 256, hsm / 2, s>>>(P, ws.idx, ws.counts, W);
-      scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
-                                     ws.cursor, ws.items);
+      {
+        const unsigned nb = (unsigned)((ws.n_keys + kScanBlock - 1) / kScanBlock);
+        scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
+        scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
+                                              ws.offsets, ws.tile_off, ws.cursor, ws.items);
+      }
       bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, W);
     } else {
       const unsigned pb = (unsigned)((n_pairs + 255) / 256);
       const Windows W{ws.n_win, ws.win_rows};
       count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs, W);
-      scan_kernel<<<1, 1024, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.offsets, ws.tile_off,
-                                     ws.cursor, ws.items);
+      {
+        const unsigned nb = (unsigned)((ws.n_keys + kScanBlock - 1) / kScanBlock);
+        scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
+        scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
+                                              ws.offsets, ws.tile_off, ws.cursor, ws.items);
+      }
       scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, n_pairs, W);
     }
   }
@@ -522,6 +584,7 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.win_rows = win_rows;
   w.max_tiles = (n_pairs + kTilePairs - 1) / kTilePairs + n_keys;
   w.items = (int4*)take(sizeof(int4) * w.max_tiles);
+  w.scan_totals = (int2*)take(sizeof(int2) * ((n_keys + 1023) / 1024));
   if (ws) *ws = w;
   return off;
 }

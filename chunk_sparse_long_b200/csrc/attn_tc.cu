@@ -76,7 +76,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
   __shared__ uint64_t q_full[NS], q_empty[NS], kv_full[2], kv_empty[2];
   __shared__ uint64_t s_full[2], sm_done[2], o_full[2], o_free[2];
   __shared__ TileDesc desc[NS];
-  __shared__ int32_t meta_r[NS][kRows];   // query row of each tile row (-1: unused)
   __shared__ uint8_t meta_nk[NS][kRows];  // keys visible to it (64, or fewer in the own chunk)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -144,7 +143,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
     int4 info = item_info(item);
     int4 info_next = item_info(item + stride);
     int32_t page_raw = raw_page(item, info);
-    int32_t pid_next = (item < n_items && info.y + my_row < info.z) ? ws.pairs[info.y + my_row] : -1;
+    // (query row, position) of this thread's row in the next tile; x = -1: unused row
+    int2 pi_next = (item < n_items && info.y + my_row < info.z) ? ws.pinfo[info.y + my_row]
+                                                                : make_int2(-1, 0);
     int n = 0;
     bool ok = true;
     for (int item_idx = 0;; ++item_idx) {
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         }
         const int tile_base = p0 + t * kRows;
         const int nv = min(kRows, p1 - tile_base);
-        const int32_t pid = pid_next;
+        const int2 pi = pi_next;
         // this row's pair in the next tile: of this item, or the first tile of the next
         {
           int pn, pend;
@@ -208,25 +209,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
             pn = info_next.y + my_row;
             pend = next_item < n_items ? info_next.z : 0;
           }
-          pid_next = pn < pend ? ws.pairs[pn] : -1;
+          pi_next = pn < pend ? ws.pinfo[pn] : make_int2(-1, 0);
         }
+        const int32_t my_r = pi.x;
         {
-          int32_t r = -1;
           int nk = kChunk;
-          if (pid >= 0) {
-            r = pid / P.k;
-            const int64_t pos = P.pos0 + ((int64_t)r / P.Hq) % P.L;
+          if (my_r >= 0) {
+            const int64_t pos = P.pos0 + pi.y;
             if (pos / kChunk == j) nk = (int)(pos - (int64_t)j * kChunk + 1);
           }
-          meta_r[st][my_row] = r;
           meta_nk[st][my_row] = (uint8_t)nk;
         }
-        __syncwarp();
         const uint32_t qdst = sbase + Lay::kQ + st * Lay::kQBytes;
 #pragma unroll
         for (int it = 0; it < 32 / RPI; ++it) {
           const int row = warp * 32 + it * RPI + lane / CPR, c = lane % CPR;
-          const int32_t r = meta_r[st][row];
+          const int32_t r = __shfl_sync(0xffffffffu, my_r, it * RPI + lane / CPR);
           const uint16_t* src =
               reinterpret_cast<const uint16_t*>(P.q) + (int64_t)(r >= 0 ? r : 0) * D + c * 8;
           tc::cp_async16(qdst + (uint32_t)(c >> 3) * (kRows * 128) + tc::swz(row, c & 7), src,

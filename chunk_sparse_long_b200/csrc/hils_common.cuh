@@ -161,8 +161,9 @@ struct PrefillWs {
   int32_t* offsets;  // [n_keys + 1] pair offsets
   int32_t* tile_off; // [n_keys + 1] tile offsets
   int32_t* cursor;   // [n_keys]
-  int32_t* pairs;    // [rows * k] pair ids (row * k + slot) in bucket order
+  int32_t* pairs;    // float32 path: [rows * k] pair ids (row * k + slot) in bucket order
   int32_t* inv;      // [rows * k] bucket position of each pair id
+  int2* pinfo;       // bf16 path: [rows * k] (query row, position index) in bucket order
   float* acc;        // [rows][d] float32 accumulator (CUDA-core attention)
   void* partial;     // [rows * k][d] bf16 per-pair O / l in bucket order (tensor-core attention)
   int32_t* queue;    // work-item counter of the persistent attention kernel

@@ -180,14 +180,26 @@ __device__ __forceinline__ int64_t pair_key(const Params& P, Windows W, int64_t 
 // its rows can see, then added to the global counts once per nonzero bin.
 // Every pair of a position i of the group's heads is one run of group * k
 // consecutive idx entries.
+// x / d for small x (x, d < 2^16) by a multiply-high with m = 2^32 / d rounded
+// up; d = 1 (where m would not fit) returns x.
+struct SmallDiv {
+  uint32_t d, m;
+  __device__ __forceinline__ explicit SmallDiv(uint32_t dd)
+      : d(dd), m(dd > 1 ? 0xFFFFFFFFu / dd + 1u : 0u) {}
+  __device__ __forceinline__ uint32_t div(uint32_t x) const { return d > 1 ? __umulhi(x, m) : x; }
+};
+
 __device__ __forceinline__ void block_hist(const Params& P, const int32_t* idx, int32_t* hist,
                                            int nvis, int64_t i0, int64_t i1, int b, int g,
                                            bool check) {
   const int per_i = P.group * P.k;
+  const SmallDiv dv(per_i);
   const int n = (int)(i1 - i0) * per_i;
+  const int32_t* base = idx + (((int64_t)b * P.L + i0) * P.Hq + g * P.group) * P.k;
+  const int64_t row_stride = (int64_t)P.Hq * P.k;   // idx entries from one position to the next
   for (int f = threadIdx.x; f < n; f += blockDim.x) {
-    const int64_t i = i0 + f / per_i;
-    const int32_t j = idx[(((int64_t)b * P.L + i) * P.Hq + g * P.group) * P.k + f % per_i];
+    const int ii = (int)dv.div((uint32_t)f);
+    const int32_t j = base[ii * row_stride + (f - ii * per_i)];
     if (j < 0) continue;
     if (j >= nvis) {
       if (check) set_device_error(kErrChunk);
@@ -216,7 +228,7 @@ __global__ void __launch_bounds__(256) bucket_count_kernel(Params P, const int32
 // each bucket, shared-memory atomics place the pairs inside it.
 __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int32_t* idx,
                                                              int32_t* cursor, int32_t* pairs,
-                                                             int32_t* inv, Windows W) {
+                                                             int32_t* inv, int2* pinfo, Windows W) {
   extern __shared__ int32_t hist[];
   const int b = blockIdx.z, g = blockIdx.y;
   const int64_t i0 = (int64_t)blockIdx.x * kBucketRows, i1 = min(i0 + kBucketRows, P.L);
@@ -234,14 +246,23 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int
   }
   __syncthreads();
   const int per_i = P.group * P.k;
+  const SmallDiv dv(per_i), dk(P.k);
   const int n = (int)(i1 - i0) * per_i;
+  const bool rows_out = pinfo != nullptr;   // tensor-core path: (row, position) per pair
   for (int f = threadIdx.x; f < n; f += blockDim.x) {
-    const int64_t p = (((int64_t)b * P.L + i0 + f / per_i) * P.Hq + g * P.group) * P.k + f % per_i;
+    const int ii = (int)dv.div((uint32_t)f);
+    const int q = f - ii * per_i;                                        // head-in-group * k + slot
+    const int64_t i = i0 + ii;
+    const int64_t row0 = ((int64_t)b * P.L + i) * P.Hq + g * P.group;   // first row of the group
+    const int64_t p = row0 * P.k + q;
     const int32_t j = idx[p];
     if (j < 0 || j >= nvis) continue;
     const int32_t at = base[j] + atomicAdd(&hist[j], 1);
-    pairs[at] = (int32_t)p;
     inv[p] = at;
+    if (rows_out)
+      pinfo[at] = make_int2((int32_t)(row0 + dk.div((uint32_t)q)), (int32_t)i);
+    else
+      pairs[at] = (int32_t)p;
   }
 }
 
@@ -260,14 +281,19 @@ __global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int6
 }
 
 __global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, int32_t* pairs,
-                               int32_t* inv, int64_t n_pairs, Windows W) {
+                               int32_t* inv, int2* pinfo, int64_t n_pairs, Windows W) {
   const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= n_pairs) return;
   const int32_t j = idx[p];
   if (j < 0 || j >= P.max_chunks) return;
   const int32_t at = atomicAdd(&cursor[pair_key(P, W, p, j)], 1);
-  pairs[at] = (int32_t)p;
   inv[p] = at;
+  if (pinfo) {
+    const int64_t r = p / P.k;
+    pinfo[at] = make_int2((int32_t)r, (int32_t)((r / P.Hq) % P.L));
+  } else {
+    pairs[at] = (int32_t)p;
+  }
 }
 
 // Exclusive scans of the bucket sizes (pair offsets) and of their work items
@@ -493,7 +519,8 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
         scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
                                               ws.offsets, ws.tile_off, ws.cursor, ws.items);
       }
-      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, W);
+      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv,
+                                                    P.dtype == HILS_BF16 ? ws.pinfo : nullptr, W);
     } else {
       const unsigned pb = (unsigned)((n_pairs + 255) / 256);
       const Windows W{ws.n_win, ws.win_rows};
@@ -504,7 +531,8 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
         scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
                                               ws.offsets, ws.tile_off, ws.cursor, ws.items);
       }
-      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv, n_pairs, W);
+      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv,
+                                        P.dtype == HILS_BF16 ? ws.pinfo : nullptr, n_pairs, W);
     }
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -556,7 +584,10 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.offsets = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
-  w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  if (P.dtype == HILS_BF16)
+    w.pinfo = (int2*)take(sizeof(int2) * n_pairs);
+  else
+    w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
   w.inv = (int32_t*)take(sizeof(int32_t) * n_pairs);
   if (P.dtype == HILS_BF16) {
     // the landmark scores and q~ images are dead before the attention writes

@@ -49,12 +49,12 @@ def peaks():
 
 # ----------------------------------------------------------------- work counts
 # DRAM traffic of the attention kernel from one ncu capture on prefill_16k_gqa
-# (dram__bytes_read.sum + dram__bytes_write.sum = 4.316 GB for 15.76M pairs),
+# (dram__bytes_read.sum + dram__bytes_write.sum = 4.391 GB for 15.76M pairs),
 # per (row, slot) pair; it grows with the pairs.  Valid only for the kernel
 # source it was taken on (sha256 below); otherwise the bench reports null.
 ATTN_TRAFFIC = {"file": "chunk_sparse_long_b200/csrc/attn_tc.cu",
-                "sha256": "8c50e4198e4cc5ff65c6ff9e218bdd09c7e13c08adb339667bf9bc9261b98bb9",
-                "bytes_per_pair": 4.316e9 / 15.76e6}
+                "sha256": "b0d9c1b9dec78ed8fe99932cd1dba126cc85deb80224227a1c6255a20ca250ae",
+                "bytes_per_pair": 4.391e9 / 15.76e6}
 
 
 def attn_traffic(pairs: float):

@@ -362,6 +362,28 @@ def oracle_prefill_sample(wl, budget_s: float, rng_seed: int = 0):
 
 
 # ----------------------------------------------------------------- main
+def dist_ops(backend: str, device: str):
+    """(barrier, maxreduce) over the initialised process group: maxreduce(x) is
+    the maximum of x over all ranks (the step time of a weakly scaled run)."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        dist.barrier()
+
+    def maxreduce(x):
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, maxreduce
+
+
+def weak_scaling_value(units_per_rank: float, n_ranks: int, step_ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own units in the step,
+    and the step takes as long as the slowest rank."""
+    return units_per_rank * n_ranks / (step_ms_max / 1e3)
+
+
 def dist_setup(torch):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -372,14 +394,7 @@ def dist_setup(torch):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
-
-        def barrier():
-            dist.barrier()
-
-        def maxreduce(x):
-            t = torch.tensor([x], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
+        barrier, maxreduce = dist_ops("nccl", "cuda")
         return ws, rank, barrier, maxreduce
     torch.cuda.set_device(local)
     return 1, 0, (lambda: None), (lambda x: x)
@@ -457,7 +472,7 @@ def main():
     torch.cuda.synchronize()
     ms, phases, clocks, _keep = time_prefill(hils, torch, wl, args.steps, args.warmup, barrier,
                                              maxreduce)
-    value = tokens_per_rank * nworld / (ms / 1e3)
+    value = weak_scaling_value(tokens_per_rank, nworld, ms)
     pk, pk_src = peaks()
     # dominant kernel of the prefill step
     dom = max(phases.items(), key=lambda kv: kv[1][0])
@@ -491,7 +506,7 @@ def main():
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_prefill_e2e(hils, torch, wl, max(1, min(args.steps, 3)), 1)
         e2e_ms = maxreduce(e2e_ms)
-        result["e2e"] = {"value": tokens_per_rank * nworld / (e2e_ms / 1e3), "unit": "tok/s",
+        result["e2e"] = {"value": weak_scaling_value(tokens_per_rank, nworld, e2e_ms), "unit": "tok/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     del wl
     torch.cuda.empty_cache()

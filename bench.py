@@ -36,7 +36,7 @@ import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_KERNELS_PER_STEP = 8   # calib, score, select, bucket count, scan, scatter, attend, merge (bf16)
-DECODE_KERNELS_PER_STEP = 3    # prep (append, calibration), scan (+selection), attend (+merge)
+DECODE_KERNELS_PER_STEP = 2    # scan (append, calibration, scores, selection), attend (+merge)
 
 
 def peaks():
@@ -527,7 +527,7 @@ def main():
             "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3 for k, v in dph.items()},
             # the step's kernels overlap (programmatic dependent launch), so the
             # roofline is taken over the whole step: its algorithmic bytes / step time
-            "roofline": {"bound": "hbm", "kernel": "decode step (prep + scan + attend, overlapped)",
+            "roofline": {"bound": "hbm", "kernel": "decode step (scan + attend, overlapped)",
                          "achieved": tot / (us / 1e6) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"], "traffic": None,
                          "peak_source": f"{pk_src} HBM copy bandwidth"},

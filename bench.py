@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_KERNELS_PER_STEP = 8   # calib, score, select, bucket count, scan, scatter, attend, merge (bf16)
+PREFILL_KERNELS_PER_STEP = 8   # calib, score+select, bucket count, scan totals, scan, scatter, attend, merge (bf16)
 DECODE_KERNELS_PER_STEP = 2    # scan (append, calibration, scores, selection), attend (+merge)
 
 
@@ -480,7 +480,7 @@ def main():
     dom_ms = dom_ms_total / max(1, dom_launches)
     if dom_name.startswith("prefill.attend"):
         work, what = counts["attention_flop"], "useful attention flop (QK^T + PV over selected keys)"
-    elif dom_name.startswith("prefill.select"):
+    elif dom_name.startswith("prefill.score_select"):
         work, what = counts["score_flop"], "useful landmark-scoring flop (q~ . landmark, causal chunks)"
     else:
         work, what = counts["attention_flop"], "useful attention flop"

@@ -18,27 +18,11 @@ constexpr int kMaxSplitLists = 512;  // decode: chunk ranges per (sequence, KV h
 constexpr int kScoreTileRows = 128;  // query rows per landmark-scoring tile
 constexpr int kScoreBlock = 128;     // landmark chunks per scoring block
 
-// Landmark-score workspace of the tensor-core prefill: the tiles of 128 query
-// rows of one (sequence, head) are stored one after another, tile t holding
-// score_tile_blocks(t) blocks of 128 chunk columns (enough for the last
-// causally visible chunk of its last row).
+// Tile t of 128 query rows sees score_tile_blocks(t) blocks of 128 landmark
+// chunks (enough for the last causally visible chunk of its last row).
 __host__ __device__ inline int64_t score_tile_blocks(int64_t L, int64_t pos0, int64_t t) {
   const int64_t last = (t + 1) * kScoreTileRows < L ? (t + 1) * kScoreTileRows - 1 : L - 1;
   return (pos0 + last) / ((int64_t)kChunk * kScoreBlock) + 1;
-}
-// Columns held by tiles 0 .. t-1.  Every tile before the last one is full, so
-// its block count is floor((t' + c) / M) + 1 with c = floor((pos0 + 127) / 128)
-// and M = 64 chunks-per-block x rows-per-chunk / rows-per-tile; the sum of
-// floor(x / M) over x < n has the closed form M q (q - 1) / 2 + q (n mod M).
-__host__ __device__ inline int64_t score_tile_cols_before(int64_t L, int64_t pos0, int64_t t) {
-  (void)L;
-  constexpr int64_t M = (int64_t)kChunk * kScoreBlock / kScoreTileRows;
-  const int64_t c = (pos0 + kScoreTileRows - 1) / kScoreTileRows;
-  auto F = [](int64_t n) {
-    const int64_t q = n / M;
-    return M * q * (q - 1) / 2 + q * (n % M);
-  };
-  return (int64_t)kScoreBlock * (t + F(t + c) - F(c));
 }
 
 // Device error word: kernels OR bits into it when a bounds check fires.
@@ -168,8 +152,6 @@ struct PrefillWs {
   void* partial;     // [rows * k][d] bf16 per-pair O / l in bucket order (tensor-core attention)
   int32_t* queue;    // work-item counter of the persistent attention kernel
   void* qimg;        // bf16: per 128-row tile the three q~ term tiles (shared-memory images)
-  float* scores;     // bf16: landmark scores, score_cols columns per (sequence, head)
-  int64_t score_cols;
   int4* items;       // [max_tiles] (key, first pair, end pair, 0) of every work item
   int2* scan_totals; // [ceil(n_keys / 1024)] (pairs, items) of each block of keys
   int n_keys;

@@ -590,22 +590,14 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
     w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
   w.inv = (int32_t*)take(sizeof(int32_t) * n_pairs);
   if (P.dtype == HILS_BF16) {
-    // the landmark scores and q~ images are dead before the attention writes
-    // its partials, so all three share one region
+    // the q~ images are dead before the attention writes its partials, so
+    // both share one region
     const int64_t T = (P.L + kScoreTileRows - 1) / kScoreTileRows;
-    const int64_t cols = T > 0 ? score_tile_cols_before(P.L, P.pos0, T - 1) +
-                                     (int64_t)kScoreBlock * score_tile_blocks(P.L, P.pos0, T - 1)
-                               : 0;
-    const size_t score_bytes = align256(sizeof(float) * P.B * P.Hq * cols * kScoreTileRows);
     const size_t qimg_bytes = (size_t)P.B * P.Hq * T * 3 * kScoreTileRows * P.d * 2;
     const size_t part_bytes = (size_t)2 * n_pairs * P.d;
-    const size_t region = part_bytes > score_bytes + qimg_bytes ? part_bytes
-                                                                : score_bytes + qimg_bytes;
-    char* reg = take(region);
+    char* reg = take(part_bytes > qimg_bytes ? part_bytes : qimg_bytes);
     w.partial = reg;
-    w.scores = (float*)reg;
-    w.qimg = reg ? reg + score_bytes : nullptr;
-    w.score_cols = cols;
+    w.qimg = reg;
   } else {
     w.acc = (float*)take(sizeof(float) * rows * P.d);
   }

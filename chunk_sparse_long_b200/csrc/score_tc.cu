@@ -1,33 +1,31 @@
 // Prefill calibration, landmark scoring, selection and fusion weights (a1-a4)
-// for bf16 inputs, as three kernels that each run at the occupancy their work
-// wants:
+// for bf16 inputs, as two kernels:
 //
 //   calib_kernel (a1)   one thread per query row computes q~ = q + (qA)B in
 //       float32 and splits it into three bf16 terms hi + mid + lo (each the
 //       bf16 rounding of what is left, so q~ - (hi + mid + lo) is below
 //       2^-27 |q~|).  The terms are written as ready-made shared-memory
 //       images: per 128-row tile, three K-major 128-byte-swizzled tiles.
-//   score_tc_kernel (a2)  persistent; per 128-row tile one bulk copy brings
-//       the three term tiles in, and for every block of 128 causally visible
-//       chunks S = sum over terms Q_term LM^T runs as 3 x d/16 tcgen05.mma
-//       (M = N = 128, float32 accumulate) into one of two TMEM buffers while
-//       the previous block is read back and streamed out as scaled float32
-//       scores.  Landmark blocks are prefetched two steps ahead, across tile
-//       boundaries too.
-//   select_kernel (a3, a4)  one thread per row keeps the k-1 best candidates
-//       j < own in a min-heap of 64-bit keys in shared memory (root = the
-//       worst kept entry), reading its scores 32 columns at a time; candidates
-//       that beat the root are inserted one set bit at a time across the
-//       warp, so lanes do not serialise each other's inserts.  Strict '>'
-//       against the root while j ascends keeps the lower index on ties.  A
-//       heap sort then yields the list best-first, and the softmax of the
-//       own and selected scores gives the weights.
-//
-// Score workspace layout: per (sequence, head), the tiles of 128 rows in
-// order; tile t holds score_tile_blocks(t) * 128 columns (the blocks of chunks
-// its rows can see) as [column / 4][128 rows][4] float32, so a warp reads or
-// writes 512 contiguous bytes per 16-byte access.
+//   score_select_kernel (a2-a4)  persistent; per 128-row tile one bulk copy
+//       brings the three term tiles in, and for every block of 128 causally
+//       visible chunks S = sum over terms Q_term LM^T runs as 3 x d/16
+//       tcgen05.mma (M = N = 128, float32 accumulate) into one of two TMEM
+//       buffers while the previous block is read back.  Landmark blocks are
+//       prefetched two steps ahead, across tile boundaries too.  The scores
+//       never leave the SM: TMEM lane r is query row r of the tile, so the
+//       thread that reads lane r keeps that row's k-1 best candidates j < own
+//       in a min-heap of 64-bit keys in shared memory (root = the worst kept
+//       entry).  Candidates that beat the root are inserted one set bit at a
+//       time across the warp, so lanes do not serialise each other's inserts;
+//       strict '>' against the root while j ascends keeps the lower index on
+//       ties.  After the tile's last block a heap sort yields the list
+//       best-first, and the softmax of the own and selected scores gives the
+//       weights.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cfloat>
+#include <mutex>
 
 #include "hils_common.cuh"
 #include "tc_common.cuh"
@@ -39,8 +37,13 @@ constexpr int kRowsS = kScoreTileRows;  // query rows per tile (M)
 constexpr int kBlk = kScoreBlock;       // landmark chunks per block (N)
 constexpr int kThrS = 128;
 constexpr int kTerms = 3;
-constexpr uint32_t kTmemColsS = 256;  // two S buffers of 128 columns
-constexpr int kLmBufs = 3;            // landmark blocks in flight: prefetch distance 2
+constexpr int kEpiWarps = 4;          // epilogue warps; warp 4 issues the MMAs and loads
+constexpr int kSBufs = 3;             // S buffers of 128 TMEM columns
+constexpr uint32_t kTmemColsS = 512;  // the S buffers, then the class maxima
+constexpr uint32_t kCmaxCol = kSBufs * 128;   // selection pass 0: 64 class maxima per row
+constexpr int kLmBufs = 2;            // landmark blocks in flight: prefetch distance 1
+constexpr int kClasses = 64;          // selection pass 0: one maximum per class j mod 64
+constexpr int kBufCap = 64;           // selection pass 1: collected candidates per row
 
 template <int D>
 struct ScoreLayout {
@@ -49,8 +52,8 @@ struct ScoreLayout {
   static constexpr uint32_t kLmB = kBlk * D * 2;              // one landmark block
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kLm = kQimg;                      // kLmBufs blocks
-  static constexpr uint32_t kEnd = kLm + kLmBufs * kLmB;
-  static constexpr uint32_t kSmem = kEnd + 1024;
+  static constexpr uint32_t kBuf = kLm + kLmBufs * kLmB;    // [kBufCap][kThrS] uint64 keys
+  static constexpr uint32_t kSmem = kBuf + kBufCap * kThrS * 8 + 1024;   // + base alignment
 };
 
 // ---- a1: calibration ------------------------------------------------------
@@ -177,202 +180,10 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
   }
 }
 
-// ---- a2: landmark scores on the tensor cores --------------------------------
-// Landmark block `blk` (chunks blk*128 ..) of (b, g) into a swizzled K-major tile.
-template <int D>
-__device__ __forceinline__ void load_lm_block(const Params& P, uint32_t lm_smem, int b, int g,
-                                              int64_t blk, int64_t last_chunk, int tid) {
-  const uint16_t* base = reinterpret_cast<const uint16_t*>(P.landmarks);
-  for (int x = tid; x < kBlk * (D / 8); x += kThrS) {
-    const int rr = x / (D / 8), c = x % (D / 8);
-    const int64_t j = blk * kBlk + rr;
-    const bool in = j <= last_chunk;
-    const uint16_t* src = base + ((((int64_t)b * P.max_chunks + (in ? j : 0)) * P.Hkv + g) * D + c * 8);
-    tc::cp_async16(lm_smem + (uint32_t)(c >> 3) * (kBlk * 128) + tc::swz(rr, c & 7), src,
-                   in ? 16u : 0u);
-  }
-}
-
-// One (tile, landmark block) step of a CTA's walk over its tiles.
-struct Step {
-  int64_t g;   // tile id ((b * Hq + h) * T + t); >= n_tiles once the walk is over
-  int blk, nblk;
-};
-
-__device__ __forceinline__ void step_set(Step& s, int64_t g, const Params& P, int T,
-                                         int64_t n_tiles) {
-  s.g = g;
-  s.blk = 0;
-  s.nblk = g < n_tiles ? (int)score_tile_blocks(P.L, P.pos0, (int)(g % T)) : 0;
-}
-
-__device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int64_t n_tiles) {
-  if (++s.blk >= s.nblk) step_set(s, s.g + gridDim.x, P, T, n_tiles);
-}
-
-template <int D>
-__device__ __forceinline__ void load_lm_step(const Params& P, uint32_t lm_smem, const Step& s,
-                                             int T, int tid) {
-  const int t = (int)(s.g % T);
-  const int64_t bh = s.g / T;
-  const int b = (int)(bh / P.Hq), g = (int)(bh % P.Hq) / P.group;
-  const int64_t last = min((int64_t)(t + 1) * kRowsS, P.L) - 1;
-  load_lm_block<D>(P, lm_smem, b, g, s.blk, (P.pos0 + last) / kChunk, tid);
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThrS, 1) score_tc_kernel(Params P, const uint8_t* qimg,
-                                                           float* scores, int T, int64_t n_tiles,
-                                                           int64_t cols_per_head) {
-  using Lay = ScoreLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar[2];   // MMAs into S buffer 0 / 1 done
-  __shared__ uint64_t qbar;     // q~ terms of the current tile landed
-  __shared__ uint32_t tmem_sh;
-  __shared__ int abort_sh;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~(uintptr_t)1023);
-  const uint32_t sbase = tc::smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  if ((int64_t)blockIdx.x >= n_tiles) return;
-
-  if (tid == 0) {
-    tc::mbar_init(&bar[0], 1);
-    tc::mbar_init(&bar[1], 1);
-    tc::mbar_init(&qbar, 1);
-    tc::fence_mbar_init();
-    abort_sh = 0;
-  }
-  if (warp == 0) {
-    tc::tmem_alloc(&tmem_sh, kTmemColsS);
-    tc::tmem_relinquish();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = tmem_sh;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  constexpr uint32_t kId = tc::idesc_bf16(kRowsS, kBlk, 0);
-
-  auto load_q = [&](int64_t g) {
-    tc::mbar_arrive_expect_tx(&qbar, Lay::kQimg);
-#pragma unroll
-    for (int term = 0; term < kTerms; ++term)
-      tc::bulk_g2s(sbase + Lay::kQ + term * Lay::kQt, qimg + g * Lay::kQimg + term * Lay::kQt,
-                   Lay::kQt, &qbar);
-  };
-
-  Step cur, pf;
-  step_set(cur, blockIdx.x, P, T, n_tiles);
-  pf = cur;
-  // landmark blocks of the first two steps; exactly one cp.async group per step
-  load_lm_step<D>(P, sbase + Lay::kLm, pf, T, tid);
-  tc::cp_async_commit();
-  step_next(pf, P, T, n_tiles);
-  if (pf.g < n_tiles) {
-    load_lm_step<D>(P, sbase + Lay::kLm + Lay::kLmB, pf, T, tid);
-    step_next(pf, P, T, n_tiles);
-  }
-  tc::cp_async_commit();
-  if (tid == 0) load_q(cur.g);
-
-  uint32_t phase[2] = {0u, 0u}, qphase = 0u;
-  Step prev = cur;   // the step whose scores are drained next
-  int64_t n = 0;     // steps issued so far
-
-  auto wait_mma = [&](int64_t sidx) {
-    const int sb = (int)(sidx & 1);
-    if (!tc::mbar_wait(&bar[sb], phase[sb])) abort_sh = 1;
-    phase[sb] ^= 1;
-    tc::tc_fence_after();
-  };
-  // S buffer of step sidx -> scaled scores of tile st.g, columns st.blk * 128 ..
-  auto drain = [&](int64_t sidx, const Step& st) {
-    const int sb = (int)(sidx & 1);
-    const int t = (int)(st.g % T);
-    const int64_t bh = st.g / T;
-    float4* dst = reinterpret_cast<float4*>(
-        scores + (bh * cols_per_head + score_tile_cols_before(P.L, P.pos0, t) +
-                  (int64_t)st.blk * kBlk) * kRowsS);
-#pragma unroll 1
-    for (int c0 = 0; c0 < kBlk; c0 += 32) {
-      uint32_t sv[32];
-      tc::tmem_ld32(tmem + sb * kBlk + lane_off + c0, sv);
-      tc::tmem_ld_wait();
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float4 v;
-        v.x = __uint_as_float(sv[4 * u]) * P.inv_sqrt_d;
-        v.y = __uint_as_float(sv[4 * u + 1]) * P.inv_sqrt_d;
-        v.z = __uint_as_float(sv[4 * u + 2]) * P.inv_sqrt_d;
-        v.w = __uint_as_float(sv[4 * u + 3]) * P.inv_sqrt_d;
-        __stcs(dst + ((c0 >> 2) + u) * kRowsS + tid, v);
-      }
-    }
-  };
-
-  while (cur.g < n_tiles) {
-    bool drained = false;
-    if (cur.blk == 0 && n > 0) {
-      // new tile: the previous tile's MMAs must finish before its q~ terms are replaced
-      wait_mma(n - 1);
-      if (tid == 0) load_q(cur.g);
-      drain(n - 1, prev);
-      drained = true;
-    }
-    // groups committed so far: steps 0 .. n+1; the one of step n must be complete
-    tc::cp_async_wait<1>();
-    tc::fence_proxy_async();
-    tc::tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      if (cur.blk == 0) {
-        if (!tc::mbar_wait(&qbar, qphase)) abort_sh = 1;
-        qphase ^= 1;
-      }
-      tc::tc_fence_after();
-      const int sb = (int)(n & 1);
-      const uint32_t lm = sbase + Lay::kLm + (uint32_t)(n % kLmBufs) * Lay::kLmB;
-#pragma unroll
-      for (int term = 0; term < kTerms; ++term) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(sbase + Lay::kQ + term * Lay::kQt +
-                                               (kk >> 2) * (kRowsS * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc(lm + (kk >> 2) * (kBlk * 128) + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + sb * kBlk, a, bd, kId, (term | kk) != 0);
-        }
-      }
-      tc::mma_commit(&bar[sb]);
-    }
-    if (n > 0 && !drained) {
-      wait_mma(n - 1);
-      drain(n - 1, prev);
-    }
-    // the landmark buffer of step n-1 is free (its MMAs are done): step n+2 goes there
-    if (pf.g < n_tiles) {
-      load_lm_step<D>(P, sbase + Lay::kLm + (uint32_t)((n + 2) % kLmBufs) * Lay::kLmB, pf, T, tid);
-      step_next(pf, P, T, n_tiles);
-    }
-    tc::cp_async_commit();
-    prev = cur;
-    step_next(cur, P, T, n_tiles);
-    ++n;
-  }
-  wait_mma(n - 1);
-  drain(n - 1, prev);
-
-  if (abort_sh && tid == 0) set_device_error(kErrTimeout);
-  tc::cp_async_wait<0>();
-  tc::tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsS);
-}
-
-// ---- a3/a4: selection and fusion weights -----------------------------------
-// Heap keys: a larger key ranks higher in (score desc, index asc).  The high
-// word is the score's bits mapped to an unsigned order (-0 taken as +0), the
-// low word is ~j.  Key 0 is an empty slot, below every real entry.
+// ---- a2-a4: landmark scores, selection and weights, fused -------------------
+// Keys: a larger key ranks higher in (score desc, index asc).  The high word
+// is the score's bits mapped to an unsigned order (-0 taken as +0), the low
+// word is ~j.  Key 0 is an empty slot, below every real entry.
 __device__ __forceinline__ uint64_t make_key(float s, int j) {
   uint32_t u = __float_as_uint(s + 0.f);
   u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -387,9 +198,8 @@ __device__ __forceinline__ int key_index(uint64_t key) {
   return (int)(0xFFFFFFFFu - (uint32_t)key);
 }
 
-// Places x at the root of the min-heap H[0 .. size) (stride kThrS) and sifts it down.
-__device__ __forceinline__ void sift_root(uint64_t* H, int size, uint64_t x) {
-  int p = 0;
+// Sifts x down from slot p of the min-heap H[0 .. size) (stride kThrS).
+__device__ __forceinline__ void sift_down(uint64_t* H, int size, int p, uint64_t x) {
   for (;;) {
     int c = 2 * p + 1;
     if (c >= size) break;
@@ -408,6 +218,16 @@ __device__ __forceinline__ void sift_root(uint64_t* H, int size, uint64_t x) {
   H[p * kThrS] = x;
 }
 
+// Keeps the best K of the n >= K keys in H[0 .. n) as a min-heap in
+// H[0 .. K): its root is then the K-th best.
+__device__ __forceinline__ void keep_best(uint64_t* H, int n, int K) {
+  for (int p = K / 2 - 1; p >= 0; --p) sift_down(H, K, p, H[p * kThrS]);
+  for (int e = K; e < n; ++e) {
+    const uint64_t x = H[e * kThrS];
+    if (x > H[0]) sift_down(H, K, 0, x);
+  }
+}
+
 // v[x] for a runtime x in 0..31 without dynamic register indexing (select tree).
 __device__ __forceinline__ float pick32(const float (&v)[32], int x) {
   float a[16];
@@ -422,82 +242,425 @@ __device__ __forceinline__ float pick32(const float (&v)[32], int x) {
   return (x & 1) ? a[1] : a[0];
 }
 
-__global__ void __launch_bounds__(kThrS, 6) select_kernel(Params P, const float* scores, int T,
-                                                       int64_t cols_per_head, int32_t* idx,
-                                                       float* w) {
-  extern __shared__ uint64_t heap_sh[];   // [k-1][kThrS]
-  const int tid = threadIdx.x;
-  const int64_t gtile = blockIdx.x;
-  const int t = (int)(gtile % T);
-  const int64_t bh = gtile / T;
-  const int h = (int)(bh % P.Hq), b = (int)(bh / P.Hq);
-  const int64_t i = (int64_t)t * kRowsS + tid;
-  const bool valid = i < P.L;
-  const int64_t own = valid ? (P.pos0 + i) / kChunk : 0;
-  const int64_t i_last = min((int64_t)(t + 1) * kRowsS, P.L) - 1;
-  const int64_t own_max = (P.pos0 + i_last) / kChunk;
-  const float* St = scores + (bh * cols_per_head + score_tile_cols_before(P.L, P.pos0, t)) * kRowsS;
-  const float4* S4 = reinterpret_cast<const float4*>(St);
-  const int K = P.k - 1;
-  uint64_t* H = heap_sh + tid;
-  for (int p = 0; p < K; ++p) H[p * kThrS] = 0;
-  float thr = -INFINITY;   // score of the root (the worst kept entry)
-
-  // candidates j < own <= own_max; the tile holds at least own_max + 1 columns
-  const int64_t n_scan = K > 0 ? own_max : 0;
-#pragma unroll 1
-  for (int64_t c0 = 0; c0 < n_scan; c0 += 32) {
-    float v[32];
+// Bitonic sorting network over N registers, descending.
+template <int N, typename T>
+__device__ __forceinline__ void sort_desc(T (&a)[N]) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 x = __ldcs(S4 + ((c0 >> 2) + u) * kRowsS + tid);
-      v[4 * u] = x.x;
-      v[4 * u + 1] = x.y;
-      v[4 * u + 2] = x.z;
-      v[4 * u + 3] = x.w;
-    }
-    uint32_t m = 0;
+  for (int k = 2; k <= N; k <<= 1) {
 #pragma unroll
-    for (int x = 0; x < 32; ++x) m |= (c0 + x < own && v[x] > thr) ? (1u << x) : 0u;
-    while (__any_sync(0xffffffffu, m != 0)) {
-      if (m) {
-        const int x = __ffs(m) - 1;
-        m &= m - 1;
-        const float s = pick32(v, x);
-        if (s > thr) {
-          sift_root(H, K, make_key(s, (int)(c0 + x)));
-          thr = key_score(H[0]);
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const T x = a[i], y = a[l];
+          const bool sw = ((i & k) == 0) ? (x < y) : (y < x);
+          a[i] = sw ? y : x;
+          a[l] = sw ? x : y;
         }
       }
     }
   }
-  if (!valid) return;
+}
 
-  const float s_own = St[(own >> 2) * (4 * kRowsS) + tid * 4 + (own & 3)];
-  // heap sort: the worst entry moves to the end each round, leaving H best-first
-  for (int n = K - 1; n > 0; --n) {
-    const uint64_t last = H[n * kThrS];
-    H[n * kThrS] = H[0];
-    sift_root(H, n, last);
+// One (tile, pass, landmark block) step of a CTA's walk.  Walk position w
+// covers (sequence, head) w / T and tile T - 1 - w % T: the tiles with the
+// most blocks come first, so the walk ends on short tiles.  Every tile takes
+// two passes over its blocks.
+struct Step {
+  int w;    // walk position; >= n_tiles once the walk is over
+  int bh;   // b * Hq + h
+  int t, pass, blk, nblk;
+};
+
+__device__ __forceinline__ void step_set(Step& s, int w, const Params& P, int T, int n_tiles) {
+  s.w = w;
+  s.pass = 0;
+  s.blk = 0;
+  if (w < n_tiles) {
+    s.bh = (int)((unsigned)w / (unsigned)T);
+    s.t = T - 1 - (w - s.bh * T);
+    s.nblk = (int)score_tile_blocks(P.L, P.pos0, s.t);
+  } else {
+    s.bh = 0;
+    s.t = 0;
+    s.nblk = 0;
   }
-  const float m = K > 0 ? fmaxf(s_own, key_score(H[0])) : s_own;
-  float z = 0.f;
-  for (int p = K - 1; p >= 0; --p) {
-    const uint64_t key = H[p * kThrS];
-    if (key) z += __expf(key_score(key) - m);
+}
+
+__device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int n_tiles) {
+  if (++s.blk < s.nblk) return;
+  if (s.pass == 0) {
+    s.pass = 1;
+    s.blk = 0;
+  } else {
+    step_set(s, s.w + (int)gridDim.x, P, T, n_tiles);
   }
-  z += __expf(s_own - m);
-  const float iz = 1.f / z;
-  const int64_t r = ((int64_t)b * P.L + i) * P.Hq + h;
-  int32_t* ix = idx + r * P.k;
-  float* wr = w + r * P.k;
-  ix[0] = (int32_t)own;
-  wr[0] = __expf(s_own - m) * iz;
-  for (int p = 0; p < K; ++p) {
-    const uint64_t key = H[p * kThrS];
-    ix[p + 1] = key ? key_index(key) : -1;
-    wr[p + 1] = key ? __expf(key_score(key) - m) * iz : 0.f;
+}
+
+// Persistent: each CTA walks its tiles; per tile one bulk copy brings the q~
+// term images in, and per landmark block of 128 chunks (a TMA load from the
+// [B][max_chunks][Hkv][d] landmark tensor, already in the swizzled K-major
+// layout) the MMAs accumulate S into one of two TMEM buffers while the four
+// warps read the other one back.  TMEM lane = query row, so thread tid owns
+// row t * 128 + tid of the tile.
+//
+// Selection in two passes over the tile's blocks, so that no per-score work
+// depends on earlier scores:
+//   pass 0  per row, the maximum score of each class j mod 64 of candidates
+//           j < own (kept in TMEM between blocks).  The K-th largest of these
+//           64 maxima (K = k-1) is a lower bound tau on the row's K-th best
+//           score: the K classes it comes from hold K distinct candidates
+//           scoring at least tau.
+//   pass 1  the same scores again; every candidate scoring at least tau is
+//           appended to the row's buffer in shared memory (column tid).  On
+//           random scores that is about K + 10.  A buffer that fills up is
+//           cut to its best K, whose K-th best then becomes an exact bar.
+// After pass 1 the best K of the buffer (a sorting network over 64 keys in
+// registers) are the selection, best first: a candidate left out scores below
+// tau, so at least K collected ones rank above it.  The softmax of the own and
+// selected scores gives the weights.  Pass 0 compares raw accumulator values;
+// tau is scaled once, and rounding is monotone, so the bound holds for the
+// scaled scores of pass 1.
+template <int D>
+__global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
+    Params P, const __grid_constant__ CUtensorMap tm_lm, const uint8_t* qimg, int T, int n_tiles,
+    int32_t* idx, float* wout) {
+  using Lay = ScoreLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t s_full[kSBufs];   // MMAs into S buffer b done
+  __shared__ uint64_t s_free[kSBufs];   // the four epilogue warps have read S buffer b
+  __shared__ uint64_t lm_bar[kLmBufs];  // landmark buffer b landed
+  __shared__ uint64_t qbar;             // q~ terms of the current tile landed
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((int)blockIdx.x >= n_tiles) return;
+
+  if (tid == 0) {
+    for (int b = 0; b < kSBufs; ++b) {
+      tc::mbar_init(&s_full[b], 1);
+      tc::mbar_init(&s_free[b], kEpiWarps);
+    }
+    for (int b = 0; b < kLmBufs; ++b) tc::mbar_init(&lm_bar[b], 1);
+    tc::mbar_init(&qbar, 1);
+    tc::fence_mbar_init();
+    abort_sh = 0;
   }
+  if (warp == 0) {
+    tc::tmem_alloc(&tmem_sh, kTmemColsS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+  volatile int* abort_v = &abort_sh;
+
+  if (warp == kEpiWarps) {
+    // ---- MMA and TMA issue (one thread) ----
+    if (lane == 0) {
+      constexpr uint32_t kId = tc::idesc_bf16(kRowsS, kBlk, 0);
+      auto load_q = [&](const Step& st) {
+        const uint8_t* src = qimg + ((int64_t)st.bh * T + st.t) * (int64_t)Lay::kQimg;
+        tc::mbar_arrive_expect_tx(&qbar, Lay::kQimg);
+#pragma unroll
+        for (int term = 0; term < kTerms; ++term)
+          tc::bulk_g2s(sbase + Lay::kQ + term * Lay::kQt, src + term * Lay::kQt, Lay::kQt, &qbar);
+      };
+      auto load_lm = [&](const Step& s, int nb) {
+        const int b = (int)((unsigned)s.bh / (unsigned)P.Hq);
+        const int g = (int)((unsigned)(s.bh - b * P.Hq) / (unsigned)P.group);
+        const uint32_t dst = sbase + Lay::kLm + (uint32_t)nb * Lay::kLmB;
+        tc::mbar_arrive_expect_tx(&lm_bar[nb], Lay::kLmB);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tc::tma_load_4d(dst + c * (kBlk * 128), &tm_lm, c * 64, g, s.blk * kBlk, b, &lm_bar[nb]);
+      };
+      // waits for the MMAs of step m
+      auto mma_done = [&](int m) {
+        return tc::mbar_wait(&s_full[m % kSBufs], (uint32_t)(m / kSBufs) & 1u);
+      };
+      Step st, pf;
+      step_set(st, blockIdx.x, P, T, n_tiles);
+      pf = st;
+      load_lm(pf, 0);
+      step_next(pf, P, T, n_tiles);
+      int n = 0;
+      int lm_issued = 1;   // landmark loads issued (steps 0 .. lm_issued-1)
+      int mma_issued = 0;  // steps whose MMAs were committed
+      uint32_t qphase = 0;
+      bool q_pending = false;
+      bool ok = true;
+      for (; st.w < n_tiles; step_next(st, P, T, n_tiles), ++n) {
+        if (*abort_v) {
+          ok = false;
+          break;
+        }
+        if (st.pass == 0 && st.blk == 0) {
+          // the previous tile's MMAs must be done before its q~ terms are replaced
+          if (n > 0 && !mma_done(n - 1)) {
+            ok = false;
+            break;
+          }
+          load_q(st);
+          q_pending = true;
+          if (!tc::mbar_wait(&qbar, qphase)) {
+            ok = false;
+            break;
+          }
+          q_pending = false;
+          qphase ^= 1;
+        }
+        const int sb = n % kSBufs;
+        if (n >= kSBufs && !tc::mbar_wait(&s_free[sb], (uint32_t)(n / kSBufs - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        if (!tc::mbar_wait(&lm_bar[n & 1], (uint32_t)(n >> 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t lm = sbase + Lay::kLm + (uint32_t)(n & 1) * Lay::kLmB;
+#pragma unroll
+        for (int term = 0; term < kTerms; ++term) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = tc::smem_desc(sbase + Lay::kQ + term * Lay::kQt +
+                                                 (kk >> 2) * (kRowsS * 128) + (kk & 3) * 32,
+                                             16, 1024);
+            const uint64_t bd =
+                tc::smem_desc(lm + (kk >> 2) * (kBlk * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem + sb * kBlk, a, bd, kId, (term | kk) != 0);
+          }
+        }
+        tc::mma_commit(&s_full[sb]);
+        mma_issued = n + 1;
+        // step n+1's landmark block goes where step n-1's was: its MMAs must be done
+        if (pf.w < n_tiles) {
+          if (n > 0 && !mma_done(n - 1)) {
+            ok = false;
+            break;
+          }
+          load_lm(pf, (n + 1) & 1);
+          ++lm_issued;
+          step_next(pf, P, T, n_tiles);
+        }
+      }
+      if (!ok) {
+        *abort_v = 1;
+        // let what was issued land before the CTA exits (bounded waits)
+        if (mma_issued > 0) mma_done(mma_issued - 1);
+        for (int m = mma_issued; m < lm_issued; ++m)
+          tc::mbar_wait(&lm_bar[m & 1], (uint32_t)(m >> 1) & 1u);
+        if (q_pending) tc::mbar_wait(&qbar, qphase);
+      }
+    }
+  } else {
+    // ---- epilogue: four warps, TMEM lane = query row ----
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int K = P.k - 1;
+    uint64_t* Bf = reinterpret_cast<uint64_t*>(smem + Lay::kBuf) + tid;   // [kBufCap] stride kThrS
+    float thr_f = -INFINITY;   // pass 1: candidates scoring below this are left out
+    uint64_t thr_key = 0;      // pass 1: and keys must exceed this (set once the buffer was cut)
+    int cnt = 0;               // pass 1: keys in the buffer
+    float s_own = 0.f;
+
+    auto append = [&](uint64_t key) {
+      Bf[cnt * kThrS] = key;
+      if (++cnt == kBufCap) {
+        keep_best(Bf, cnt, K);
+        cnt = K;
+        thr_key = Bf[0];
+        thr_f = key_score(thr_key);
+      }
+    };
+
+    // best K of the buffer, best first; weights and the row's outputs
+    auto finish_tile = [&](const Step& st) {
+      const int i = st.t * kRowsS + tid;
+      uint64_t a[kBufCap];
+#pragma unroll
+      for (int e = 0; e < kBufCap; ++e) a[e] = e < cnt ? Bf[e * kThrS] : 0ull;
+      sort_desc<kBufCap>(a);
+      if (i < P.L) {
+        const int b = (int)((unsigned)st.bh / (unsigned)P.Hq);
+        const int h = st.bh - b * P.Hq;
+        const int own = (int)((P.pos0 + i) / kChunk);
+        const float mx = K > 0 ? fmaxf(s_own, key_score(a[0])) : s_own;
+        float sc[kMaxTopK];
+        float z = 0.f;
+#pragma unroll
+        for (int p = 0; p < kMaxTopK; ++p) {
+          const float e =
+              p == 0 ? __expf(s_own - mx)
+                     : ((p - 1 < K && a[p - 1]) ? __expf(key_score(a[p - 1]) - mx) : 0.f);
+          sc[p] = e;
+          z += e;
+        }
+        const float iz = 1.f / z;
+        const int64_t r = ((int64_t)b * P.L + i) * P.Hq + h;
+        int32_t* ix = idx + r * P.k;
+        float* wr = wout + r * P.k;
+        auto jat = [&](int p) -> int32_t {
+          return p == 0 ? own : (a[p - 1] ? key_index(a[p - 1]) : -1);
+        };
+        if ((P.k & 3) == 0) {
+#pragma unroll
+          for (int p = 0; p < kMaxTopK; p += 4) {
+            if (p < P.k) {
+              *reinterpret_cast<int4*>(ix + p) =
+                  make_int4(jat(p), jat(p + 1), jat(p + 2), jat(p + 3));
+              *reinterpret_cast<float4*>(wr + p) =
+                  make_float4(sc[p] * iz, sc[p + 1] * iz, sc[p + 2] * iz, sc[p + 3] * iz);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < kMaxTopK; ++p) {
+            if (p < P.k) {
+              ix[p] = jat(p);
+              wr[p] = sc[p] * iz;
+            }
+          }
+        }
+      }
+      cnt = 0;
+      thr_key = 0;
+    };
+
+    // S buffer sb: tile st's rows against chunks st.blk * 128 ..
+    auto drain = [&](int sb, const Step& st) {
+      const int i = st.t * kRowsS + tid;
+      const int i_last = min((st.t + 1) * kRowsS, (int)P.L) - 1;
+      const int own = i < P.L ? (int)((P.pos0 + i) / kChunk) : 0;
+      const int own_min = (int)((P.pos0 + st.t * kRowsS) / kChunk);
+      const int own_max = (int)((P.pos0 + i_last) / kChunk);
+      const int jb0 = st.blk * kBlk;
+      const uint32_t ta = tmem + sb * kBlk + lane_off;
+      const uint32_t tc_max = tmem + kCmaxCol + lane_off;
+      if (st.pass == 0) {
+        if (K == 0) return;
+        // class maxima: TMEM -> registers for this block only
+        float cm[kClasses];
+        if (st.blk == 0) {
+#pragma unroll
+          for (int x = 0; x < kClasses; ++x) cm[x] = -INFINITY;
+        } else {
+          uint32_t u0[32], u1[32];
+          tc::tmem_ld32(tc_max, u0);
+          tc::tmem_ld32(tc_max + 32, u1);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            cm[x] = __uint_as_float(u0[x]);
+            cm[32 + x] = __uint_as_float(u1[x]);
+          }
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBlk && jb0 + c0 < own_max; c0 += kClasses) {
+          const int jb = jb0 + c0;
+          uint32_t s0[32], s1[32];
+          tc::tmem_ld32(ta + c0, s0);
+          tc::tmem_ld32(ta + c0 + 32, s1);
+          tc::tmem_ld_wait();
+          if (jb + kClasses <= own_min) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              cm[x] = fmaxf(cm[x], __uint_as_float(s0[x]));
+              cm[32 + x] = fmaxf(cm[32 + x], __uint_as_float(s1[x]));
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              cm[x] = fmaxf(cm[x], jb + x < own ? __uint_as_float(s0[x]) : -INFINITY);
+              cm[32 + x] =
+                  fmaxf(cm[32 + x], jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY);
+            }
+          }
+        }
+        if (st.blk == st.nblk - 1) {
+          sort_desc<kClasses>(cm);
+          float tau = cm[0];
+#pragma unroll
+          for (int p = 1; p < kClasses; ++p) tau = (p == K - 1) ? cm[p] : tau;
+          thr_f = tau * P.inv_sqrt_d;
+        } else {
+          uint32_t u0[32], u1[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            u0[x] = __float_as_uint(cm[x]);
+            u1[x] = __float_as_uint(cm[32 + x]);
+          }
+          tc::tmem_st32(tc_max, u0);
+          tc::tmem_st32(tc_max + 32, u1);
+          tc::tmem_st_wait();
+        }
+        return;
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBlk && jb0 + c0 <= own_max; c0 += 64) {
+        uint32_t sv[2][32];
+        tc::tmem_ld32(ta + c0, sv[0]);
+        tc::tmem_ld32(ta + c0 + 32, sv[1]);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int jb = jb0 + c0 + hf * 32;
+          if (jb > own_max) break;
+          float v[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(sv[hf][x]) * P.inv_sqrt_d;
+          const int od = own - jb;
+          if (od >= 0 && od < 32) s_own = pick32(v, od);
+          if (K > 0 && jb < own_max) {
+            uint32_t m = 0;
+            if (jb + 32 <= own_min) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) m |= v[x] >= thr_f ? (1u << x) : 0u;
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) m |= (jb + x < own && v[x] >= thr_f) ? (1u << x) : 0u;
+            }
+            // one candidate per lane per round, so lanes do not serialise each other
+            while (__any_sync(0xffffffffu, m != 0)) {
+              if (m) {
+                const int x = __ffs(m) - 1;
+                m &= m - 1;
+                const uint64_t key = make_key(pick32(v, x), jb + x);
+                if (key > thr_key) append(key);
+              }
+            }
+          }
+        }
+      }
+      if (st.blk == st.nblk - 1) finish_tile(st);
+    };
+
+    Step st;
+    step_set(st, blockIdx.x, P, T, n_tiles);
+    for (int n = 0; st.w < n_tiles; step_next(st, P, T, n_tiles), ++n) {
+      const int sb = n % kSBufs;
+      if (!tc::warp_wait(&s_full[sb], (uint32_t)(n / kSBufs) & 1u) || *abort_v) {
+        if (lane == 0) *abort_v = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      drain(sb, st);
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s_free[sb]);
+    }
+  }
+
+  if (tid == 0 && *abort_v) set_device_error(kErrTimeout);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsS);
 }
 
 template <int D, int RP>
@@ -514,6 +677,42 @@ cudaError_t run_calib(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, in
   HILS_PROFILE("prefill.calib", s);
   calib_kernel<D, RP, NR><<<(unsigned)grid, kThrS, sm, s>>>(P, qimg, T, n_tiles);
   return cudaGetLastError();
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The landmark tensor [B][max_chunks][Hkv][D] as a 4-d TMA map, innermost
+// first; one box = 64 dimensions x 128 chunks of one (sequence, KV head), in
+// the 128-byte swizzle the MMA descriptors expect.  Chunks past max_chunks
+// read as zeros.
+template <int D>
+cudaError_t landmark_tmap(const Params& P, CUtensorMap* tm) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P.Hkv, (cuuint64_t)P.max_chunks,
+                              (cuuint64_t)P.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P.Hkv * D * 2,
+                                 (cuuint64_t)P.max_chunks * P.Hkv * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBlk, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(P.landmarks),
+                         dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int D>
@@ -538,25 +737,14 @@ cudaError_t run_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, fl
   }
   if (e != cudaSuccess) return e;
 
-  e = set_smem(score_tc_kernel<D>, Lay::kSmem);
+  CUtensorMap tm;
+  if ((e = landmark_tmap<D>(P, &tm)) != cudaSuccess) return e;
+  const size_t smem = Lay::kSmem;
+  e = set_smem(score_select_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_tc_kernel<D>, kThrS,
-                                                    Lay::kSmem);
-  if (e != cudaSuccess) return e;
-  {
-    const int64_t grid = min(n_tiles, (int64_t)n_sm * max(1, per_sm));
-    HILS_PROFILE("prefill.score_tc", s);
-    score_tc_kernel<D><<<(unsigned)grid, kThrS, Lay::kSmem, s>>>(P, qimg, ws.scores, T, n_tiles,
-                                                                 ws.score_cols);
-  }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  const size_t hs = sizeof(uint64_t) * kThrS * (size_t)max(1, P.k - 1);
-  {
-    HILS_PROFILE("prefill.select", s);
-    select_kernel<<<(unsigned)n_tiles, kThrS, hs, s>>>(P, ws.scores, T, ws.score_cols, idx, w);
-  }
+  const int64_t grid = min(n_tiles, (int64_t)n_sm);
+  HILS_PROFILE("prefill.score_select", s);
+  score_select_kernel<D><<<(unsigned)grid, kThrS + 32, smem, s>>>(P, tm, qimg, T, (int)n_tiles, idx, w);
   return cudaGetLastError();
 }
 

@@ -263,6 +263,23 @@ __device__ __forceinline__ void sort_desc(T (&a)[N]) {
   }
 }
 
+// Sorts a bitonic sequence of N registers descending (half-cleaner cascade).
+template <int N, typename T>
+__device__ __forceinline__ void merge_desc(T (&a)[N]) {
+#pragma unroll
+  for (int j = N >> 1; j > 0; j >>= 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if ((i & j) == 0) {
+        const T x = a[i], y = a[i + j];
+        const bool sw = x < y;
+        a[i] = sw ? y : x;
+        a[i + j] = sw ? x : y;
+      }
+    }
+  }
+}
+
 // One (tile, pass, landmark block) step of a CTA's walk.  Walk position w
 // covers (sequence, head) w / T and tile T - 1 - w % T: the tiles with the
 // most blocks come first, so the walk ends on short tiles.  Every tile takes
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       };
       // waits for the MMAs of step m
       auto mma_done = [&](int m) {
-        return tc::mbar_wait(&s_full[m % kSBufs], (uint32_t)(m / kSBufs) & 1u);
+        return tc::mbar_wait_sleep(&s_full[m % kSBufs], (uint32_t)(m / kSBufs) & 1u);
       };
       Step st, pf;
       step_set(st, blockIdx.x, P, T, n_tiles);
@@ -408,7 +425,7 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
           }
           load_q(st);
           q_pending = true;
-          if (!tc::mbar_wait(&qbar, qphase)) {
+          if (!tc::mbar_wait_sleep(&qbar, qphase)) {
             ok = false;
             break;
           }
@@ -416,11 +433,11 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
           qphase ^= 1;
         }
         const int sb = n % kSBufs;
-        if (n >= kSBufs && !tc::mbar_wait(&s_free[sb], (uint32_t)(n / kSBufs - 1) & 1u)) {
+        if (n >= kSBufs && !tc::mbar_wait_sleep(&s_free[sb], (uint32_t)(n / kSBufs - 1) & 1u)) {
           ok = false;
           break;
         }
-        if (!tc::mbar_wait(&lm_bar[n & 1], (uint32_t)(n >> 1) & 1u)) {
+        if (!tc::mbar_wait_sleep(&lm_bar[n & 1], (uint32_t)(n >> 1) & 1u)) {
           ok = false;
           break;
         }
@@ -456,8 +473,8 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
         // let what was issued land before the CTA exits (bounded waits)
         if (mma_issued > 0) mma_done(mma_issued - 1);
         for (int m = mma_issued; m < lm_issued; ++m)
-          tc::mbar_wait(&lm_bar[m & 1], (uint32_t)(m >> 1) & 1u);
-        if (q_pending) tc::mbar_wait(&qbar, qphase);
+          tc::mbar_wait_sleep(&lm_bar[m & 1], (uint32_t)(m >> 1) & 1u);
+        if (q_pending) tc::mbar_wait_sleep(&qbar, qphase);
       }
     }
   } else {
@@ -480,13 +497,33 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       }
     };
 
-    // best K of the buffer, best first; weights and the row's outputs
+    // best K of the buffer, best first; weights and the row's outputs.  The
+    // buffer is sorted 32 keys at a time by one sorting network in registers
+    // (the loop keeps a single copy of its code); the second half, when
+    // present, is merged in: the slot-wise maximum of the first half and the
+    // reversed second half holds the best 32 of both as a bitonic sequence,
+    // which a half-cleaner cascade sorts.
     auto finish_tile = [&](const Step& st) {
       const int i = st.t * kRowsS + tid;
-      uint64_t a[kBufCap];
+      uint64_t a[32];
 #pragma unroll
-      for (int e = 0; e < kBufCap; ++e) a[e] = e < cnt ? Bf[e * kThrS] : 0ull;
-      sort_desc<kBufCap>(a);
+      for (int p = 0; p < 32; ++p) a[p] = 0ull;
+      const int n_e = __reduce_max_sync(0xffffffffu, (unsigned)cnt);
+#pragma unroll 1
+      for (int h = 0; h * 32 < n_e; ++h) {
+        uint64_t c[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) c[e] = h * 32 + e < cnt ? Bf[(h * 32 + e) * kThrS] : 0ull;
+        sort_desc<32>(c);
+        if (h == 0) {
+#pragma unroll
+          for (int p = 0; p < 32; ++p) a[p] = c[p];
+        } else {
+#pragma unroll
+          for (int p = 0; p < 32; ++p) a[p] = a[p] > c[31 - p] ? a[p] : c[31 - p];
+          merge_desc<32>(a);
+        }
+      }
       if (i < P.L) {
         const int b = (int)((unsigned)st.bh / (unsigned)P.Hq);
         const int h = st.bh - b * P.Hq;
@@ -604,36 +641,49 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       }
 #pragma unroll 1
       for (int c0 = 0; c0 < kBlk && jb0 + c0 <= own_max; c0 += 64) {
+        const int jb = jb0 + c0;
         uint32_t sv[2][32];
         tc::tmem_ld32(ta + c0, sv[0]);
         tc::tmem_ld32(ta + c0 + 32, sv[1]);
         tc::tmem_ld_wait();
+        float v0[32], v1[32];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int jb = jb0 + c0 + hf * 32;
-          if (jb > own_max) break;
-          float v[32];
+        for (int x = 0; x < 32; ++x) {
+          v0[x] = __uint_as_float(sv[0][x]) * P.inv_sqrt_d;
+          v1[x] = __uint_as_float(sv[1][x]) * P.inv_sqrt_d;
+        }
+        const int od = own - jb;
+        if (od >= 0 && od < 32) s_own = pick32(v0, od);
+        if (od >= 32 && od < 64) s_own = pick32(v1, od - 32);
+        if (K > 0 && jb < own_max) {
+          uint32_t m0 = 0, m1 = 0;
+          if (jb + 64 <= own_min) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(sv[hf][x]) * P.inv_sqrt_d;
-          const int od = own - jb;
-          if (od >= 0 && od < 32) s_own = pick32(v, od);
-          if (K > 0 && jb < own_max) {
-            uint32_t m = 0;
-            if (jb + 32 <= own_min) {
-#pragma unroll
-              for (int x = 0; x < 32; ++x) m |= v[x] >= thr_f ? (1u << x) : 0u;
-            } else {
-#pragma unroll
-              for (int x = 0; x < 32; ++x) m |= (jb + x < own && v[x] >= thr_f) ? (1u << x) : 0u;
+            for (int x = 0; x < 32; ++x) {
+              m0 |= v0[x] >= thr_f ? (1u << x) : 0u;
+              m1 |= v1[x] >= thr_f ? (1u << x) : 0u;
             }
-            // one candidate per lane per round, so lanes do not serialise each other
-            while (__any_sync(0xffffffffu, m != 0)) {
-              if (m) {
-                const int x = __ffs(m) - 1;
-                m &= m - 1;
-                const uint64_t key = make_key(pick32(v, x), jb + x);
-                if (key > thr_key) append(key);
-              }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              m0 |= (jb + x < own && v0[x] >= thr_f) ? (1u << x) : 0u;
+              m1 |= (jb + 32 + x < own && v1[x] >= thr_f) ? (1u << x) : 0u;
+            }
+          }
+          // per round one candidate of each half per lane: lanes do not
+          // serialise each other, and the two extractions are independent
+          while (__any_sync(0xffffffffu, (m0 | m1) != 0)) {
+            if (m0) {
+              const int x = __ffs(m0) - 1;
+              m0 &= m0 - 1;
+              const uint64_t key = make_key(pick32(v0, x), jb + x);
+              if (key > thr_key) append(key);
+            }
+            if (m1) {
+              const int x = __ffs(m1) - 1;
+              m1 &= m1 - 1;
+              const uint64_t key = make_key(pick32(v1, x), jb + 32 + x);
+              if (key > thr_key) append(key);
             }
           }
         }
@@ -645,7 +695,8 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
     step_set(st, blockIdx.x, P, T, n_tiles);
     for (int n = 0; st.w < n_tiles; step_next(st, P, T, n_tiles), ++n) {
       const int sb = n % kSBufs;
-      if (!tc::warp_wait(&s_full[sb], (uint32_t)(n / kSBufs) & 1u) || *abort_v) {
+      const bool got = tc::mbar_wait_sleep(&s_full[sb], (uint32_t)(n / kSBufs) & 1u);
+      if (!__all_sync(0xffffffffu, got) || *abort_v) {
         if (lane == 0) *abort_v = 1;
         break;
       }

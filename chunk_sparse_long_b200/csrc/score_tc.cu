@@ -95,19 +95,31 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
     for (int v = 0; v < NR; ++v)
 #pragma unroll
       for (int a = 0; a < RP; ++a) ta[v][a] = 0.f;
+    // q is read 8 elements (16 bytes) at a time; the next group's load is
+    // issued before the current one is used, so its latency overlaps the FMAs
+    const uint16_t* qb = reinterpret_cast<const uint16_t*>(P.q);
+    auto ldq = [&](int v, int e) -> uint4 {
+      return valid[v] ? __ldg(reinterpret_cast<const uint4*>(qb + qoff[v] + e)) : make_uint4(0, 0, 0, 0);
+    };
+    auto unpack = [](uint4 u, float (&f)[8]) {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        f[2 * a] = __uint_as_float(w[a] << 16);
+        f[2 * a + 1] = __uint_as_float(w[a] & 0xFFFF0000u);
+      }
+    };
     if (P.r > 0) {
+      uint4 qr[NR], qn[NR];
+#pragma unroll
+      for (int v = 0; v < NR; ++v) qr[v] = ldq(v, 0);
 #pragma unroll 1
       for (int e0 = 0; e0 < D; e0 += 8) {
+#pragma unroll
+        for (int v = 0; v < NR; ++v) qn[v] = e0 + 8 < D ? ldq(v, e0 + 8) : qr[v];
         float qv[NR][8];
 #pragma unroll
-        for (int v = 0; v < NR; ++v) {
-          if (valid[v]) {
-            load8(P.q, HILS_BF16, qoff[v] + e0, qv[v]);
-          } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) qv[v][u] = 0.f;
-          }
-        }
+        for (int v = 0; v < NR; ++v) unpack(qr[v], qv[v]);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
 #pragma unroll
@@ -122,21 +134,21 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
             }
           }
         }
+#pragma unroll
+        for (int v = 0; v < NR; ++v) qr[v] = qn[v];
       }
     }
     // q~ = q + t B (a ascending), then the three-term split, 8 elements at a time
+    uint4 xr[NR], xn[NR];
+#pragma unroll
+    for (int v = 0; v < NR; ++v) xr[v] = ldq(v, 0);
 #pragma unroll 1
     for (int c = 0; c < D / 8; ++c) {
+#pragma unroll
+      for (int v = 0; v < NR; ++v) xn[v] = c + 1 < D / 8 ? ldq(v, (c + 1) * 8) : xr[v];
       float x[NR][8];
 #pragma unroll
-      for (int v = 0; v < NR; ++v) {
-        if (valid[v]) {
-          load8(P.q, HILS_BF16, qoff[v] + c * 8, x[v]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) x[v][u] = 0.f;
-        }
-      }
+      for (int v = 0; v < NR; ++v) unpack(xr[v], x[v]);
 #pragma unroll
       for (int a = 0; a < RP; ++a) {
         if (a < P.r) {
@@ -176,6 +188,8 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
         *reinterpret_cast<uint4*>(img + 1 * Lay::kQt + off) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
         *reinterpret_cast<uint4*>(img + 2 * Lay::kQt + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
+#pragma unroll
+      for (int v = 0; v < NR; ++v) xr[v] = xn[v];
     }
   }
 }
@@ -425,6 +439,14 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
           }
           load_q(st);
           q_pending = true;
+          {
+            // the CTA's next tile: its q~ terms into L2 while this tile runs
+            Step nx;
+            step_set(nx, st.w + (int)gridDim.x, P, T, n_tiles);
+            if (nx.w < n_tiles)
+              tc::bulk_prefetch_l2(qimg + ((int64_t)nx.bh * T + nx.t) * (int64_t)Lay::kQimg,
+                                   Lay::kQimg);
+          }
           if (!tc::mbar_wait_sleep(&qbar, qphase)) {
             ok = false;
             break;
@@ -582,43 +604,61 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       const uint32_t tc_max = tmem + kCmaxCol + lane_off;
       if (st.pass == 0) {
         if (K == 0) return;
-        // class maxima: TMEM -> registers for this block only
-        float cm[kClasses];
-        if (st.blk == 0) {
-#pragma unroll
-          for (int x = 0; x < kClasses; ++x) cm[x] = -INFINITY;
-        } else {
-          uint32_t u0[32], u1[32];
-          tc::tmem_ld32(tc_max, u0);
-          tc::tmem_ld32(tc_max + 32, u1);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            cm[x] = __uint_as_float(u0[x]);
-            cm[32 + x] = __uint_as_float(u1[x]);
-          }
-        }
-#pragma unroll 1
-        for (int c0 = 0; c0 < kBlk && jb0 + c0 < own_max; c0 += kClasses) {
-          const int jb = jb0 + c0;
-          uint32_t s0[32], s1[32];
-          tc::tmem_ld32(ta + c0, s0);
-          tc::tmem_ld32(ta + c0 + 32, s1);
-          tc::tmem_ld_wait();
+        // class maxima: TMEM -> registers for this block only, read together
+        // with the first 64 scores (one wait); the previous block's store of
+        // them is waited for here, not right after it was issued
+        uint32_t cmu[2][32];
+        tc::tmem_st_wait();
+        auto fold = [&](int jb, const uint32_t (&s0)[32], const uint32_t (&s1)[32]) {
           if (jb + kClasses <= own_min) {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              cm[x] = fmaxf(cm[x], __uint_as_float(s0[x]));
-              cm[32 + x] = fmaxf(cm[32 + x], __uint_as_float(s1[x]));
+              cmu[0][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[0][x]), __uint_as_float(s0[x])));
+              cmu[1][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[1][x]), __uint_as_float(s1[x])));
             }
           } else {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              cm[x] = fmaxf(cm[x], jb + x < own ? __uint_as_float(s0[x]) : -INFINITY);
-              cm[32 + x] =
-                  fmaxf(cm[32 + x], jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY);
+              cmu[0][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[0][x]),
+                                                jb + x < own ? __uint_as_float(s0[x]) : -INFINITY));
+              cmu[1][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[1][x]),
+                                                jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY));
             }
           }
+        };
+        if (jb0 < own_max) {
+          uint32_t s0[32], s1[32];
+          if (st.blk != 0) {
+            tc::tmem_ld32(tc_max, cmu[0]);
+            tc::tmem_ld32(tc_max + 32, cmu[1]);
+          }
+          tc::tmem_ld32(ta, s0);
+          tc::tmem_ld32(ta + 32, s1);
+          tc::tmem_ld_wait();
+          if (st.blk == 0) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
+          }
+          fold(jb0, s0, s1);
+          if (jb0 + kClasses < own_max) {
+            tc::tmem_ld32(ta + kClasses, s0);
+            tc::tmem_ld32(ta + kClasses + 32, s1);
+            tc::tmem_ld_wait();
+            fold(jb0 + kClasses, s0, s1);
+          }
+        } else if (st.blk != 0) {
+          tc::tmem_ld32(tc_max, cmu[0]);
+          tc::tmem_ld32(tc_max + 32, cmu[1]);
+          tc::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
+        }
+        float cm[kClasses];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          cm[x] = __uint_as_float(cmu[0][x]);
+          cm[32 + x] = __uint_as_float(cmu[1][x]);
         }
         if (st.blk == st.nblk - 1) {
           sort_desc<kClasses>(cm);
@@ -627,15 +667,8 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
           for (int p = 1; p < kClasses; ++p) tau = (p == K - 1) ? cm[p] : tau;
           thr_f = tau * P.inv_sqrt_d;
         } else {
-          uint32_t u0[32], u1[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            u0[x] = __float_as_uint(cm[x]);
-            u1[x] = __float_as_uint(cm[32 + x]);
-          }
-          tc::tmem_st32(tc_max, u0);
-          tc::tmem_st32(tc_max + 32, u1);
-          tc::tmem_st_wait();
+          tc::tmem_st32(tc_max, cmu[0]);
+          tc::tmem_st32(tc_max + 32, cmu[1]);
         }
         return;
       }

@@ -37,13 +37,13 @@ constexpr int kRowsS = kScoreTileRows;  // query rows per tile (M)
 constexpr int kBlk = kScoreBlock;       // landmark chunks per block (N)
 constexpr int kThrS = 128;
 constexpr int kTerms = 3;
-constexpr int kEpiWarps = 4;          // epilogue warps; warp 4 issues the MMAs and loads
+constexpr int kEpiWarps = 8;          // epilogue warps; warp 8 issues the MMAs and loads
 constexpr int kSBufs = 3;             // S buffers of 128 TMEM columns
 constexpr uint32_t kTmemColsS = 512;  // the S buffers, then the class maxima
-constexpr uint32_t kCmaxCol = kSBufs * 128;   // selection pass 0: 64 class maxima per row
+constexpr uint32_t kCmaxCol = kSBufs * 128;   // selection pass 0: 128 class maxima per row
 constexpr int kLmBufs = 2;            // landmark blocks in flight: prefetch distance 1
 constexpr int kClasses = 64;          // selection pass 0: one maximum per class j mod 64
-constexpr int kBufCap = 64;           // selection pass 1: collected candidates per row
+constexpr int kHalfCap = 32;          // selection pass 1: collected candidates per row and column half
 
 template <int D>
 struct ScoreLayout {
@@ -52,8 +52,8 @@ struct ScoreLayout {
   static constexpr uint32_t kLmB = kBlk * D * 2;              // one landmark block
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kLm = kQimg;                      // kLmBufs blocks
-  static constexpr uint32_t kBuf = kLm + kLmBufs * kLmB;    // [kBufCap][kThrS] uint64 keys
-  static constexpr uint32_t kSmem = kBuf + kBufCap * kThrS * 8 + 1024;   // + base alignment
+  static constexpr uint32_t kBuf = kLm + kLmBufs * kLmB;    // [2][kHalfCap][kThrS] uint64 keys
+  static constexpr uint32_t kSmem = kBuf + 2 * kHalfCap * kThrS * 8 + 1024;   // + base alignment
 };
 
 // ---- a1: calibration ------------------------------------------------------
@@ -354,7 +354,7 @@ __device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int n
 // tau is scaled once, and rounding is monotone, so the bound holds for the
 // scaled scores of pass 1.
 template <int D>
-__global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
+__global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
     Params P, const __grid_constant__ CUtensorMap tm_lm, const uint8_t* qimg, int T, int n_tiles,
     int32_t* idx, float* wout) {
   using Lay = ScoreLayout<D>;
@@ -365,6 +365,7 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
   __shared__ uint64_t qbar;             // q~ terms of the current tile landed
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
+  __shared__ float s_own_sh[kRowsS];  // each row's own-chunk score, from whichever half saw it
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t sbase = tc::smem_u32(smem);
@@ -500,18 +501,28 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       }
     }
   } else {
-    // ---- epilogue: four warps, TMEM lane = query row ----
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ---- epilogue: eight warps.  Warps q and q + 4 share TMEM lanes 32q ..
+    // 32q + 31 (query rows of the tile) and take the first and the second 64
+    // columns of every block: two warps per SM sub-partition, so one hides the
+    // other's dependent-instruction latency.  Each half keeps its own class
+    // maxima (classes j mod 128 over the two halves) and its own collection
+    // buffer; the pair meets on a named barrier to combine them.
+    const int q = warp & 3, hf = warp >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const int co = hf * 64;
+    const int bar_id = 1 + q;
     const int K = P.k - 1;
-    uint64_t* Bf = reinterpret_cast<uint64_t*>(smem + Lay::kBuf) + tid;   // [kBufCap] stride kThrS
+    uint64_t* const buf = reinterpret_cast<uint64_t*>(smem + Lay::kBuf);
+    uint64_t* Bf = buf + hf * kHalfCap * kThrS + row;         // this half, stride kThrS
+    uint64_t* Bo = buf + (1 - hf) * kHalfCap * kThrS + row;   // the partner's half
     float thr_f = -INFINITY;   // pass 1: candidates scoring below this are left out
     uint64_t thr_key = 0;      // pass 1: and keys must exceed this (set once the buffer was cut)
-    int cnt = 0;               // pass 1: keys in the buffer
-    float s_own = 0.f;
+    int cnt = 0;               // pass 1: keys in this half's buffer
 
     auto append = [&](uint64_t key) {
       Bf[cnt * kThrS] = key;
-      if (++cnt == kBufCap) {
+      if (++cnt == kHalfCap) {
         keep_best(Bf, cnt, K);
         cnt = K;
         thr_key = Bf[0];
@@ -519,71 +530,69 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       }
     };
 
-    // best K of the buffer, best first; weights and the row's outputs.  The
-    // buffer is sorted 32 keys at a time by one sorting network in registers
-    // (the loop keeps a single copy of its code); the second half, when
-    // present, is merged in: the slot-wise maximum of the first half and the
-    // reversed second half holds the best 32 of both as a bitonic sequence,
-    // which a half-cleaner cascade sorts.
+    // Both halves sort their buffers (one sorting network in registers); the
+    // second half hands its sorted keys over, and the first merges them in: the
+    // slot-wise maximum of its list and the reversed other list holds the best
+    // 32 of both as a bitonic sequence, which a half-cleaner cascade sorts.  The
+    // top K, best first, and the own chunk's score give idx and w.
     auto finish_tile = [&](const Step& st) {
-      const int i = st.t * kRowsS + tid;
-      uint64_t a[32];
+      uint64_t c[32];
 #pragma unroll
-      for (int p = 0; p < 32; ++p) a[p] = 0ull;
-      const int n_e = __reduce_max_sync(0xffffffffu, (unsigned)cnt);
-#pragma unroll 1
-      for (int h = 0; h * 32 < n_e; ++h) {
-        uint64_t c[32];
+      for (int e = 0; e < 32; ++e) c[e] = e < cnt ? Bf[e * kThrS] : 0ull;
+      sort_desc<32>(c);
+      if (hf == 1) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) c[e] = h * 32 + e < cnt ? Bf[(h * 32 + e) * kThrS] : 0ull;
-        sort_desc<32>(c);
-        if (h == 0) {
-#pragma unroll
-          for (int p = 0; p < 32; ++p) a[p] = c[p];
-        } else {
-#pragma unroll
-          for (int p = 0; p < 32; ++p) a[p] = a[p] > c[31 - p] ? a[p] : c[31 - p];
-          merge_desc<32>(a);
-        }
+        for (int e = 0; e < 32; ++e) Bf[e * kThrS] = c[e];
       }
-      if (i < P.L) {
-        const int b = (int)((unsigned)st.bh / (unsigned)P.Hq);
-        const int h = st.bh - b * P.Hq;
-        const int own = (int)((P.pos0 + i) / kChunk);
-        const float mx = K > 0 ? fmaxf(s_own, key_score(a[0])) : s_own;
-        float sc[kMaxTopK];
-        float z = 0.f;
+      tc::named_barrier(bar_id, 64);
+      if (hf == 0) {
 #pragma unroll
-        for (int p = 0; p < kMaxTopK; ++p) {
-          const float e =
-              p == 0 ? __expf(s_own - mx)
-                     : ((p - 1 < K && a[p - 1]) ? __expf(key_score(a[p - 1]) - mx) : 0.f);
-          sc[p] = e;
-          z += e;
+        for (int p = 0; p < 32; ++p) {
+          const uint64_t y = Bo[(31 - p) * kThrS];
+          c[p] = c[p] > y ? c[p] : y;
         }
-        const float iz = 1.f / z;
-        const int64_t r = ((int64_t)b * P.L + i) * P.Hq + h;
-        int32_t* ix = idx + r * P.k;
-        float* wr = wout + r * P.k;
-        auto jat = [&](int p) -> int32_t {
-          return p == 0 ? own : (a[p - 1] ? key_index(a[p - 1]) : -1);
-        };
-        if ((P.k & 3) == 0) {
-#pragma unroll
-          for (int p = 0; p < kMaxTopK; p += 4) {
-            if (p < P.k) {
-              *reinterpret_cast<int4*>(ix + p) =
-                  make_int4(jat(p), jat(p + 1), jat(p + 2), jat(p + 3));
-              *reinterpret_cast<float4*>(wr + p) =
-                  make_float4(sc[p] * iz, sc[p + 1] * iz, sc[p + 2] * iz, sc[p + 3] * iz);
-            }
-          }
-        } else {
+        merge_desc<32>(c);
+        const int i = st.t * kRowsS + row;
+        if (i < P.L) {
+          const int b = (int)((unsigned)st.bh / (unsigned)P.Hq);
+          const int h = st.bh - b * P.Hq;
+          const int own = (int)((P.pos0 + i) / kChunk);
+          const float s_own = s_own_sh[row];
+          const float mx = K > 0 ? fmaxf(s_own, key_score(c[0])) : s_own;
+          float sc[kMaxTopK];
+          float z = 0.f;
 #pragma unroll
           for (int p = 0; p < kMaxTopK; ++p) {
-            if (p < P.k) {
-              ix[p] = jat(p);
-              wr[p] = sc[p] * iz;
+            const float e =
+                p == 0 ? __expf(s_own - mx)
+                       : ((p - 1 < K && c[p - 1]) ? __expf(key_score(c[p - 1]) - mx) : 0.f);
+            sc[p] = e;
+            z += e;
+          }
+          const float iz = 1.f / z;
+          const int64_t r = ((int64_t)b * P.L + i) * P.Hq + h;
+          int32_t* ix = idx + r * P.k;
+          float* wr = wout + r * P.k;
+          auto jat = [&](int p) -> int32_t {
+            return p == 0 ? own : (c[p - 1] ? key_index(c[p - 1]) : -1);
+          };
+          if ((P.k & 3) == 0) {
+#pragma unroll
+            for (int p = 0; p < kMaxTopK; p += 4) {
+              if (p < P.k) {
+                *reinterpret_cast<int4*>(ix + p) =
+                    make_int4(jat(p), jat(p + 1), jat(p + 2), jat(p + 3));
+                *reinterpret_cast<float4*>(wr + p) =
+                    make_float4(sc[p] * iz, sc[p + 1] * iz, sc[p + 2] * iz, sc[p + 3] * iz);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int p = 0; p < kMaxTopK; ++p) {
+              if (p < P.k) {
+                ix[p] = jat(p);
+                wr[p] = sc[p] * iz;
+              }
             }
           }
         }
@@ -592,25 +601,38 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
       thr_key = 0;
     };
 
-    // S buffer sb: tile st's rows against chunks st.blk * 128 ..
+    // S buffer sb, this half's 64 columns: tile st's rows against chunks
+    // st.blk * 128 + co ..
     auto drain = [&](int sb, const Step& st) {
-      const int i = st.t * kRowsS + tid;
+      const int i = st.t * kRowsS + row;
       const int i_last = min((st.t + 1) * kRowsS, (int)P.L) - 1;
       const int own = i < P.L ? (int)((P.pos0 + i) / kChunk) : 0;
       const int own_min = (int)((P.pos0 + st.t * kRowsS) / kChunk);
       const int own_max = (int)((P.pos0 + i_last) / kChunk);
-      const int jb0 = st.blk * kBlk;
-      const uint32_t ta = tmem + sb * kBlk + lane_off;
-      const uint32_t tc_max = tmem + kCmaxCol + lane_off;
+      const int jb = st.blk * kBlk + co;
+      const uint32_t ta = tmem + sb * kBlk + co + lane_off;
+      const uint32_t tc_max = tmem + kCmaxCol + co + lane_off;
       if (st.pass == 0) {
         if (K == 0) return;
         // class maxima: TMEM -> registers for this block only, read together
-        // with the first 64 scores (one wait); the previous block's store of
-        // them is waited for here, not right after it was issued
+        // with the 64 scores (one wait); the previous block's store of them is
+        // waited for here, not right after it was issued
         uint32_t cmu[2][32];
         tc::tmem_st_wait();
-        auto fold = [&](int jb, const uint32_t (&s0)[32], const uint32_t (&s1)[32]) {
-          if (jb + kClasses <= own_min) {
+        if (jb < own_max) {
+          uint32_t s0[32], s1[32];
+          if (st.blk != 0) {
+            tc::tmem_ld32(tc_max, cmu[0]);
+            tc::tmem_ld32(tc_max + 32, cmu[1]);
+          }
+          tc::tmem_ld32(ta, s0);
+          tc::tmem_ld32(ta + 32, s1);
+          tc::tmem_ld_wait();
+          if (st.blk == 0) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
+          }
+          if (jb + 64 <= own_min) {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
               cmu[0][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[0][x]), __uint_as_float(s0[x])));
@@ -625,27 +647,6 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
                                                 jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY));
             }
           }
-        };
-        if (jb0 < own_max) {
-          uint32_t s0[32], s1[32];
-          if (st.blk != 0) {
-            tc::tmem_ld32(tc_max, cmu[0]);
-            tc::tmem_ld32(tc_max + 32, cmu[1]);
-          }
-          tc::tmem_ld32(ta, s0);
-          tc::tmem_ld32(ta + 32, s1);
-          tc::tmem_ld_wait();
-          if (st.blk == 0) {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
-          }
-          fold(jb0, s0, s1);
-          if (jb0 + kClasses < own_max) {
-            tc::tmem_ld32(ta + kClasses, s0);
-            tc::tmem_ld32(ta + kClasses + 32, s1);
-            tc::tmem_ld_wait();
-            fold(jb0 + kClasses, s0, s1);
-          }
         } else if (st.blk != 0) {
           tc::tmem_ld32(tc_max, cmu[0]);
           tc::tmem_ld32(tc_max + 32, cmu[1]);
@@ -654,17 +655,30 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
 #pragma unroll
           for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
         }
-        float cm[kClasses];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          cm[x] = __uint_as_float(cmu[0][x]);
-          cm[32 + x] = __uint_as_float(cmu[1][x]);
-        }
         if (st.blk == st.nblk - 1) {
-          sort_desc<kClasses>(cm);
-          float tau = cm[0];
+          float cm[64];
 #pragma unroll
-          for (int p = 1; p < kClasses; ++p) tau = (p == K - 1) ? cm[p] : tau;
+          for (int x = 0; x < 32; ++x) {
+            cm[x] = __uint_as_float(cmu[0][x]);
+            cm[32 + x] = __uint_as_float(cmu[1][x]);
+          }
+          sort_desc<64>(cm);
+          // the two halves' best 32 maxima meet in the (empty) collection
+          // buffers: the K-th largest of all 128 class maxima is the bound
+          tc::named_barrier(bar_id, 64);   // the partner is done with the last finish
+#pragma unroll
+          for (int s = 0; s < 32; ++s) Bf[s * kThrS] = __float_as_uint(cm[s]);
+          tc::named_barrier(bar_id, 64);
+#pragma unroll
+          for (int p = 0; p < 32; ++p) cm[p] = fmaxf(cm[p], __uint_as_float((uint32_t)Bo[(31 - p) * kThrS]));
+          tc::named_barrier(bar_id, 64);   // read before pass 1 appends
+          float top[32];
+#pragma unroll
+          for (int p = 0; p < 32; ++p) top[p] = cm[p];
+          merge_desc<32>(top);
+          float tau = top[0];
+#pragma unroll
+          for (int p = 1; p < 32; ++p) tau = (p == K - 1) ? top[p] : tau;
           thr_f = tau * P.inv_sqrt_d;
         } else {
           tc::tmem_st32(tc_max, cmu[0]);
@@ -672,12 +686,10 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
         }
         return;
       }
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBlk && jb0 + c0 <= own_max; c0 += 64) {
-        const int jb = jb0 + c0;
+      if (jb <= own_max) {
         uint32_t sv[2][32];
-        tc::tmem_ld32(ta + c0, sv[0]);
-        tc::tmem_ld32(ta + c0 + 32, sv[1]);
+        tc::tmem_ld32(ta, sv[0]);
+        tc::tmem_ld32(ta + 32, sv[1]);
         tc::tmem_ld_wait();
         float v0[32], v1[32];
 #pragma unroll
@@ -686,8 +698,8 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
           v1[x] = __uint_as_float(sv[1][x]) * P.inv_sqrt_d;
         }
         const int od = own - jb;
-        if (od >= 0 && od < 32) s_own = pick32(v0, od);
-        if (od >= 32 && od < 64) s_own = pick32(v1, od - 32);
+        if (od >= 0 && od < 32) s_own_sh[row] = pick32(v0, od);
+        if (od >= 32 && od < 64) s_own_sh[row] = pick32(v1, od - 32);
         if (K > 0 && jb < own_max) {
           uint32_t m0 = 0, m1 = 0;
           if (jb + 64 <= own_min) {
@@ -703,7 +715,7 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
               m1 |= (jb + 32 + x < own && v1[x] >= thr_f) ? (1u << x) : 0u;
             }
           }
-          // per round one candidate of each half per lane: lanes do not
+          // per round one candidate of each 32 columns per lane: lanes do not
           // serialise each other, and the two extractions are independent
           while (__any_sync(0xffffffffu, (m0 | m1) != 0)) {
             if (m0) {
@@ -729,7 +741,8 @@ __global__ void __launch_bounds__(kThrS + 32, 1) score_select_kernel(
     for (int n = 0; st.w < n_tiles; step_next(st, P, T, n_tiles), ++n) {
       const int sb = n % kSBufs;
       const bool got = tc::mbar_wait_sleep(&s_full[sb], (uint32_t)(n / kSBufs) & 1u);
-      if (!__all_sync(0xffffffffu, got) || *abort_v) {
+      // the pair decides together, so neither is ever left alone at its named barrier
+      if (tc::named_barrier_or(bar_id, 64, !got || *abort_v != 0)) {
         if (lane == 0) *abort_v = 1;
         break;
       }
@@ -828,7 +841,7 @@ cudaError_t run_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, fl
   if (e != cudaSuccess) return e;
   const int64_t grid = min(n_tiles, (int64_t)n_sm);
   HILS_PROFILE("prefill.score_select", s);
-  score_select_kernel<D><<<(unsigned)grid, kThrS + 32, smem, s>>>(P, tm, qimg, T, (int)n_tiles, idx, w);
+  score_select_kernel<D><<<(unsigned)grid, 2 * kThrS + 32, smem, s>>>(P, tm, qimg, T, (int)n_tiles, idx, w);
   return cudaGetLastError();
 }
 

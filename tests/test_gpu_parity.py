@@ -82,6 +82,48 @@ def test_prefill_matches_oracle(name):
     print(name, rep)
 
 
+@pytest.mark.parametrize("dtype,head_dim", [(BF16, 128), (BF16, 64), (F32, 64)])
+def test_prefill_tied_scores_keep_the_lowest_chunks(dtype, head_dim):
+    """Every chunk of a KV head carries the same landmark, so all of a row's
+    scores tie and the order (score desc, index asc) fixes the selection:
+    idx = [own, 0, 1, .., k-2] (fewer when fewer chunks are visible), with
+    uniform weights.  At 8192 positions a row sees up to 127 candidates, more
+    than a collection buffer holds, so the cut of a full buffer to its best
+    k-1 runs on every long row."""
+    gu = _gu()
+    p = random_problem(chunk_size=64, batch=1, n_q_heads=4, n_kv_heads=2, head_dim=head_dim,
+                       top_k=32, calib_rank=8, seq_len=8192, dtype=dtype, seed=21)
+    p.landmarks[:] = p.landmarks[:, :1]
+    dp = gu.DevProblem(p)
+    out, idx, w = gu.run_prefill(dp)
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    _, _, _, rp = p.rows()
+    own = rp // 64
+    n_sel = np.minimum(own, p.top_k - 1)
+    exp = np.full(idx.shape, -1, dtype=np.int32)
+    exp[:, 0] = own
+    for r in range(idx.shape[0]):
+        exp[r, 1:1 + n_sel[r]] = np.arange(n_sel[r])
+    np.testing.assert_array_equal(idx, exp)
+    exp_w = np.where(exp >= 0, 1.0 / (1 + n_sel)[:, None], 0.0)
+    np.testing.assert_allclose(w, exp_w, rtol=0, atol=1e-6)
+    # outputs against the oracle on every 16th row
+    from oracle import oracle
+    qr, rb, rh, rp = p.rows()
+    sel = np.arange(0, qr.shape[0], 16)
+    orc = oracle.hils_rows(ocfg(p), qr[sel], rb[sel], rh[sel], rp[sel], p.A, p.B, p.pages,
+                           p.block_table, p.landmarks)
+    np.testing.assert_array_equal(orc["idx"], exp[sel])
+
+    def rerun(rows, forced):
+        s_ = sel[rows]
+        return oracle.hils_rows(ocfg(p), qr[s_], rb[s_], rh[s_], rp[s_], p.A, p.B, p.pages,
+                                p.block_table, p.landmarks, forced)
+    rep = gu.compare(idx[sel], w[sel], gu.to_f64(out).reshape(-1, p.head_dim)[sel], orc, rerun,
+                     p.dtype)
+    print(rep)
+
+
 @pytest.mark.parametrize("name", ["tiny_f32_workload", "bf16_d128_gqa", "chunked_prefill"])
 def test_score_and_topk_match_oracle(name):
     gu = _gu()
@@ -125,6 +167,10 @@ def _decode_problem(batch, n_q_heads, n_kv_heads, head_dim, top_k, calib_rank, t
          steps=20, dtype=BF16, seed=12),
     dict(batch=2, n_q_heads=2, n_kv_heads=2, head_dim=64, top_k=16, calib_rank=8, t0=100,
          steps=40, dtype=F32, seed=13),
+    # every landmark of a KV head the same: all scores tie, so each step must
+    # keep chunks 0 .. k-2; 516+ chunks span two scan ranges at d=64 bf16
+    dict(batch=2, n_q_heads=4, n_kv_heads=2, head_dim=64, top_k=16, calib_rank=8, t0=33000,
+         steps=12, dtype=BF16, seed=14, tied=True),
 ])
 def test_decode_steps_match_oracle(case):
     """Each step appends (k_t, v_t) and attends at t; step s of sequence b is
@@ -132,7 +178,11 @@ def test_decode_steps_match_oracle(case):
     gu = _gu()
     from chunk_sparse_long_b200 import hils
     from oracle import oracle
+    case = dict(case)
+    tied = case.pop("tied", False)
     p, t0s = _decode_problem(**case)
+    if tied:
+        p.landmarks[:] = p.landmarks[:, :1]
     dp = gu.DevProblem(p)
     # the device cache starts with only the first t0_b tokens of each sequence
     pages = p.pages.copy()
@@ -170,6 +220,15 @@ def test_decode_steps_match_oracle(case):
     def rerun(rows, forced):
         return oracle.hils_rows(ocfg(p), qr[rows], rb[rows], rh[rows], rp[rows], p.A, p.B, p.pages,
                                 p.block_table, p.landmarks, forced)
+    if tied:
+        own = rp // 64
+        n_sel = np.minimum(own, k - 1)
+        exp = np.full((rp.shape[0], k), -1, dtype=np.int32)
+        exp[:, 0] = own
+        for r in range(rp.shape[0]):
+            exp[r, 1:1 + n_sel[r]] = np.arange(n_sel[r])
+        np.testing.assert_array_equal(idxs.cpu().numpy().reshape(-1, k), exp)
+        np.testing.assert_array_equal(orc["idx"], exp)
     rep = gu.compare(idxs.cpu().numpy().reshape(-1, k), wts.cpu().numpy().reshape(-1, k),
                      gu.to_f64(outs).reshape(-1, d), orc, rerun, p.dtype)
     print(case, rep)

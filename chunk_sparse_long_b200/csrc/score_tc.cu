@@ -6,21 +6,18 @@
 //       bf16 rounding of what is left, so q~ - (hi + mid + lo) is below
 //       2^-27 |q~|).  The terms are written as ready-made shared-memory
 //       images: per 128-row tile, three K-major 128-byte-swizzled tiles.
-//   score_select_kernel (a2-a4)  persistent; per 128-row tile one bulk copy
-//       brings the three term tiles in, and for every block of 128 causally
-//       visible chunks S = sum over terms Q_term LM^T runs as 3 x d/16
-//       tcgen05.mma (M = N = 128, float32 accumulate) into one of two TMEM
-//       buffers while the previous block is read back.  Landmark blocks are
-//       prefetched two steps ahead, across tile boundaries too.  The scores
-//       never leave the SM: TMEM lane r is query row r of the tile, so the
-//       thread that reads lane r keeps that row's k-1 best candidates j < own
-//       in a min-heap of 64-bit keys in shared memory (root = the worst kept
-//       entry).  Candidates that beat the root are inserted one set bit at a
-//       time across the warp, so lanes do not serialise each other's inserts;
-//       strict '>' against the root while j ascends keeps the lower index on
-//       ties.  After the tile's last block a heap sort yields the list
-//       best-first, and the softmax of the own and selected scores gives the
-//       weights.
+//   score_select_kernel (a2-a4)  persistent and warp-specialised; per
+//       128-row tile one bulk copy brings the three term tiles in, and for
+//       every block of 128 causally visible chunks S = sum over terms
+//       Q_term LM^T runs as 3 x d/16 tcgen05.mma (M = N = 128, float32
+//       accumulate) into one of three TMEM buffers while eight epilogue
+//       warps read the others back.  The scores never leave the SM: TMEM
+//       lane r is query row r of the tile, and two passes over a tile's
+//       blocks first bound each row's (k-1)-th best score from below by
+//       class maxima, then collect the few candidates above the bound.  A
+//       sorting network in registers turns them into the selection, best
+//       first, and the softmax of the own and selected scores gives the
+//       weights.  Its comment below has the details.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,7 +39,6 @@ constexpr int kSBufs = 3;             // S buffers of 128 TMEM columns
 constexpr uint32_t kTmemColsS = 512;  // the S buffers, then the class maxima
 constexpr uint32_t kCmaxCol = kSBufs * 128;   // selection pass 0: 128 class maxima per row
 constexpr int kLmBufs = 2;            // landmark blocks in flight: prefetch distance 1
-constexpr int kClasses = 64;          // selection pass 0: one maximum per class j mod 64
 constexpr int kHalfCap = 32;          // selection pass 1: collected candidates per row and column half
 
 template <int D>
@@ -329,30 +325,34 @@ __device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int n
   }
 }
 
-// Persistent: each CTA walks its tiles; per tile one bulk copy brings the q~
-// term images in, and per landmark block of 128 chunks (a TMA load from the
-// [B][max_chunks][Hkv][d] landmark tensor, already in the swizzled K-major
-// layout) the MMAs accumulate S into one of two TMEM buffers while the four
-// warps read the other one back.  TMEM lane = query row, so thread tid owns
-// row t * 128 + tid of the tile.
+// Persistent: each CTA walks its tiles.  Warp 8 issues: per tile one bulk
+// copy brings the q~ term images in, and per landmark block of 128 chunks (a
+// TMA load from the [B][max_chunks][Hkv][d] landmark tensor, already in the
+// swizzled K-major layout) the MMAs accumulate S into one of three TMEM
+// buffers.  Warps 0-7 read them back: warps q and q + 4 share TMEM lanes
+// 32q .. 32q+31, the tile's rows, and take the first and the second 64
+// columns of every block.
 //
 // Selection in two passes over the tile's blocks, so that no per-score work
 // depends on earlier scores:
-//   pass 0  per row, the maximum score of each class j mod 64 of candidates
-//           j < own (kept in TMEM between blocks).  The K-th largest of these
-//           64 maxima (K = k-1) is a lower bound tau on the row's K-th best
-//           score: the K classes it comes from hold K distinct candidates
-//           scoring at least tau.
+//   pass 0  per row and column half, the maximum score of each column class
+//           of candidates j < own, kept in TMEM between blocks: over both
+//           halves, the maxima of the 128 classes j mod 128.  The K-th
+//           largest of these maxima (K = k-1) is a lower bound tau on the
+//           row's K-th best score: the K classes it comes from hold K
+//           distinct candidates scoring at least tau.  The two halves swap
+//           their best 32 maxima to find it.
 //   pass 1  the same scores again; every candidate scoring at least tau is
-//           appended to the row's buffer in shared memory (column tid).  On
-//           random scores that is about K + 10.  A buffer that fills up is
-//           cut to its best K, whose K-th best then becomes an exact bar.
-// After pass 1 the best K of the buffer (a sorting network over 64 keys in
-// registers) are the selection, best first: a candidate left out scores below
-// tau, so at least K collected ones rank above it.  The softmax of the own and
-// selected scores gives the weights.  Pass 0 compares raw accumulator values;
-// tau is scaled once, and rounding is monotone, so the bound holds for the
-// scaled scores of pass 1.
+//           appended to its half's buffer in shared memory (column = row).
+//           On random scores that is a few more than K per row.  A half
+//           buffer that fills up is cut to its own best K, whose K-th best
+//           then becomes an exact bar for that half.
+// After pass 1 each half sorts its buffer and the first half merges in the
+// second's: the best K are the selection, best first.  A candidate left out
+// scores below tau, or below a half's bar, so at least K collected ones rank
+// above it.  The softmax of the own and selected scores gives the weights.
+// Pass 0 compares raw accumulator values; tau is scaled once, and rounding is
+// monotone, so the bound holds for the scaled scores of pass 1.
 template <int D>
 __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
     Params P, const __grid_constant__ CUtensorMap tm_lm, const uint8_t* qimg, int T, int n_tiles,
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
   using Lay = ScoreLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t s_full[kSBufs];   // MMAs into S buffer b done
-  __shared__ uint64_t s_free[kSBufs];   // the four epilogue warps have read S buffer b
+  __shared__ uint64_t s_free[kSBufs];   // the eight epilogue warps have read S buffer b
   __shared__ uint64_t lm_bar[kLmBufs];  // landmark buffer b landed
   __shared__ uint64_t qbar;             // q~ terms of the current tile landed
   __shared__ uint32_t tmem_sh;

@@ -191,7 +191,7 @@ __device__ __forceinline__ void fence_proxy_async() {
 }
 
 // Tiled TMA load of one box of a 4-d tensor map into shared memory; completes
-// its bytes on `bar`.  No multicast.  x * element size must be a multiple of 16.
+// its bytes on `bar`.  One CTA only.  x * element size must be a multiple of 16.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int x, int y, int z,
                                             int w, uint64_t* bar) {
   asm volatile(

@@ -53,8 +53,8 @@ def peaks():
 # per (row, slot) pair; it grows with the pairs.  Valid only for the kernel
 # source it was taken on (sha256 below); otherwise the bench reports null.
 ATTN_TRAFFIC = {"file": "chunk_sparse_long_b200/csrc/attn_tc.cu",
-                "sha256": "b0d9c1b9dec78ed8fe99932cd1dba126cc85deb80224227a1c6255a20ca250ae",
-                "bytes_per_pair": 4.391e9 / 15.76e6}
+                "sha256": "726b33a4854ca776577f02fa71415dc0a3b058fce348c6832b982bf4ea3a8afe",
+                "bytes_per_pair": (394345216 + 3976426752) / 15.76e6}
 
 
 def attn_traffic(pairs: float):

@@ -21,8 +21,12 @@
 //   warps 5-8, 9-12 (two groups, even / odd tiles)  thread t of a group owns
 //       tile row t (TMEM lane t): softmax of its 64 logits, keys after the
 //       query masked in the own chunk, P (bf16) written over the consumed Q
-//       stage; then O / l -> bf16 into the same stage, and one thread writes
-//       the whole tile with a single bulk copy.
+//       stage; then O / l -> bf16 into the same stage, which is handed to
+//       the store warp, and the group moves on to its next tile.
+//   warps 13, 14 (stores)  warp 13 + g serves group g: one thread writes each
+//       staged tile with a single bulk copy, waits until the copy has read
+//       the stage, and only then frees the stage for the producers.  The
+//       groups never wait for their stores.
 //
 // Partials are stored in bucket order, one row of d bf16 per pair (16-byte
 // chunk c of the row at chunk slot c ^ (position & 7)); merge_kernel then sums
@@ -39,7 +43,8 @@ namespace {
 constexpr int kRows = 128;          // pairs per MMA tile (M)
 constexpr int kProducers = 4;       // producer warps
 constexpr int kMmaWarp = kProducers;
-constexpr int kWarps = kProducers + 1 + 8;  // producers, MMA, two groups of four
+constexpr int kWarps = kProducers + 1 + 8 + 2;  // producers, MMA, two groups of four, stores
+constexpr int kStoreWarp = kProducers + 1 + 8;  // first of the two store warps
 constexpr int kThreads = kWarps * 32;
 
 template <int D>
@@ -76,6 +81,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
   __shared__ uint64_t q_full[NS], q_empty[NS], kv_full[2], kv_empty[2];
   __shared__ uint64_t s_full[2], sm_done[2], o_full[2], o_free[2];
   __shared__ TileDesc desc[NS];
+  __shared__ uint64_t staged[NS];         // a group has written the stage's output rows
+  __shared__ int64_t st_dst[NS];          // their byte offset in the partials
+  __shared__ uint32_t st_bytes[NS];       // and size; 0 marks the group's end
   __shared__ uint8_t meta_nk[NS][kRows];  // keys visible to it (64, or fewer in the own chunk)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -88,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
     for (int x = 0; x < NS; ++x) {
       tc::mbar_init(&q_full[x], 64 * kProducers);   // a cp.async and a plain arrival per producer
       tc::mbar_init(&q_empty[x], 1);
+      tc::mbar_init(&staged[x], 1);
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(&kv_full[x], 32 * kProducers);
@@ -337,6 +346,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
       }
     }
     __syncwarp();
+  } else if (warp >= kStoreWarp) {
+    // ------------------------------------------------------------------ stores
+    // warp kStoreWarp + g takes group g's tiles (n = g, g + 2, ..): stages
+    // g, g + 2 (mod NS)
+    if (lane == 0) {
+      bool ok = true;
+      for (int n = warp - kStoreWarp;; n += 2) {
+        const int st = n % NS;
+        if (!tc::mbar_wait_sleep(&staged[st], (n / NS) & 1)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bytes = st_bytes[st];
+        if (bytes == 0) break;
+        tc::bulk_s2g(reinterpret_cast<uint8_t*>(ws.partial) + st_dst[st],
+                     sbase + Lay::kQ + st * Lay::kQBytes, bytes);
+        tc::bulk_commit();
+        tc::bulk_wait_read();
+        tc::mbar_arrive(&q_empty[st]);
+      }
+      if (!ok) abort_sh = 1;
+      tc::bulk_wait_all();
+    }
+    __syncwarp();
   } else {
     // ---------------------------------------------- softmax + epilogue groups
     const int wg = (warp - kMmaWarp - 1) >> 2;
@@ -353,7 +386,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         ok = false;
         break;
       }
-      if (d.end) break;
+      if (d.end) {
+        if (row == 0) {
+          st_bytes[st] = 0;
+          tc::mbar_arrive(&staged[st]);
+        }
+        break;
+      }
       const int nk = meta_nk[st][row];
       uint8_t* stage = smem + Lay::kQ + st * Lay::kQBytes;
       bad = !tc::warp_wait(&s_full[wg], u & 1);
@@ -446,16 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params P, PrefillW
         ok = false;
         break;
       }
+      // every row of the group is written (and fenced for the async proxy):
+      // hand the stage to the store warp
       if (row == 0) {
-        uint8_t* dst = reinterpret_cast<uint8_t*>(ws.partial) + (int64_t)d.tile_base * (D * 2);
-        tc::bulk_s2g(dst, sbase + Lay::kQ + st * Lay::kQBytes, (uint32_t)d.n_valid * (D * 2));
-        tc::bulk_commit();
-        tc::bulk_wait_read();
-        tc::mbar_arrive(&q_empty[st]);
+        st_dst[st] = (int64_t)d.tile_base * (D * 2);
+        st_bytes[st] = (uint32_t)d.n_valid * (D * 2);
+        tc::mbar_arrive(&staged[st]);
       }
     }
     if (!ok) abort_sh = 1;
-    if (row == 0) tc::bulk_wait_all();
   }
 
   if (abort_sh && tid == 0) set_device_error(kErrTimeout);

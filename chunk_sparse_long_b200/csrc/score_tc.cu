@@ -576,7 +576,12 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
           auto jat = [&](int p) -> int32_t {
             return p == 0 ? own : (c[p - 1] ? key_index(c[p - 1]) : -1);
           };
-          if ((P.k & 3) == 0) {
+          // 16-byte stores when every row starts 16-byte aligned (the output
+          // pointers are the caller's: only 4-byte alignment is required)
+          const bool vec = (P.k & 3) == 0 &&
+                           ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(wout)) &
+                            15u) == 0;
+          if (vec) {
 #pragma unroll
             for (int p = 0; p < kMaxTopK; p += 4) {
               if (p < P.k) {

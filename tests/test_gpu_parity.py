@@ -124,6 +124,29 @@ def test_prefill_tied_scores_keep_the_lowest_chunks(dtype, head_dim):
     print(rep)
 
 
+def test_prefill_outputs_only_4_byte_aligned():
+    """idx and w need only int32 / float alignment: views one element into
+    larger buffers must receive exactly what aligned buffers receive."""
+    gu = _gu()
+    from chunk_sparse_long_b200 import hils
+    p = random_problem(chunk_size=64, **PREFILL_CASES["bf16_d128_gqa"])   # k = 8
+    dp = gu.DevProblem(p)
+    out, idx, w = gu.run_prefill(dp)
+    rows = p.batch * p.q_len * p.n_q_heads
+    ibuf = torch.full((rows * p.top_k + 1,), -7, dtype=torch.int32, device="cuda")
+    wbuf = torch.full((rows * p.top_k + 1,), -7.0, dtype=torch.float32, device="cuda")
+    idx_u, w_u = ibuf[1:].view(rows, p.top_k), wbuf[1:].view(rows, p.top_k)
+    assert idx_u.data_ptr() % 16 == 4 and w_u.data_ptr() % 16 == 4
+    out2 = torch.empty_like(out)
+    nbytes = hils.workspace_size(dp.cfg, hils.OP_PREFILL, p.q_len, p.max_chunks)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    hils.prefill(dp.cfg, dp.q, p.q_len, p.q_pos0, dp.A, dp.B, dp.cache, out2, idx_u, w_u, ws, nbytes)
+    hils.device_status()
+    assert int(ibuf[0]) == -7 and float(wbuf[0]) == -7.0
+    assert torch.equal(idx_u, idx) and torch.equal(w_u, w)
+    assert torch.equal(out2, out)
+
+
 @pytest.mark.parametrize("name", ["tiny_f32_workload", "bf16_d128_gqa", "chunked_prefill"])
 def test_score_and_topk_match_oracle(name):
     gu = _gu()

@@ -211,6 +211,8 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
   if (!out) return fail(HILS_ERR_INVALID_ARG, "out is NULL");
   if ((k_new == nullptr) != (v_new == nullptr))
     return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (!cache->seq_lens) return fail(HILS_ERR_INVALID_ARG, "cache->seq_lens is required for decode");
   if (P.Hq > 64) return fail(HILS_ERR_UNSUPPORTED, "decode supports up to 64 query heads");
   P.q = q;

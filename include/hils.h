@@ -113,7 +113,8 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
 
 /* a8: one decode step for every sequence of the batch.
  * q             [B][Hq][d]: one query per sequence.
- * k_new, v_new  [B][Hkv][d] or both NULL.  When given, each sequence's new token is
+ * k_new, v_new  [B][Hkv][d], 16-byte aligned, or both NULL.  When given, each
+ *               sequence's new token is
  *               written at position t = seq_lens[b] (its chunk's page must be in the
  *               block table) and seq_lens[b] is advanced to t+1 on the device at the
  *               end of the step, so repeated calls (or a captured graph) walk forward.

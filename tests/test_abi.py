@@ -104,6 +104,11 @@ def test_decode_argument_checks(lib):
     # the calibration matrices are read in 16-byte units
     st, msg = status_of(hils.decode, c, FAKE, None, None, FAKE + 4, FAKE, cache(), FAKE, None, None, FAKE, ws, 0)
     assert st == 1 and "aligned" in msg
+    # and so are the appended token's k and v
+    st, msg = status_of(hils.decode, c, FAKE, FAKE + 4, FAKE, FAKE, FAKE, cache(), FAKE, None, None, FAKE, ws, 0)
+    assert st == 1 and "aligned" in msg
+    st, msg = status_of(hils.decode, c, FAKE, FAKE, FAKE + 8, FAKE, FAKE, cache(), FAKE, None, None, FAKE, ws, 0)
+    assert st == 1 and "aligned" in msg
 
 
 def test_score_and_topk_argument_checks(lib):

@@ -114,10 +114,10 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
 /* a8: one decode step for every sequence of the batch.
  * q             [B][Hq][d]: one query per sequence.
  * k_new, v_new  [B][Hkv][d], 16-byte aligned, or both NULL.  When given, each
- *               sequence's new token is
- *               written at position t = seq_lens[b] (its chunk's page must be in the
- *               block table) and seq_lens[b] is advanced to t+1 on the device at the
- *               end of the step, so repeated calls (or a captured graph) walk forward.
+ *               sequence's new token is written at position t = seq_lens[b] (its
+ *               chunk's page must be in the block table) and seq_lens[b] is advanced
+ *               to t+1 on the device at the end of the step, so repeated calls (or a
+ *               captured graph) walk forward.
  *               When NULL, the token at t = seq_lens[b]-1 must already be present.
  * out           [B][Hq][d] in cfg->dtype; idx_out, w_out optional [B][Hq][k].
  * ws            at least hils_workspace_size(cfg, HILS_OP_DECODE, 1, max_chunks) bytes,

@@ -420,7 +420,14 @@ def main():
     args.warmup = max(args.warmup, 3)
 
     import torch
-    nworld, rank, barrier, maxreduce = dist_setup(torch)
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores alone; no process group is needed
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))   # the input generator
+        nworld, rank = int(os.environ.get("WORLD_SIZE", "1")), 0
+    else:
+        nworld, rank, barrier, maxreduce = dist_setup(torch)
     w = hi.WORKLOADS[args.workload]
     counts = prefill_counts(w)
     tokens_per_rank = w.batch * w.seq_len
@@ -432,8 +439,6 @@ def main():
               "l2": "inputs larger than L2 (q 1.07 GB, K/V 0.54 GB per step)"}
 
     if args.impl == "reference":
-        if rank != 0:
-            return
         wl = hi.device_workload(w)
         budget = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup) * 2)
         per = []

@@ -66,3 +66,18 @@ def test_weak_scaling_value_is_units_over_slowest_step():
     import bench
     assert bench.weak_scaling_value(1000, 1, 1.0) == pytest.approx(1e6)
     assert bench.weak_scaling_value(1000, 8, 2.0) == pytest.approx(4e6)
+
+
+def test_reference_arm_runs_on_rank_0_only():
+    """Under torchrun the reference arm (the oracle on host cores) runs on rank
+    0 alone; the other ranks leave at once, with status 0 and no output, and
+    touch neither CUDA nor a process group (this runs on a CPU-only host)."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2", CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""

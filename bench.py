@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PREFILL_KERNELS_PER_STEP = 8   # calib, score+select, bucket count, scan totals, scan, scatter, attend, merge (bf16)
+PREFILL_KERNELS_PER_STEP = 7   # calib, score+select, bucket count, scan totals, scan, scatter, attend + merge (bf16)
 DECODE_KERNELS_PER_STEP = 2    # scan (append, calibration, scores, selection), attend (+merge)
 
 

@@ -1,127 +1,121 @@
 // Decode step (a8): append, calibration, landmark scan, selection, split-k
 // chunk attention, as two kernels; the second is launched as a programmatic
-// dependent of the first (it may start early and waits for it before reading
-// its results).
+// dependent of the first (it starts early, does what does not depend on the
+// selection, and waits for the first before reading its results).
 //
 //   scan    grid (n_split, Hkv, B), 256 threads.  A CTA owns one KV head and a
 //           contiguous range of chunks of one sequence.  Every thread first
-//           issues its 256 bytes of landmark loads and the loads of A, B and
-//           the group's queries; q~ = q + (q A) B of the group's query heads is
-//           computed while the landmarks land, then every chunk of the range is
-//           scored.  Per query head, each warp sorts its part of the range
-//           (warp bitonic sort and merges) and warp 0 merges the warps' lists
-//           into the range's best k-1, written out best first.  The last CTA of
-//           a (sequence, KV head) -- one ticket per CTA -- merges the ranges'
-//           lists into the head's best k-1, adds the own chunk (its score from
-//           the own landmark), and writes the selection and the fusion weights.
+//           issues the small loads (A, B, the group's queries, the own
+//           landmark), then its 256 bytes of landmark rows; q~ = q + (q A) B of
+//           the group's query heads is computed while the landmarks land, then
+//           every chunk of the range is scored.  Per query head, each warp
+//           sorts its part of the range with a bitonic network on 64-bit keys
+//           (score, then chunk) and the warps' sorted lists are merged pairwise
+//           (a tree of bitonic merges): the range's best k-1, best first.  The
+//           last CTA of a (sequence, KV head) -- one ticket per CTA -- merges
+//           the ranges' lists the same way, adds the own chunk (its score from
+//           the own landmark), writes the selection, the fusion weights and the
+//           selected pages, and starts bringing those pages' K and V into L2.
 //           The first CTA of a (sequence, KV head) appends k_t and v_t.
-//   attend  grid (k, Hq, B), 128 threads.  The CTA of a (sequence, head, slot)
-//           attends to the slot's chunk: K and V staged in shared memory,
-//           softmax (keys after the query masked in the own chunk), P.V, the
-//           weighted partial to the workspace.  The last CTA of a (sequence,
-//           head) sums the k partials in slot order (deterministic); the last
+//   attend  grid (n_cta, Hq, B) in clusters of n_cta CTAs, one cluster per
+//           (sequence, query head); each CTA takes spc slots (128 threads per
+//           slot).  The own chunk (slot 0) does not depend on the selection:
+//           its attention runs before the wait, with the new token taken from
+//           k_new / v_new.  Every other slot stages its chunk's K and V in
+//           shared memory, then softmax (keys after the query masked in the own
+//           chunk) and P.V.  The weighted slot outputs are summed inside the CTA;
+//           every CTA writes its sum into the first CTA's shared memory
+//           (distributed shared memory) and arrives on its barrier, and the
+//           first CTA adds them up in slot order (deterministic).  The last
 //           head of a sequence advances seq_lens.
+#include <cooperative_groups.h>
+
 #include <cfloat>
 
 #include "hils_common.cuh"
 #include "tc_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hils {
 namespace {
 
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kAttThreads = 128;
+constexpr int kSlotThreads = 128;
 constexpr unsigned kFull = 0xffffffffu;
 
-// Selection keys.  A score maps to an unsigned key that orders like the score
-// (-0 taken as +0); key 0 means "no entry" and lies below every real score, and
-// -inf (a chunk that is not a candidate) maps to it as well.  Among equal keys
-// the lower chunk index ranks higher.
-__device__ __forceinline__ uint32_t score_key(float s) {
-  if (s == -INFINITY) return 0u;
-  const uint32_t u = __float_as_uint(s + 0.f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+// Selection keys.  The high word is the score mapped to an unsigned order
+// (-0 taken as +0), the low word ~j, so a larger key ranks higher in (score
+// desc, index asc).  Key 0 means "no entry" and lies below every real score;
+// -inf (a chunk that is not a candidate) maps to it.
+__device__ __forceinline__ uint64_t sel_key(float s, int64_t j) {
+  if (s == -INFINITY) return 0ull;
+  uint32_t u = __float_as_uint(s + 0.f);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((uint64_t)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)j);
 }
-__device__ __forceinline__ float key_score(uint32_t u) {
-  return u == 0u ? -INFINITY : __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+__device__ __forceinline__ float key_score(uint64_t key) {
+  if (key == 0ull) return -INFINITY;
+  const uint32_t u = (uint32_t)(key >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+__device__ __forceinline__ int key_chunk(uint64_t key) {
+  return key == 0ull ? -1 : (int)(0xFFFFFFFFu - (uint32_t)key);
 }
 
-// The best (key, chunk) offered by the warp's lanes: the largest key, and among
-// lanes holding it the lowest chunk.  Two warp reductions.
-__device__ __forceinline__ void warp_best(uint32_t u, int j, uint32_t& bu, int& bj) {
-  bu = __reduce_max_sync(kFull, u);
-  bj = (int)__reduce_min_sync(kFull, u == bu ? (uint32_t)j : 0xFFFFFFFFu);
+__device__ __forceinline__ uint64_t shfl64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(kFull, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(kFull, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(kFull, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(kFull, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
 }
 
-// Best k (<= 32) of the V entries each lane holds, by rounds of extraction;
-// lane a of the result holds the a-th best (key 0: none).  The entries are
-// consumed.
+// Bitonic sort of the warp's 32 keys (one per lane), descending across lanes.
+__device__ __forceinline__ uint64_t warp_sort32(uint64_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint64_t y = shfl_xor64(v, j);
+      const bool desc = (lane & k) == 0;
+      const bool lower = (lane & j) == 0;
+      v = (lower == desc) ? (v > y ? v : y) : (v < y ? v : y);
+    }
+  }
+  return v;
+}
+
+// The best 32 of two lists sorted descending across lanes, sorted descending:
+// the lane-wise maximum of one list and the reversed other is a bitonic
+// sequence holding them, which a half-cleaner cascade sorts.
+__device__ __forceinline__ uint64_t warp_merge32(uint64_t a, uint64_t b) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t br = shfl64(b, 31 - lane);
+  uint64_t c = a > br ? a : br;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t y = shfl_xor64(c, j);
+    c = ((lane & j) == 0) ? (c > y ? c : y) : (c < y ? c : y);
+  }
+  return c;
+}
+
+// The best 32 of the warp's 32 V keys (v[q] on every lane), sorted descending.
 template <int V>
-__device__ __forceinline__ void warp_topk(uint32_t (&u)[V], int (&j)[V], int k, uint32_t& ou,
-                                          int& oj) {
-  const int lane = threadIdx.x & 31;
-  ou = 0u;
-  oj = INT32_MAX;
-  for (int it = 0; it < k; ++it) {
-    uint32_t cu = 0u;
-    int cj = INT32_MAX;
+__device__ __forceinline__ uint64_t warp_top32(uint64_t (&v)[V]) {
 #pragma unroll
-    for (int q = 0; q < V; ++q)
-      if (u[q] > cu || (u[q] == cu && j[q] < cj)) {
-        cu = u[q];
-        cj = j[q];
-      }
-    uint32_t bu;
-    int bj;
-    warp_best(cu, cj, bu, bj);
-    if (bu == 0u) break;
-    if (lane == it) {
-      ou = bu;
-      oj = bj;
-    }
+  for (int q = 0; q < V; ++q) v[q] = warp_sort32(v[q]);
 #pragma unroll
-    for (int q = 0; q < V; ++q)
-      if (u[q] == bu && j[q] == bj) u[q] = 0u;
-  }
-}
-
-// Best k (<= 32) of n lists sorted best first, each of length k, in shared
-// memory (list l at lu[l * k], lj[l * k]); lane a of the result holds the a-th
-// best.  Lane x follows lists x, x + 32, ...; hp[] holds the lists' read
-// positions (shared memory, n entries, reset here).
-__device__ __forceinline__ void warp_merge_lists(const uint32_t* lu, const int* lj, int n, int k,
-                                                 int* hp, uint32_t& ou, int& oj) {
-  const int lane = threadIdx.x & 31;
-  for (int l = lane; l < n; l += 32) hp[l] = 0;
-  __syncwarp();
-  ou = 0u;
-  oj = INT32_MAX;
-  for (int it = 0; it < k; ++it) {
-    uint32_t cu = 0u;
-    int cj = INT32_MAX, cl = -1;
-    for (int l = lane; l < n; l += 32) {
-      const int p = hp[l];
-      if (p >= k) continue;
-      const uint32_t u = lu[l * k + p];
-      const int j = lj[l * k + p];
-      if (u > cu || (u == cu && j < cj)) {
-        cu = u;
-        cj = j;
-        cl = l;
-      }
-    }
-    uint32_t bu;
-    int bj;
-    warp_best(cu, cj, bu, bj);
-    if (bu == 0u) break;
-    if (lane == it) {
-      ou = bu;
-      oj = bj;
-    }
-    if (cl >= 0 && cu == bu && cj == bj) hp[cl] += 1;   // the owner moves past its entry
-    __syncwarp();
-  }
+  for (int w = 1; w < V; w <<= 1)
+#pragma unroll
+    for (int q = 0; q + w < V; q += 2 * w) v[q] = warp_merge32(v[q], v[q + w]);
+  return v[0];
 }
 
 template <int EB>
@@ -163,16 +157,23 @@ struct ScanGeo {
   static constexpr int EPU = 16 / EB;                     // elements per 16-byte load
   static constexpr int UPC = EPT / EPU;                   // 16-byte loads per (thread, chunk)
   static constexpr int SEG = CPS / kScanWarps;            // chunks a warp sorts
+  static constexpr int V = SEG >= 32 ? SEG / 32 : 1;     // keys per lane in the warp sort
 };
 
-template <int D>
+// Dynamic shared memory of the scan, in this order: A [D][r], B [r][D] (float),
+// raw q [group][D], q~ [group][D + 4], q A [group][kMaxRank], scores
+// [CPS][group], own landmark [D], the warps' lists [kScanWarps][32] (64-bit),
+// and, for the last CTA, the ranges' lists of one head [n_split][k-1] (64-bit).
 struct ScanSmem {
-  // the last part stages the ranges' lists of one query head for the last CTA:
-  // keys, chunks and read positions
-  static size_t bytes(int r, int group, int cps, int n_split, int k1) {
-    return sizeof(float) * (size_t)(2 * D * r + group * D + group * (D + 4) + group * kMaxRank +
-                                    cps * group + 2 * kScanWarps * 32 + D +
-                                    n_split * (2 * k1 + 1));
+  int D, r, group, cps, n_split, K;
+  __host__ __device__ size_t floats() const {
+    return (size_t)2 * D * r + (size_t)group * D + (size_t)group * (D + 4) +
+           (size_t)group * kMaxRank + (size_t)cps * group + D;
+  }
+  __host__ __device__ size_t lists_off() const { return (floats() * 4 + 15) & ~(size_t)15; }
+  __host__ __device__ size_t merge_off() const { return lists_off() + kScanWarps * 32 * 8; }
+  __host__ __device__ size_t bytes() const {
+    return merge_off() + (size_t)n_split * (K > 0 ? K : 1) * 8;
   }
 };
 
@@ -185,45 +186,35 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int QS = D + 4;                        // padded q~ row
   const int group = P.group, K = P.k - 1;
-  extern __shared__ float sm[];
-  float* sA = sm;                                  // [D][r]
+  const ScanSmem L{D, P.r, group, G::CPS, ws.n_split, K};
+  extern __shared__ __align__(16) uint8_t sraw[];
+  float* sA = reinterpret_cast<float*>(sraw);      // [D][r]
   float* sB = sA + D * P.r;                        // [r][D]
   float* sq = sB + P.r * D;                        // [group][D] raw q
   float* sqt = sq + group * D;                     // [group][QS] q~
   float* sT = sqt + group * QS;                    // [group][kMaxRank] q A
   float* sS = sT + group * kMaxRank;               // [CPS][group] scores
-  uint32_t* lu = reinterpret_cast<uint32_t*>(sS + G::CPS * group);  // [kScanWarps][k-1] warp lists
-  int* lj = reinterpret_cast<int*>(lu + kScanWarps * 32);           // chunks of those
-  float* slm = reinterpret_cast<float*>(lj + kScanWarps * 32);      // [D] own chunk's landmark
-  uint32_t* mu = reinterpret_cast<uint32_t*>(slm + D);  // [n_split][k-1] ranges' lists (last CTA)
-  int* mj = reinterpret_cast<int*>(mu + ws.n_split * K);
-  int* mhp = mj + ws.n_split * K;                       // [max(n_split, warps)] read positions
+  float* slm = sS + G::CPS * group;                // [D] own chunk's landmark
+  uint64_t* wl = reinterpret_cast<uint64_t*>(sraw + L.lists_off());   // [kScanWarps][32]
+  uint64_t* ml = reinterpret_cast<uint64_t*>(sraw + L.merge_off());   // [n_split][K]
   __shared__ int last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const bool append = ws.append != 0;
   const int64_t t = decode_pos(P, b, append, tid == 0 && split == 0 && g == 0);
   const int64_t own = t / kChunk;
-  const int64_t c0 = (int64_t)split * G::CPS;
+  const int cps = ws.chunks_per_split;                          // chunks of this range (<= CPS)
+  const int64_t c0 = (int64_t)split * cps;
   const int cl0 = G::TPC == 1 ? tid * G::CPT : tid / G::TPC;   // first local chunk
   const int part = G::TPC == 1 ? 0 : tid % G::TPC;              // element part of the row
 
-  // ---- every load first ---------------------------------------------------------
-  uint4 lm[G::CPT][G::UPC];
-#pragma unroll
-  for (int ci = 0; ci < G::CPT; ++ci) {
-    const int64_t j = c0 + cl0 + ci;
-    const bool cand = j < own;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        reinterpret_cast<const uint8_t*>(P.landmarks) +
-        ((((int64_t)b * P.max_chunks + (cand ? j : 0)) * P.Hkv + g) * D + part * G::EPT) * EB);
-#pragma unroll
-    for (int u = 0; u < G::UPC; ++u) lm[ci][u] = cand ? __ldcs(src + u) : make_uint4(0, 0, 0, 0);
-  }
+  // ---- loads: the small ones first, then the landmark rows; q~ is computed
+  // while the landmark rows are still in flight ----------------------------------
+  constexpr int NQ = (64 * D / G::EPU + kScanThreads - 1) / kScanThreads;
+  const int nq = group * D / G::EPU;
+  uint4 rq[NQ], rl = make_uint4(0, 0, 0, 0);
   {
-    constexpr int NQ = (64 * D / G::EPU + kScanThreads - 1) / kScanThreads;
-    const int na = D * P.r / 4, nq = group * D / G::EPU;
-    uint4 rq[NQ], rl = make_uint4(0, 0, 0, 0);
+    const int na = D * P.r / 4;
     // A and B straight into shared memory (asynchronous copies, no registers)
     for (int x = tid; x < na; x += kScanThreads) {
       tc::cp_async16(tc::smem_u32(sA + 4 * x), reinterpret_cast<const float4*>(P.A) + x, 16u);
@@ -241,37 +232,48 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       rl = __ldg(reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(P.landmarks) +
           (((int64_t)b * P.max_chunks + own) * P.Hkv + g) * D * EB) + tid);
-    // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
-    if (append && split == 0 && tid < 2 * (D / G::EPU)) {
-      const int64_t page = page_of(P, b, own);
-      if (page >= 0) {
-        const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x;
-        uint4* dst = reinterpret_cast<uint4*>(
-            reinterpret_cast<uint8_t*>(const_cast<void*>(P.pages)) +
-            page_offset(P, page, kind, g, (int)(t % kChunk)) * EB) + x;
-        *dst = __ldg(src);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < NQ; ++u) {
-      const int x = u * kScanThreads + tid;
-      if (x < nq) {
-        float v[G::EPU];
-        unpack16<EB>(rq[u], v);
-#pragma unroll
-        for (int e = 0; e < G::EPU; ++e) sq[x * G::EPU + e] = v[e];
-      }
-    }
-    if (tid < D / G::EPU) {
-      float v[G::EPU];
-      unpack16<EB>(rl, v);
-#pragma unroll
-      for (int e = 0; e < G::EPU; ++e) slm[tid * G::EPU + e] = v[e];
-    }
-    tc::cp_async_wait<0>();
   }
+  uint4 lm[G::CPT][G::UPC];
+#pragma unroll
+  for (int ci = 0; ci < G::CPT; ++ci) {
+    const int64_t j = c0 + cl0 + ci;
+    const bool cand = cl0 + ci < cps && j < own;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        reinterpret_cast<const uint8_t*>(P.landmarks) +
+        ((((int64_t)b * P.max_chunks + (cand ? j : 0)) * P.Hkv + g) * D + part * G::EPT) * EB);
+#pragma unroll
+    for (int u = 0; u < G::UPC; ++u) lm[ci][u] = cand ? __ldcs(src + u) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int u = 0; u < NQ; ++u) {
+    const int x = u * kScanThreads + tid;
+    if (x < nq) {
+      float v[G::EPU];
+      unpack16<EB>(rq[u], v);
+#pragma unroll
+      for (int e = 0; e < G::EPU; ++e) sq[x * G::EPU + e] = v[e];
+    }
+  }
+  if (tid < D / G::EPU) {
+    float v[G::EPU];
+    unpack16<EB>(rl, v);
+#pragma unroll
+    for (int e = 0; e < G::EPU; ++e) slm[tid * G::EPU + e] = v[e];
+  }
+  // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
+  if (append && split == 0 && tid < 2 * (D / G::EPU)) {
+    const int64_t page = page_of(P, b, own);
+    if (page >= 0) {
+      const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x;
+      uint4* dst = reinterpret_cast<uint4*>(
+          reinterpret_cast<uint8_t*>(const_cast<void*>(P.pages)) +
+          page_offset(P, page, kind, g, (int)(t % kChunk)) * EB) + x;
+      *dst = __ldg(src);
+    }
+  }
+  tc::cp_async_wait<0>();
   __syncthreads();
 
   // ---- a1: q~ = q + (q A) B of the group's heads --------------------------------
@@ -323,42 +325,33 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       }
 #pragma unroll
       for (int o = 1; o < G::TPC; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
-      if (part == 0) sS[(cl0 + ci) * group + hh] = j < own ? acc * P.inv_sqrt_d : -INFINITY;
+      if (part == 0)
+        sS[(cl0 + ci) * group + hh] = (cl0 + ci < cps && j < own) ? acc * P.inv_sqrt_d : -INFINITY;
     }
   }
   __syncthreads();
 
   // ---- a3 (range): best k-1 of the range per query head ---------------------------
-  // each warp extracts the best k-1 of its part of the range, warp 0 merges the
-  // warps' lists
+  // each warp sorts its part of the range; the warps' lists are merged pairwise
   for (int hh = 0; hh < group && K > 0; ++hh) {
     const int h = g * group + hh;
-    constexpr int V = G::SEG >= 32 ? G::SEG / 32 : 1;
-    uint32_t u[V];
-    int jj[V];
+    uint64_t v[G::V];
 #pragma unroll
-    for (int q = 0; q < V; ++q) {
+    for (int q = 0; q < G::V; ++q) {
       const int x = q * 32 + lane;
       const int cl = warp * G::SEG + x;
-      u[q] = x < G::SEG ? score_key(sS[cl * group + hh]) : 0u;
-      jj[q] = (int)(c0 + cl);
+      v[q] = x < G::SEG ? sel_key(sS[cl * group + hh], c0 + cl) : 0ull;
     }
-    uint32_t ou;
-    int oj;
-    warp_topk<V>(u, jj, K, ou, oj);
-    if (lane < K) {
-      lu[warp * K + lane] = ou;
-      lj[warp * K + lane] = oj;
+    wl[warp * 32 + lane] = warp_top32<G::V>(v);
+#pragma unroll
+    for (int step = 1; step < kScanWarps; step <<= 1) {
+      __syncthreads();
+      if ((warp & (2 * step - 1)) == 0)
+        wl[warp * 32 + lane] = warp_merge32(wl[warp * 32 + lane], wl[(warp + step) * 32 + lane]);
     }
     __syncthreads();
-    if (warp == 0) {
-      warp_merge_lists(lu, lj, kScanWarps, K, mhp, ou, oj);
-      if (lane < K) {
-        const int64_t o = (((int64_t)b * P.Hq + h) * ws.n_split + split) * K + lane;
-        ws.cand_s[o] = key_score(ou);
-        ws.cand_j[o] = ou == 0u ? -1 : oj;
-      }
-    }
+    if (warp == 0 && lane < K)
+      ws.cand[(((int64_t)b * P.Hq + h) * ws.n_split + split) * K + lane] = wl[lane];
     __syncthreads();
   }
 
@@ -372,18 +365,23 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   for (int hh = 0; hh < group; ++hh) {
     const int h = g * group + hh;
     const int64_t bh = (int64_t)b * P.Hq + h;
-    // the ranges' lists of this head into shared memory
-    for (int x = tid; x < ws.n_split * K; x += kScanThreads) {
-      const float v = __ldcg(ws.cand_s + bh * ws.n_split * K + x);
-      const int vj = __ldcg(ws.cand_j + bh * ws.n_split * K + x);
-      mu[x] = vj < 0 ? 0u : score_key(v);
-      mj[x] = vj < 0 ? INT32_MAX : vj;
+    if (K > 0) {
+      // the ranges' lists of this head into shared memory, then a tree of merges
+      for (int x = tid; x < ws.n_split * K; x += kScanThreads)
+        ml[x] = __ldcg(ws.cand + bh * ws.n_split * K + x);
+      for (int step = 1; step < ws.n_split; step <<= 1) {
+        __syncthreads();
+        for (int a = warp * 2 * step; a + step < ws.n_split; a += kScanWarps * 2 * step) {
+          const uint64_t x = lane < K ? ml[a * K + lane] : 0ull;
+          const uint64_t y = lane < K ? ml[(a + step) * K + lane] : 0ull;
+          const uint64_t c = warp_merge32(x, y);
+          if (lane < K) ml[a * K + lane] = c;
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
     if (warp == 0) {
-      uint32_t ou = 0u;
-      int oj = INT32_MAX;
-      if (K > 0) warp_merge_lists(mu, mj, ws.n_split, K, mhp, ou, oj);
+      const uint64_t key = (K > 0 && lane < K) ? ml[lane] : 0ull;
       // the own chunk's score
       float so = 0.f;
       for (int e = lane; e < D; e += 32) so = fmaf(sqt[hh * QS + e], slm[e], so);
@@ -391,10 +389,9 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       for (int o = 16; o > 0; o >>= 1) so += __shfl_xor_sync(kFull, so, o);
       so *= P.inv_sqrt_d;
       // a4: slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
-      const uint32_t sh_u = __shfl_sync(kFull, ou, (lane + 31) & 31);
-      const int sh_j = __shfl_sync(kFull, oj, (lane + 31) & 31);
-      const float my_s = lane == 0 ? so : key_score(sh_u);
-      const int my_j = lane == 0 ? (int)own : (sh_u == 0u ? -1 : sh_j);
+      const uint64_t sh = shfl64(key, (lane + 31) & 31);
+      const float my_s = lane == 0 ? so : key_score(sh);
+      const int my_j = lane == 0 ? (int)own : key_chunk(sh);
       const bool live = lane < P.k && my_j >= 0;
       float m = live ? my_s : -INFINITY;
 #pragma unroll
@@ -406,11 +403,19 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       if (lane < P.k) {
         const int jv = live ? my_j : -1;
         const float wv = live ? ex / z : 0.f;
+        const int64_t page = live ? page_of(P, b, jv) : -1;
         const int64_t o = bh * P.k + lane;
         ws.idx[o] = jv;
         ws.w[o] = wv;
+        ws.page[o] = (int32_t)page;
         if (idx_out) idx_out[o] = jv;
         if (w_out) w_out[o] = wv;
+        // the attention kernel reads these pages next: start bringing them into L2
+        if (page >= 0 && lane > 0) {
+          const uint8_t* base = reinterpret_cast<const uint8_t*>(P.pages);
+          tc::bulk_prefetch_l2(base + page_offset(P, page, 0, g, 0) * EB, kChunk * D * EB);
+          tc::bulk_prefetch_l2(base + page_offset(P, page, 1, g, 0) * EB, kChunk * D * EB);
+        }
       }
     }
     __syncthreads();
@@ -418,154 +423,244 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   if (tid == 0) ws.tickets[b * P.Hkv + g] = 0;
 }
 
+// Shared memory of one slot's K and V tiles: [2][kChunk][KL] elements with a
+// padded row of KL elements.
 template <int D, int EB>
-__global__ void __launch_bounds__(kAttThreads)
-    attend_kernel(Params P, DecodeWs ws, void* out) {
-  constexpr int EPU = 16 / EB;                 // elements per 16-byte load
-  constexpr int KL = D + (EB == 2 ? 8 : 4);    // padded shared-memory row (elements)
-  extern __shared__ __align__(16) uint8_t kv_raw[];   // [2][kChunk][KL] elements
+struct SlotTiles {
+  static constexpr int KL = D + (EB == 2 ? 8 : 4);
+  static constexpr size_t kBytes = (size_t)2 * kChunk * KL * EB;
+};
+
+// Attention of query `sq` to one chunk staged at `kv` (K rows then V rows),
+// keys 0 .. nk-1, by the 128 threads of a slot group (index st).  Leaves the
+// unnormalised output, dimension st % D, summed over the group's key halves in
+// `acc` (valid for st < D) and returns l, the sum of the probabilities.
+template <int D, int EB>
+__device__ __forceinline__ float chunk_attend(const float* sq, const uint8_t* kv, int nk,
+                                              float inv_sqrt_d, float* sp, float* red,
+                                              float* half_o, int st, float& acc, int bar_id) {
+  using T = SlotTiles<D, EB>;
+  const int lane = st & 31, wrp = st >> 5;
+  // scores: two threads per key, each half of the dimensions
+  const int key = st >> 1, hf = st & 1;
+  float a = 0.f;
+  const uint8_t* krow = kv + (key * T::KL + hf * (D / 2)) * EB;
+#pragma unroll 8
+  for (int e = 0; e < D / 2; ++e) {
+    const float kv_e = EB == 2 ? __uint_as_float(((uint32_t)reinterpret_cast<const uint16_t*>(krow)[e]) << 16)
+                               : reinterpret_cast<const float*>(krow)[e];
+    a = fmaf(sq[hf * (D / 2) + e], kv_e, a);
+  }
+  a += __shfl_xor_sync(kFull, a, 1);
+  const float s = key < nk ? a * inv_sqrt_d : -INFINITY;
+  float m = s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  if (lane == 0) red[wrp] = m;
+  tc::named_barrier(bar_id, kSlotThreads);
+  m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float ex = key < nk ? __expf(s - m) : 0.f;
+  if (hf == 0) sp[key] = ex;
+  float z = hf == 0 ? ex : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+  if (lane == 0) red[4 + wrp] = z;
+  tc::named_barrier(bar_id, kSlotThreads);
+  const float l = red[4] + red[5] + red[6] + red[7];
+  // P.V: thread -> one output dimension over one part of the keys
+  constexpr int KH = kSlotThreads / D;       // key groups (2 for D=64, 1 for D=128)
+  const int e = st % D, kg = st / D;
+  float o = 0.f;
+  for (int kk = kg * (kChunk / KH); kk < (kg + 1) * (kChunk / KH); ++kk) {
+    const uint8_t* vrow = kv + ((kChunk + kk) * T::KL + e) * EB;
+    const float vv = EB == 2 ? __uint_as_float(((uint32_t)*reinterpret_cast<const uint16_t*>(vrow)) << 16)
+                             : *reinterpret_cast<const float*>(vrow);
+    o = fmaf(sp[kk], vv, o);
+  }
+  half_o[st] = o;
+  tc::named_barrier(bar_id, kSlotThreads);
+  acc = 0.f;
+  if (st < D) {
+#pragma unroll
+    for (int x = 0; x < KH; ++x) acc += half_o[x * D + st];
+  }
+  return l;
+}
+
+// Stages rows [0, 64) of K and V of (page, KV head g) into `kv` with every
+// 16-byte load of the slot group in flight at once.
+template <int D, int EB>
+__device__ __forceinline__ void stage_tiles(const Params& P, int64_t page, int g, uint8_t* kv,
+                                            int st) {
+  using T = SlotTiles<D, EB>;
+  constexpr int EPU = 16 / EB;
+  constexpr int NU = kChunk * D / EPU;     // 16-byte units per tile
+  constexpr int PER = 2 * NU / kSlotThreads;
+  const uint8_t* kp = reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 0, g, 0) * EB;
+  const uint8_t* vp = reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 1, g, 0) * EB;
+  uint4 u4[PER];
+#pragma unroll
+  for (int a = 0; a < PER; ++a) {
+    const int x = a * kSlotThreads + st;
+    const int which = x / NU, y = x % NU;
+    u4[a] = __ldcg(reinterpret_cast<const uint4*>((which ? vp : kp) + (int64_t)y * 16));
+  }
+#pragma unroll
+  for (int a = 0; a < PER; ++a) {
+    const int x = a * kSlotThreads + st;
+    const int which = x / NU, y = x % NU;
+    const int key = y / (D / EPU), c = y % (D / EPU);
+    *reinterpret_cast<uint4*>(kv + ((which * kChunk + key) * T::KL + c * EPU) * EB) = u4[a];
+  }
+}
+
+template <int D, int EB>
+__global__ void __launch_bounds__(kSlotThreads * 2)
+    attend_kernel(Params P, DecodeWs ws, const void* k_new, const void* v_new, void* out,
+                  int spc) {
+  using T = SlotTiles<D, EB>;
+  constexpr int EPU = 16 / EB;
+  extern __shared__ __align__(16) uint8_t kv_raw[];   // spc x [2][kChunk][KL] elements
   __shared__ float sq[D];
-  __shared__ float sp[kChunk];
-  __shared__ float red[8];
-  __shared__ float half_o[kAttThreads];
-  __shared__ int last;
-  const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
-  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  __shared__ float sp[2][kChunk];
+  __shared__ float red[2][8];
+  __shared__ float half_o[2][kSlotThreads];
+  __shared__ float part[2][D];
+  __shared__ float cpart[16][D];   // rank 0: every CTA's sum, at its rank
+  __shared__ uint64_t cpart_bar;   // rank 0: one arrival per other CTA of the cluster
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x;
+  const int sg = tid / kSlotThreads, st = tid % kSlotThreads;
+  const int rank = (int)cluster.block_rank();
+  const int n_cta = (int)cluster.num_blocks();
+  const int h = blockIdx.y, b = blockIdx.z;
   const int g = h / P.group;
   const int64_t bh = (int64_t)b * P.Hq + h;
-  // this head's query does not depend on the scan
-  for (int e = tid; e < D; e += kAttThreads)
+  const int slot = rank * spc + sg;
+  const bool active = slot < P.k;
+  const bool append = ws.append != 0;
+  uint8_t* kv = kv_raw + sg * T::kBytes;
+  const int bar_id = 1 + sg;
+  // none of this depends on the scan: the query, the position, and the own chunk
+  for (int e = tid; e < D; e += blockDim.x)
     sq[e] = load_elem(P.q, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e);
-  // wait for the scan (programmatic dependent launch: this grid may start early)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int64_t t = decode_pos(P, b, ws.append != 0, false);
+  const int64_t t = decode_pos(P, b, append, false);
   const int64_t own = t / kChunk;
-  const int32_t j = __ldcg(ws.idx + bh * P.k + slot);
-  const float wj = __ldcg(ws.w + bh * P.k + slot);
-  const int64_t page = j >= 0 ? page_of(P, b, j) : -1;
-
-  // ---- a5: attention to this slot's chunk ----------------------------------
-  float* part = ws.part + (bh * P.k + slot) * D;
-  if (page >= 0) {
-    // K and V tiles of the chunk into shared memory: every 16-byte load in flight at once
-    const uint8_t* kp = reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 0, g, 0) * EB;
-    const uint8_t* vp = reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 1, g, 0) * EB;
-    constexpr int NU = kChunk * D / EPU;     // 16-byte units per tile
-    constexpr int PER = 2 * NU / kAttThreads;
-    uint4 u4[PER];
-#pragma unroll
-    for (int a = 0; a < PER; ++a) {
-      const int x = a * kAttThreads + tid;
-      const int which = x / NU, y = x % NU;
-      u4[a] = __ldg(reinterpret_cast<const uint4*>((which ? vp : kp) + (int64_t)y * 16));
-    }
-#pragma unroll
-    for (int a = 0; a < PER; ++a) {
-      const int x = a * kAttThreads + tid;
-      const int which = x / NU, y = x % NU;
-      const int key = y / (D / EPU), c = y % (D / EPU);
-      *reinterpret_cast<uint4*>(kv_raw + ((which * kChunk + key) * KL + c * EPU) * EB) = u4[a];
+  const int tr = (int)(t % kChunk);
+  if (rank == 0 && tid == 0) {
+    tc::mbar_init(&cpart_bar, n_cta > 1 ? n_cta - 1 : 1);
+    tc::fence_mbar_init();
+  }
+  // the barrier exists before any CTA of the cluster can arrive on it
+  cluster.sync();
+  float acc = 0.f, l = 0.f;
+  bool have = false;
+  if (active && slot == 0) {
+    const int64_t page = page_of(P, b, own);
+    if (page >= 0) {
+      stage_tiles<D, EB>(P, page, g, kv, st);
+      tc::named_barrier(bar_id, kSlotThreads);
+      // the new token is written by the scan: take it from the inputs
+      if (append && st < 2 * (D / EPU)) {
+        const int kind = st / (D / EPU), x = st % (D / EPU);
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x);
+        *reinterpret_cast<uint4*>(kv + ((kind * kChunk + tr) * T::KL + x * EPU) * EB) = v;
+      }
+      tc::named_barrier(bar_id, kSlotThreads);
+      l = chunk_attend<D, EB>(sq, kv, tr + 1, P.inv_sqrt_d, sp[sg], red[sg], half_o[sg], st, acc,
+                              bar_id);
+      have = true;
     }
   }
-  __syncthreads();
-  if (page >= 0) {
-    const int nk = (j == own) ? (int)(t - (int64_t)j * kChunk + 1) : kChunk;
-    // scores: two threads per key, each half of the dimensions
-    const int key = tid >> 1, hf = tid & 1;
-    float acc = 0.f;
-    const uint8_t* krow = kv_raw + (key * KL + hf * (D / 2)) * EB;
-#pragma unroll 8
-    for (int e = 0; e < D / 2; ++e) {
-      const float kv = EB == 2 ? __uint_as_float(((uint32_t)reinterpret_cast<const uint16_t*>(krow)[e]) << 16)
-                               : reinterpret_cast<const float*>(krow)[e];
-      acc = fmaf(sq[hf * (D / 2) + e], kv, acc);
-    }
-    acc += __shfl_xor_sync(kFull, acc, 1);
-    const float s = key < nk ? acc * P.inv_sqrt_d : -INFINITY;
-    float m = s;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    if (lane == 0) red[wrp] = m;
-    __syncthreads();
-    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const float ex = key < nk ? __expf(s - m) : 0.f;
-    if (hf == 0) sp[key] = ex;
-    float z = hf == 0 ? ex : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-    if (lane == 0) red[4 + wrp] = z;
-    __syncthreads();
-    const float l = red[4] + red[5] + red[6] + red[7];
-    // P.V: thread -> one output dimension over one part of the keys
-    constexpr int KH = kAttThreads / D;       // key groups (2 for D=64, 1 for D=128)
-    const int e = tid % D, kg = tid / D;
-    float o = 0.f;
-    for (int kk = kg * (kChunk / KH); kk < (kg + 1) * (kChunk / KH); ++kk) {
-      const uint8_t* vrow = kv_raw + ((kChunk + kk) * KL + e) * EB;
-      const float vv = EB == 2 ? __uint_as_float(((uint32_t)*reinterpret_cast<const uint16_t*>(vrow)) << 16)
-                               : *reinterpret_cast<const float*>(vrow);
-      o = fmaf(sp[kk], vv, o);
-    }
-    half_o[tid] = o;
-    __syncthreads();
-    if (tid < D) {
-      float tot = 0.f;
-#pragma unroll
-      for (int a = 0; a < KH; ++a) tot += half_o[a * D + tid];
-      part[tid] = l > 0.f ? tot * (wj / l) : 0.f;
-    }
-  } else {
-    for (int e = tid; e < D; e += kAttThreads) part[e] = 0.f;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int old = atomicAdd(&ws.tickets[P.B * P.Hq + bh], 1);
-    last = old == P.k - 1;
-  }
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  for (int e = tid; e < D; e += kAttThreads) {
-    float acc = 0.f;
-    for (int a = 0; a < P.k; ++a) acc += __ldcg(ws.part + (bh * P.k + a) * D + e);
-    store_elem(out, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e, acc);
-  }
-  if (tid == 0) {
-    ws.tickets[P.B * P.Hq + bh] = 0;
-    // every kernel of the step has read seq_lens: the last head of the sequence advances it
-    if (ws.append) {
-      int32_t* done = ws.tickets + 2 * P.B * P.Hq + b;
-      if (atomicAdd(done, 1) == P.Hq - 1) {
-        P.seq_lens[b] = (int32_t)(t + 1);
-        *done = 0;
+  // wait for the scan (programmatic dependent launch: this grid started early)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  float wj = 0.f;
+  if (active) {
+    wj = __ldcg(ws.w + bh * P.k + slot);
+    if (slot > 0) {
+      const int32_t page = __ldcg(ws.page + bh * P.k + slot);
+      if (page >= 0) {
+        const int32_t j = __ldcg(ws.idx + bh * P.k + slot);
+        stage_tiles<D, EB>(P, page, g, kv, st);
+        tc::named_barrier(bar_id, kSlotThreads);
+        l = chunk_attend<D, EB>(sq, kv, j == own ? tr + 1 : kChunk, P.inv_sqrt_d, sp[sg],
+                                red[sg], half_o[sg], st, acc, bar_id);
+        have = true;
       }
     }
   }
+  if (st < D) part[sg][st] = (have && l > 0.f) ? acc * (wj / l) : 0.f;
+  __syncthreads();
+  // this CTA's slots summed in slot order, into rank 0's shared memory
+  float* dst = cluster.map_shared_rank(&cpart[0][0], 0) + rank * D;
+  if (tid < D) {
+    float c = 0.f;
+    for (int x = 0; x < spc; ++x) c += part[x][tid];
+    dst[tid] = c;
+  }
+  if (rank != 0) {
+    __syncthreads();
+    if (tid == 0) tc::mbar_arrive_remote_cluster(&cpart_bar, 0);
+    return;
+  }
+  // rank 0: the cluster's sums in rank (= slot) order, once every other CTA's has landed
+  bool ok = true;
+  if (n_cta > 1) ok = tc::mbar_wait_cluster(&cpart_bar, 0);
+  if (!ok) {
+    if (tid == 0) set_device_error(kErrTimeout);
+    return;
+  }
+  __syncthreads();
+  if (tid < D) {
+    float o = 0.f;
+    for (int r = 0; r < n_cta; ++r) o += cpart[r][tid];
+    store_elem(out, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + tid, o);
+  }
+  // every kernel of the step has read seq_lens: the last head of the sequence advances it
+  if (tid == 0 && append) {
+    __threadfence();
+    int32_t* done = ws.tickets + P.B * P.Hkv + b;
+    if (atomicAdd(done, 1) == P.Hq - 1) {
+      P.seq_lens[b] = (int32_t)(t + 1);
+      *done = 0;
+    }
+  }
 }
 
-size_t scan_smem(const Params& P, int D, int cps, int n_split) {
-  const int k1 = P.k - 1, ns = n_split > kScanWarps ? n_split : kScanWarps;
-  return D == 64 ? ScanSmem<64>::bytes(P.r, P.group, cps, ns, k1)
-                 : ScanSmem<128>::bytes(P.r, P.group, cps, ns, k1);
-}
-
-// Launch with programmatic stream serialization: the kernel may start while
-// the previous one in the stream is still running.
+// Launch with programmatic stream serialization (the kernel may start while
+// the previous one in the stream is still running) and, when cluster > 1, in
+// clusters of `cluster` CTAs along x.
 template <typename... Args, typename... Actual>
-cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem,
+cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, int cluster,
                        cudaStream_t s, Actual... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Slots per attention CTA and CTAs per cluster: at most two slots per CTA, at
+// most 8 CTAs per cluster up to k = 16 (16, a non-portable size, above).
+void attend_shape(int k, int* spc, int* n_cta) {
+  *n_cta = k <= 8 ? k : (k <= 16 ? 8 : 16);
+  *spc = (k + *n_cta - 1) / *n_cta;
+}
+
+size_t scan_smem(const Params& P, int D, int cps, int n_split) {
+  const ScanSmem L{D, P.r, P.group, cps, n_split, P.k - 1};
+  return L.bytes();
 }
 
 template <int D, int EB>
@@ -581,11 +676,23 @@ cudaError_t run_decode(const Params& P, const void* k_new, const void* v_new, vo
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
-    const size_t kv_bytes = (size_t)2 * kChunk * (D + (EB == 2 ? 8 : 4)) * EB;
+    int spc, n_cta;
+    attend_shape(P.k, &spc, &n_cta);
+    const size_t kv_bytes = (size_t)spc * SlotTiles<D, EB>::kBytes;
     if ((e = set_smem(attend_kernel<D, EB>, kv_bytes)) != cudaSuccess) return e;
+    if (n_cta > 8) {
+      static bool np_set[2][2] = {};   // one flag per instantiation
+      bool& done = np_set[D == 128][EB == 4];
+      if (!done) {
+        e = cudaFuncSetAttribute(attend_kernel<D, EB>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        done = true;
+      }
+    }
     HILS_PROFILE("decode.attend", s);
-    e = launch_pdl(attend_kernel<D, EB>, dim3(P.k, P.Hq, P.B), dim3(kAttThreads), kv_bytes, s, P,
-                   ws, out);
+    e = launch_pdl(attend_kernel<D, EB>, dim3(n_cta, P.Hq, P.B), dim3(kSlotThreads * spc),
+                   kv_bytes, n_cta, s, P, ws, k_new, v_new, out, spc);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -602,9 +709,11 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
   DecodeWs w{};
-  w.chunks_per_split = chunks_per_split(P);
-  w.n_split = (P.max_chunks + w.chunks_per_split - 1) / w.chunks_per_split;
+  // as few ranges as the CTA geometry allows, then the chunks spread evenly over them
+  const int cps_max = chunks_per_split(P);
+  w.n_split = (P.max_chunks + cps_max - 1) / cps_max;
   if (w.n_split < 1) w.n_split = 1;
+  w.chunks_per_split = (P.max_chunks + w.n_split - 1) / w.n_split;
   const int K = P.k - 1 > 0 ? P.k - 1 : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -613,16 +722,15 @@ size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
     return p;
   };
   const int64_t nc = (int64_t)P.B * P.Hq * w.n_split * K;
-  w.cand_s = (float*)take(sizeof(float) * nc);
-  w.cand_j = (int32_t*)take(sizeof(int32_t) * nc);
+  w.cand = (uint64_t*)take(sizeof(uint64_t) * nc);
   w.idx = (int32_t*)take(sizeof(int32_t) * P.B * P.Hq * P.k);
   w.w = (float*)take(sizeof(float) * P.B * P.Hq * P.k);
-  w.part = (float*)take(sizeof(float) * P.B * P.Hq * P.k * P.d);
-  w.tickets = (int32_t*)take(sizeof(int32_t) * (2 * P.B * P.Hq + P.B));
+  w.page = (int32_t*)take(sizeof(int32_t) * P.B * P.Hq * P.k);
+  w.ticket_bytes = sizeof(int32_t) * ((size_t)P.B * P.Hkv + P.B);
+  w.tickets = (int32_t*)take(w.ticket_bytes);
   if (out) *out = w;
   return off;
 }
-
 
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                           int32_t* idx_out, float* w_out, const DecodeWs& ws_in, cudaStream_t s) {

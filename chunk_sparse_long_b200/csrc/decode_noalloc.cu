@@ -74,24 +74,8 @@ extern "C" int hils_decode_noalloc(const hils_config* cfg, const void* q, const 
   void* scratch = nullptr;
   int st = scratch_address(&scratch);
   if (st != HILS_OK) return st;
-  // The array keeps whatever the previous call left.  The completion counters
-  // must start at zero: clear them (their place depends on the configuration).
-  hils::Params P{};   // the fields the workspace carve-up reads
-  P.B = cfg->batch;
-  P.Hq = cfg->n_q_heads;
-  P.Hkv = cfg->n_kv_heads;
-  P.d = cfg->head_dim;
-  P.k = cfg->top_k;
-  P.r = cfg->calib_rank;
-  P.dtype = cfg->dtype;
-  P.max_chunks = cache->max_chunks;
-  hils::DecodeWs w{};
-  hils::decode_ws_bytes(P, &w, (char*)scratch);
-  const size_t ticket_bytes = sizeof(int32_t) * (2 * (size_t)P.B * P.Hq + P.B);
-  cudaError_t e = cudaMemsetAsync(w.tickets, 0, ticket_bytes, (cudaStream_t)stream);
-  if (e != cudaSuccess)
-    return noalloc_fail(HILS_ERR_CUDA, std::string("clearing scratch counters: ") + cudaGetErrorString(e));
-  st = hils_decode(cfg, q, k_new, v_new, A, B, cache, out, idx_out, w_out, scratch, kScratchBytes,
-                   stream);
-  return st;
+  // The array keeps whatever the previous call left; the step's completion
+  // counters must start at zero, so the call clears them (after its checks)
+  return hils::decode_call(cfg, q, k_new, v_new, A, B, cache, out, idx_out, w_out, scratch,
+                           kScratchBytes, true, stream);
 }

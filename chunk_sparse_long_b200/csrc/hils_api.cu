@@ -202,35 +202,8 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
 int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const void* v_new,
                 const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, void* stream) {
-  hils::Params P{};
-  int st;
-  if ((st = check_config(cfg, &P)) || (st = check_calib(cfg, A, B, &P)) ||
-      (st = check_pages(cache, &P)))
-    return st;
-  if (!q || !aligned16(q)) return fail(HILS_ERR_INVALID_ARG, "q is NULL or misaligned");
-  if (!out) return fail(HILS_ERR_INVALID_ARG, "out is NULL");
-  if ((k_new == nullptr) != (v_new == nullptr))
-    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
-  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
-    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
-  if (!cache->seq_lens) return fail(HILS_ERR_INVALID_ARG, "cache->seq_lens is required for decode");
-  if (P.Hq > 64) return fail(HILS_ERR_UNSUPPORTED, "decode supports up to 64 query heads");
-  P.q = q;
-  P.L = 1;
-  P.pos0 = 0;
-  hils::DecodeWs w{};
-  const size_t need = hils::decode_ws_bytes(P, &w, nullptr);
-  if (w.n_split > hils::kMaxSplitLists)
-    return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
-                hils::kMaxSplitLists, P.max_chunks, w.n_split);
-  if (!ws || ws_bytes < need)
-    return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
-  if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  hils::decode_ws_bytes(P, &w, (char*)ws);
-  if (P.B == 0) return HILS_OK;
-  cudaError_t e =
-      hils::launch_decode(P, k_new, v_new, out, idx_out, w_out, w, (cudaStream_t)stream);
-  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode");
+  return hils::decode_call(cfg, q, k_new, v_new, A, B, cache, out, idx_out, w_out, ws, ws_bytes,
+                           false, stream);
 }
 
 int hils_device_status(void* stream) {
@@ -270,5 +243,44 @@ cudaError_t set_smem_impl(const void* func, size_t bytes) {
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) have = bytes;
   return e;
+}
+}  // namespace hils
+
+namespace hils {
+int decode_call(const hils_config* cfg, const void* q, const void* k_new, const void* v_new,
+                const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
+                float* w_out, void* ws, size_t ws_bytes, bool clear_counters, void* stream) {
+  Params P{};
+  int st;
+  if ((st = check_config(cfg, &P)) || (st = check_calib(cfg, A, B, &P)) ||
+      (st = check_pages(cache, &P)))
+    return st;
+  if (!q || !aligned16(q)) return fail(HILS_ERR_INVALID_ARG, "q is NULL or misaligned");
+  if (!out) return fail(HILS_ERR_INVALID_ARG, "out is NULL");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  if (!cache->seq_lens) return fail(HILS_ERR_INVALID_ARG, "cache->seq_lens is required for decode");
+  if (P.Hq > 64) return fail(HILS_ERR_UNSUPPORTED, "decode supports up to 64 query heads");
+  P.q = q;
+  P.L = 1;
+  P.pos0 = 0;
+  DecodeWs w{};
+  const size_t need = decode_ws_bytes(P, &w, nullptr);
+  if (w.n_split > kMaxSplitLists)
+    return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
+                kMaxSplitLists, P.max_chunks, w.n_split);
+  if (!ws || ws_bytes < need)
+    return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
+  if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  decode_ws_bytes(P, &w, (char*)ws);
+  if (P.B == 0) return HILS_OK;
+  cudaError_t e;
+  if (clear_counters &&
+      (e = cudaMemsetAsync(w.tickets, 0, w.ticket_bytes, (cudaStream_t)stream)) != cudaSuccess)
+    return cuda_fail(e, "clearing the completion counters");
+  e = launch_decode(P, k_new, v_new, out, idx_out, w_out, w, (cudaStream_t)stream);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode");
 }
 }  // namespace hils

@@ -1,6 +1,7 @@
 // Internal declarations shared by the HiLS CUDA kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -133,6 +134,13 @@ cudaError_t set_smem(F* func, size_t bytes) {
   return set_smem_impl(reinterpret_cast<const void*>(func), bytes);
 }
 
+// Tensor map of a bf16 tensor with `rank` (2..5) dimensions, innermost first:
+// dims[x] elements along dimension x, strides[x] bytes from one index of
+// dimension x + 1 to the next (rank - 1 of them), box[x] elements per copy;
+// 128-byte swizzle, elements outside the tensor read as zeros.
+cudaError_t encode_tmap_bf16(CUtensorMap* tm, int rank, const void* base, const uint64_t* dims,
+                             const uint64_t* strides, const uint32_t* box);
+
 // ---- launchers (each returns cudaError_t of its launches) -----------------
 cudaError_t launch_score(const Params& P, float* scores, int n_cols, cudaStream_t s);
 cudaError_t launch_topk(const Params& P, const float* scores, int n_cols, int32_t* idx, float* w,
@@ -146,11 +154,9 @@ struct PrefillWs {
   int32_t* tile_off; // [n_keys + 1] tile offsets
   int32_t* cursor;   // [n_keys]
   int32_t* pairs;    // float32 path: [rows * k] pair ids (row * k + slot) in bucket order
-  int32_t* inv;      // [rows * k] bucket position of each pair id
-  int2* pinfo;       // bf16 path: [rows * k] (query row, position index) in bucket order
+  int4* pinfo;       // bf16 path: [rows * k] (query row, fusion weight bits, visible keys, 0)
+                     // in bucket order
   float* acc;        // [rows][d] float32 accumulator (CUDA-core attention)
-  void* partial;     // [rows * k][d] bf16 per-pair O / l in bucket order (tensor-core attention)
-  int32_t* queue;    // work-item counter of the persistent attention kernel
   void* qimg;        // bf16: per 128-row tile the three q~ term tiles (shared-memory images)
   int4* items;       // [max_tiles] (key, first pair, end pair, 0) of every work item
   int2* scan_totals; // [ceil(n_keys / 1024)] (pairs, items) of each block of keys
@@ -164,21 +170,27 @@ cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* 
                            const PrefillWs& ws, cudaStream_t s);
 cudaError_t launch_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, float* w,
                              cudaStream_t s);
-cudaError_t launch_attn_tc(const Params& P, void* out, const int32_t* idx, const float* w,
-                           const PrefillWs& ws, cudaStream_t s);
+cudaError_t launch_attn_tc(const Params& P, void* out, const PrefillWs& ws, cudaStream_t s);
 
 struct DecodeWs {
-  float* cand_s;       // [B][Hq][n_split][k-1] each range's best candidates, best first
-  int32_t* cand_j;     // same (-1: none)
+  uint64_t* cand;      // [B][Hq][n_split][k-1] each range's best candidates as selection keys,
+                       // best first
   int32_t* idx;        // [B][Hq][k] selected chunks (slot 0 = own)
   float* w;            // [B][Hq][k] fusion weights
-  float* part;         // [B][Hq][k][d] weighted per-slot outputs
-  int32_t* tickets;    // [B][Hkv] scan tickets, at B*Hq: [B][Hq] attention tickets, at
-                       // 2*B*Hq: [B] heads done; all return to zero after each step
+  int32_t* page;       // [B][Hq][k] their pages (-1: none)
+  int32_t* tickets;    // [B][Hkv] scan tickets, then [B] heads done; all return to zero
+                       // at the end of every step
+  size_t ticket_bytes;
   int n_split, chunks_per_split;
   int append;          // k_new / v_new given
 };
 size_t decode_ws_bytes(const Params& P, DecodeWs* ws, char* base);
+// hils_decode with its scratch at `ws`: validates every argument, lays the
+// workspace out, then (clear_counters) zeroes its completion counters on the
+// stream and launches the step.  Nothing is queued when a check fails.
+int decode_call(const hils_config* cfg, const void* q, const void* k_new, const void* v_new,
+                const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
+                float* w_out, void* ws, size_t ws_bytes, bool clear_counters, void* stream);
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                           int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s);
 

@@ -175,6 +175,15 @@ __device__ __forceinline__ int64_t pair_key(const Params& P, Windows W, int64_t 
   return bucket_key(P, W, (int)(bi / P.L), h / P.group, bi % P.L, j);
 }
 
+// The record of pair (query row, chunk j) for the tensor-core attention:
+// (row, fusion weight bits, keys of chunk j visible to the row, 0).  The
+// visible keys are 64 except in the row's own chunk, where they end at the
+// row's position.
+__device__ __forceinline__ int4 pair_record(int32_t row, float w, int64_t pos, int32_t j) {
+  const int nk = pos / kChunk == j ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
+  return make_int4(row, __float_as_int(w), nk, 0);
+}
+
 // One CTA per (sequence b, KV head g, block of kBucketRows query positions):
 // the block's pairs are counted into a shared-memory histogram over the chunks
 // its rows can see, then added to the global counts once per nonzero bin.
@@ -227,8 +236,9 @@ __global__ void __launch_bounds__(256) bucket_count_kernel(Params P, const int32
 // Same blocks: one global atomic per nonzero bin reserves the block's range of
 // each bucket, shared-memory atomics place the pairs inside it.
 __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int32_t* idx,
-                                                             int32_t* cursor, int32_t* pairs,
-                                                             int32_t* inv, int2* pinfo, Windows W) {
+                                                             const float* wts, int32_t* cursor,
+                                                             int32_t* pairs, int4* pinfo,
+                                                             Windows W) {
   extern __shared__ int32_t hist[];
   const int b = blockIdx.z, g = blockIdx.y;
   const int64_t i0 = (int64_t)blockIdx.x * kBucketRows, i1 = min(i0 + kBucketRows, P.L);
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int
   const int per_i = P.group * P.k;
   const SmallDiv dv(per_i), dk(P.k);
   const int n = (int)(i1 - i0) * per_i;
-  const bool rows_out = pinfo != nullptr;   // tensor-core path: (row, position) per pair
+  const bool rows_out = pinfo != nullptr;   // tensor-core path: a record per pair
   for (int f = threadIdx.x; f < n; f += blockDim.x) {
     const int ii = (int)dv.div((uint32_t)f);
     const int q = f - ii * per_i;                                        // head-in-group * k + slot
@@ -258,9 +268,8 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int
     const int32_t j = idx[p];
     if (j < 0 || j >= nvis) continue;
     const int32_t at = base[j] + atomicAdd(&hist[j], 1);
-    inv[p] = at;
     if (rows_out)
-      pinfo[at] = make_int2((int32_t)(row0 + dk.div((uint32_t)q)), (int32_t)i);
+      pinfo[at] = pair_record((int32_t)(row0 + dk.div((uint32_t)q)), wts[p], P.pos0 + i, j);
     else
       pairs[at] = (int32_t)p;
   }
@@ -280,17 +289,16 @@ __global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int6
   atomicAdd(&counts[pair_key(P, W, p, j)], 1);
 }
 
-__global__ void scatter_kernel(Params P, const int32_t* idx, int32_t* cursor, int32_t* pairs,
-                               int32_t* inv, int2* pinfo, int64_t n_pairs, Windows W) {
+__global__ void scatter_kernel(Params P, const int32_t* idx, const float* wts, int32_t* cursor,
+                               int32_t* pairs, int4* pinfo, int64_t n_pairs, Windows W) {
   const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= n_pairs) return;
   const int32_t j = idx[p];
   if (j < 0 || j >= P.max_chunks) return;
   const int32_t at = atomicAdd(&cursor[pair_key(P, W, p, j)], 1);
-  inv[p] = at;
   if (pinfo) {
     const int64_t r = p / P.k;
-    pinfo[at] = make_int2((int32_t)r, (int32_t)((r / P.Hq) % P.L));
+    pinfo[at] = pair_record((int32_t)r, wts[p], P.pos0 + (r / P.Hq) % P.L, j);
   } else {
     pairs[at] = (int32_t)p;
   }
@@ -519,7 +527,7 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
         scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
                                               ws.offsets, ws.tile_off, ws.cursor, ws.items);
       }
-      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv,
+      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.w, ws.cursor, ws.pairs,
                                                     P.dtype == HILS_BF16 ? ws.pinfo : nullptr, W);
     } else {
       const unsigned pb = (unsigned)((n_pairs + 255) / 256);
@@ -531,13 +539,13 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
         scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
                                               ws.offsets, ws.tile_off, ws.cursor, ws.items);
       }
-      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.cursor, ws.pairs, ws.inv,
+      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.w, ws.cursor, ws.pairs,
                                         P.dtype == HILS_BF16 ? ws.pinfo : nullptr, n_pairs, W);
     }
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // a5 + a6
-  if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws.idx, ws.w, ws, s);
+  if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws, s);
   if ((e = cudaMemsetAsync(ws.acc, 0, sizeof(float) * rows * D, s)) != cudaSuccess) return e;
   constexpr size_t asm_ = attend_smem<D>();
   e = set_smem(attend_kernel<D>, asm_);
@@ -585,23 +593,15 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
   if (P.dtype == HILS_BF16)
-    w.pinfo = (int2*)take(sizeof(int2) * n_pairs);
+    w.pinfo = (int4*)take(sizeof(int4) * n_pairs);
   else
     w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
-  w.inv = (int32_t*)take(sizeof(int32_t) * n_pairs);
   if (P.dtype == HILS_BF16) {
-    // the q~ images are dead before the attention writes its partials, so
-    // both share one region
     const int64_t T = (P.L + kScoreTileRows - 1) / kScoreTileRows;
-    const size_t qimg_bytes = (size_t)P.B * P.Hq * T * 3 * kScoreTileRows * P.d * 2;
-    const size_t part_bytes = (size_t)2 * n_pairs * P.d;
-    char* reg = take(part_bytes > qimg_bytes ? part_bytes : qimg_bytes);
-    w.partial = reg;
-    w.qimg = reg;
+    w.qimg = take((size_t)P.B * P.Hq * T * 3 * kScoreTileRows * P.d * 2);
   } else {
     w.acc = (float*)take(sizeof(float) * rows * P.d);
   }
-  w.queue = (int32_t*)take(sizeof(int32_t));
   w.n_keys = (int)n_keys;
   w.n_win = n_win;
   w.win_rows = win_rows;

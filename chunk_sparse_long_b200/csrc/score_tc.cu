@@ -18,11 +18,7 @@
 //       sorting network in registers turns them into the selection, best
 //       first, and the softmax of the own and selected scores gives the
 //       weights.  Its comment below has the details.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <cfloat>
-#include <mutex>
 
 #include "hils_common.cuh"
 #include "tc_common.cuh"
@@ -781,40 +777,17 @@ cudaError_t run_calib(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, in
   return cudaGetLastError();
 }
 
-// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
-PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // The landmark tensor [B][max_chunks][Hkv][D] as a 4-d TMA map, innermost
 // first; one box = 64 dimensions x 128 chunks of one (sequence, KV head), in
 // the 128-byte swizzle the MMA descriptors expect.  Chunks past max_chunks
 // read as zeros.
 template <int D>
 cudaError_t landmark_tmap(const Params& P, CUtensorMap* tm) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P.Hkv, (cuuint64_t)P.max_chunks,
-                              (cuuint64_t)P.B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P.Hkv * D * 2,
-                                 (cuuint64_t)P.max_chunks * P.Hkv * D * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBlk, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(P.landmarks),
-                         dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hkv, (uint64_t)P.max_chunks, (uint64_t)P.B};
+  const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)P.Hkv * D * 2,
+                               (uint64_t)P.max_chunks * P.Hkv * D * 2};
+  const uint32_t box[4] = {64, 1, (uint32_t)kBlk, 1};
+  return encode_tmap_bf16(tm, 4, P.landmarks, dims, strides, box);
 }
 
 template <int D>

@@ -144,7 +144,9 @@ def test_prefill_outputs_only_4_byte_aligned():
     hils.device_status()
     assert int(ibuf[0]) == -7 and float(wbuf[0]) == -7.0
     assert torch.equal(idx_u, idx) and torch.equal(w_u, w)
-    assert torch.equal(out2, out)
+    # the bf16 output sums a row's k shares by atomic additions in no fixed
+    # order, so two runs agree to the rounding of those additions only
+    assert float((out2.float() - out.float()).abs().max()) <= 2e-2
 
 
 @pytest.mark.parametrize("name", ["tiny_f32_workload", "bf16_d128_gqa", "chunked_prefill"])
@@ -280,7 +282,7 @@ def test_decode_equals_prefill_rows_on_gpu():
         np.testing.assert_allclose(w.cpu().numpy().reshape(4, 6),
                                    w_p.cpu().numpy().reshape(900, 4, 6)[t], atol=1e-6)
         # both paths are checked against the oracle elsewhere at max-abs 2e-2; here the
-        # CUDA-core decode and the tensor-core prefill (bf16 P, bf16 partials) agree to 2e-2
+        # CUDA-core decode and the tensor-core prefill (bf16 P, bf16 sums) agree to 2e-2
         np.testing.assert_allclose(gu.to_f64(out).reshape(4, 64),
                                    gu.to_f64(out_p).reshape(900, 4, 64)[t], atol=2e-2)
 

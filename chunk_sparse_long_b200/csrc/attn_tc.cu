@@ -11,20 +11,23 @@
 //       its 128 pair records (query row, fusion weight, visible keys) into a
 //       ring of kRing slots; per item one TMA copy of K and one of V (3-d
 //       tensor map over the page pool) into one of two buffers.
-//   warps 10-13 (gathers)  per tile, the pairs' query rows into one of NS
-//       stages with 16-byte cp.async, 128-byte swizzled, 32 rows per warp.
+//   warps 10-11 (gathers)  per tile, the pairs' query rows into one of NS
+//       stages with 16-byte cp.async, 128-byte swizzled, 64 rows per warp.
 //   warp 1 (MMA)  one thread issues, as each becomes ready, S = Q K^T
 //       (M = 128, N = 64) into one of the two TMEM S buffers of the tile's
-//       group, and O = P V (N = d) with P read from tensor memory.  A stage is
-//       free once its S product is done.
-//   warps 2-5, 6-9 (two groups, even / odd tiles)  thread t of a group owns
-//       tile row t (TMEM lane t).  For every tile: softmax of its 64 logits
-//       (keys after the query masked in the own chunk), P as bf16 into the
-//       first 32 columns of the S buffer; then the epilogue of the group's
-//       previous tile, so that its P V ran meanwhile: O scaled by w / l,
-//       rounded to bf16, and added into the output row in L2
-//       (red.global.add.bf16x2).  The output is zeroed before the kernel, and
-//       every pair adds its share, so no partial results are stored.
+//       group, and O = P V (N = d) with P read from tensor memory into the
+//       group's O buffer.  A stage is free once its S product is done.
+//   warps 2-5, 6-9 (two softmax groups, even / odd tiles)  thread t of a
+//       group owns tile row t (TMEM lane t): softmax of its 64 logits (keys
+//       after the query masked in the own chunk), l = sum of the
+//       probabilities, and P scaled by w / l as bf16 into the first 32
+//       columns of the S buffer, so that P V is already the pair's share of
+//       the output row.
+//   warps 12-15 (epilogue)  tile after tile, one TMEM lane quarter each: O to
+//       bf16, staged in shared memory and added into the output rows in L2
+//       (red.global.add.bf16x2, 128 contiguous bytes of each of four rows per
+//       warp instruction).  The output is zeroed before the kernel, and every
+//       pair adds its share, so no partial results are stored.
 //
 // The sum over a row's k pairs is taken by bf16 atomic additions in L2, in no
 // fixed order: the output is not bit-reproducible from run to run, and each
@@ -41,12 +44,13 @@ constexpr int kRows = 128;        // pairs per MMA tile (M)
 constexpr int kProdWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kGroupWarp0 = 2;    // group g: warps 2 + 4g .. 5 + 4g
-constexpr int kGatherWarp0 = 10;  // warps 10-13: query-row gathers
-constexpr int kGatherWarps = 4;
-constexpr int kWarps = 14;
+constexpr int kGatherWarp0 = 10;  // warps 10-11: query-row gathers
+constexpr int kGatherWarps = 2;
+constexpr int kEpiWarp0 = 12;     // warps 12-15: epilogue, one per TMEM lane quarter
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRing = 8;          // tiles whose descriptors and pair records are in flight
-constexpr uint32_t kStageRowBytes = 64;   // epilogue staging: 32 bf16 of one row
+constexpr uint32_t kStageRowBytes = 128;  // epilogue staging: 64 bf16 of one row
 
 template <int D>
 struct AttnLayout {
@@ -56,9 +60,9 @@ struct AttnLayout {
   static constexpr uint32_t kQ = 0;                     // NS stages
   static constexpr uint32_t kK = NS * kQBytes;          // two K buffers
   static constexpr uint32_t kV = kK + 2 * kKVBytes;     // two V buffers
-  static constexpr uint32_t kStage = kV + 2 * kKVBytes; // 8 warps x 32 rows x 64 bytes
+  static constexpr uint32_t kStage = kV + 2 * kKVBytes; // 4 warps x 32 rows x 128 bytes
   static constexpr uint32_t kStageWarp = 32 * kStageRowBytes;
-  static constexpr uint32_t kMeta = kStage + 8 * kStageWarp;   // [kRing][128] pair records
+  static constexpr uint32_t kMeta = kStage + 4 * kStageWarp;   // [kRing][128] pair records
   static constexpr uint32_t kEnd = kMeta + kRing * kRows * 16;
   static constexpr uint32_t kSmem = kEnd + 1024;                // + slack for 1024-byte alignment
   static_assert(kSmem + 1024 <= 232448, "dynamic + static shared memory above 227 KB");
@@ -102,13 +106,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < kRing; ++x) {
       tc::mbar_init(&ring_full[x], 1);   // the producer's expect_tx arrival; the records' bytes
-      tc::mbar_init(&ring_free[x], 5);   // the group's four warps and the MMA thread
+      tc::mbar_init(&ring_free[x], 9);   // the group's four warps, the MMA thread, the epilogue
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(&kv_full[x], 1);
       tc::mbar_init(&kv_empty[x], 1);
       tc::mbar_init(&o_full[x], 1);
-      tc::mbar_init(&o_free[x], 128);
+      tc::mbar_init(&o_free[x], 4);   // the four epilogue warps
       for (int y = 0; y < 2; ++y) {
         tc::mbar_init(&s_full[x][y], 1);
         tc::mbar_init(&sm_done[x][y], 128);
@@ -227,10 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int x = max(0, kv_issued - 2); x < kv_issued; ++x)
         tc::mbar_wait(&kv_full[x & 1], (x >> 1) & 1);
     }
-  } else if (warp >= kGatherWarp0) {
+  } else if (warp >= kGatherWarp0 && warp < kEpiWarp0) {
     // ---------------------------------------------------------------- gathers
     // Tile after tile: once its records have landed and its stage is free,
-    // warp w copies the query rows 32 w' .. 32 w' + 31 (w' = w - 10) into the
+    // warp w copies the query rows 64 w' .. 64 w' + 63 (w' = w - 10) into the
     // stage, 16 bytes per cp.async, in the 128-byte-swizzled K-major layout;
     // every lane arrives on the stage's barrier when its copies have landed.
     constexpr int CPR = D / 8;        // 16-byte chunks per row
@@ -254,17 +258,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int4* rec = meta + slot * kRows;
-      const int my_row = gw * 32 + lane;
-      const int32_t my_r = my_row < d.n_valid ? rec[my_row].x : rec[0].x;
       const uint32_t qdst = sbase + Lay::kQ + st * Lay::kQBytes;
       const uint16_t* qb = reinterpret_cast<const uint16_t*>(P.q);
 #pragma unroll
-      for (int it = 0; it < 32 / RPI; ++it) {
-        const int rr = it * RPI + lane / CPR, c = lane % CPR;
-        const int row = gw * 32 + rr;
-        const int32_t r = __shfl_sync(0xffffffffu, my_r, rr);
-        tc::cp_async16(qdst + (uint32_t)(c >> 3) * (kRows * 128) + tc::swz(row, c & 7),
-                       qb + (int64_t)r * D + c * 8, 16u);
+      for (int h = 0; h < 2; ++h) {
+        const int my_row = gw * 64 + h * 32 + lane;
+        const int32_t my_r = my_row < d.n_valid ? rec[my_row].x : rec[0].x;
+#pragma unroll
+        for (int it = 0; it < 32 / RPI; ++it) {
+          const int rr = it * RPI + lane / CPR, c = lane % CPR;
+          const int row = gw * 64 + h * 32 + rr;
+          const int32_t r = __shfl_sync(0xffffffffu, my_r, rr);
+          tc::cp_async16(qdst + (uint32_t)(c >> 3) * (kRows * 128) + tc::swz(row, c & 7),
+                         qb + (int64_t)r * D + c * 8, 16u);
+        }
       }
       tc::cp_async_mbar_arrive(&q_full[st]);
       if (*abort_v) {
@@ -362,70 +369,91 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp >= kEpiWarp0) {
+    // --------------------------------------------------------------- epilogue
+    // Tile after tile (both groups): O, already scaled by w / l through P, is
+    // rounded to bf16 and added into the output rows.  Warp e owns TMEM lanes
+    // 32 e .. 32 e + 31 (tile rows).  Each 64-column slice is staged in shared
+    // memory (row r's 16-byte chunk c at chunk c ^ (r & 7)) and read back so
+    // that one warp instruction adds 128 contiguous bytes into each of four
+    // rows.
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint8_t* stg = smem + Lay::kStage + (warp - kEpiWarp0) * Lay::kStageWarp;
+    uint16_t* const outp = reinterpret_cast<uint16_t*>(out);
+    bool ok = true;
+    for (int n = 0;; ++n) {
+      const int slot = n % kRing, g = n & 1, u = n >> 1;
+      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1) || *abort_v != 0) {
+        ok = false;
+        break;
+      }
+      const TileDesc d = desc[slot];
+      if (d.end) break;
+      const int32_t rid = row < d.n_valid ? meta[slot * kRows + row].x : -1;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
+      if (!tc::warp_wait(&o_full[g], u & 1)) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t to = tmem + lane_off + g * Lay::kGroupCols + Lay::kOCol;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t o[64];
+        {
+          uint32_t a[32], b[32];
+          tc::tmem_ld32(to + c0, a);
+          tc::tmem_ld32(to + c0 + 32, b);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            o[x] = a[x];
+            o[32 + x] = b[x];
+          }
+        }
+        if (c0 + 64 == D) {
+          // all of O is in registers: the group's next P V may overwrite it
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&o_free[g]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4 v;
+          v.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]), __uint_as_float(o[8 * q + 1]));
+          v.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
+          v.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]));
+          v.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
+          *reinterpret_cast<uint4*>(stg + tc::swz(lane, q)) = v;
+        }
+        __syncwarp();
+        int32_t r[8];
+        uint4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int src = 4 * i + (lane >> 3);
+          r[i] = __shfl_sync(0xffffffffu, rid, src);
+          v[i] = *reinterpret_cast<const uint4*>(stg + tc::swz(src, lane & 7));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (r[i] >= 0) tc::red_add_bf16x8(outp + (int64_t)r[i] * D + c0 + (lane & 7) * 8, v[i]);
+      }
+    }
+    if (!ok) *abort_v = 1;
   } else {
-    // ---------------------------------------------- softmax + epilogue groups
+    // -------------------------------------------------------- softmax groups
     const int g = (warp - kGroupWarp0) >> 2;
     const int quarter = warp & 3;                   // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tg = tmem + lane_off + g * Lay::kGroupCols;
     const float scale_log2 = P.inv_sqrt_d * 1.4426950408889634f;
-    uint8_t* stg = smem + Lay::kStage + (warp - kGroupWarp0) * Lay::kStageWarp;
-    const uint32_t stg_sw = (uint32_t)((lane >> 1) & 3);   // this row's chunk swizzle
-    uint16_t* const outp = reinterpret_cast<uint16_t*>(out);
-
-    // Epilogue of the group's tile number pu: O * (w / l) -> bf16, added into
-    // the output rows.  Each 32-column slice is staged per warp in shared
-    // memory (row r's 16-byte chunk c at chunk c ^ ((r >> 1) & 3)) and read
-    // back so that one warp instruction adds 64 contiguous bytes into each of
-    // eight rows.
-    auto epilogue = [&](int pu, float scale, int32_t rid) -> bool {
-      if (!tc::warp_wait(&o_full[g], pu & 1)) return false;
-      tc::tc_fence_after();
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tc::tmem_ld32(tg + Lay::kOCol + c0, o);
-        tc::tmem_ld_wait();
-        if (c0 + 32 == D) {
-          tc::tc_fence_before();
-          tc::mbar_arrive(&o_free[g]);
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 v;
-          v.x = tc::pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * scale,
-                                __uint_as_float(o[8 * q4 + 1]) * scale);
-          v.y = tc::pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * scale,
-                                __uint_as_float(o[8 * q4 + 3]) * scale);
-          v.z = tc::pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * scale,
-                                __uint_as_float(o[8 * q4 + 5]) * scale);
-          v.w = tc::pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * scale,
-                                __uint_as_float(o[8 * q4 + 7]) * scale);
-          *reinterpret_cast<uint4*>(stg + lane * kStageRowBytes + ((q4 ^ stg_sw) << 4)) = v;
-        }
-        __syncwarp();
-        int32_t r[4];
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int src = 8 * i + (lane >> 2), ch = lane & 3;
-          r[i] = __shfl_sync(0xffffffffu, rid, src);
-          v[i] = *reinterpret_cast<const uint4*>(stg + src * kStageRowBytes +
-                                                 ((ch ^ ((src >> 1) & 3)) << 4));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (r[i] >= 0) tc::red_add_bf16x8(outp + (int64_t)r[i] * D + c0 + (lane & 3) * 8, v[i]);
-      }
-      return true;
-    };
-
-    bool ok = true, has_prev = false;
-    int prev_u = 0;
-    float prev_scale = 0.f;
-    int32_t prev_rid = -1;
+    bool ok = true;
     for (int u = 0;; ++u) {
       const int n = 2 * u + g, slot = n % kRing;
       // every wait below is on an mbarrier whose phase the whole group (or
@@ -443,66 +471,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
       const int bf = u & 1;
-      float l = 0.f;
-      bool bad = !tc::warp_wait(&s_full[g][bf], (u >> 1) & 1);
-      if (!bad) {
-        tc::tc_fence_after();
-        uint32_t sr[64];
-        {
-          uint32_t a[32], c[32];
-          tc::tmem_ld32(tg + bf * kChunk, a);
-          tc::tmem_ld32(tg + bf * kChunk + 32, c);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            sr[x] = a[x];
-            sr[32 + x] = c[x];
-          }
-        }
-        // keys after the query exist only in the own chunk: a warp-uniform branch
-        const bool masked = !__all_sync(0xffffffffu, nk == kChunk);
-        float m = -INFINITY;
-        if (!masked) {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) m = fmaxf(m, __uint_as_float(sr[x]));
-        } else {
-#pragma unroll
-          for (int x = 0; x < 64; ++x)
-            if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
-        }
-        const float mb = m * scale_log2;
-        uint32_t pk[32];
-        float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int x = 0; x < 64; x += 2) {
-          float e0 = tc::ex2_approx(fmaf(__uint_as_float(sr[x]), scale_log2, -mb));
-          float e1 = tc::ex2_approx(fmaf(__uint_as_float(sr[x + 1]), scale_log2, -mb));
-          if (masked) {
-            e0 = x < nk ? e0 : 0.f;
-            e1 = x + 1 < nk ? e1 : 0.f;
-          }
-          l4[(x >> 1) & 3] += e0 + e1;
-          pk[x >> 1] = tc::pack_bf16x2(e0, e1);
-        }
-        l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-        // P over the first 32 columns of the S buffer (the logits are in registers)
-        tc::tmem_st32(tg + bf * kChunk, pk);
-        tc::tmem_st_wait();
-        tc::tc_fence_before();
-        tc::mbar_arrive(&sm_done[g][bf]);
-      }
-      if (has_prev && !bad) bad = !epilogue(prev_u, prev_scale, prev_rid);
-      if (bad) {
+      if (!tc::warp_wait(&s_full[g][bf], (u >> 1) & 1)) {
         ok = false;
-        has_prev = false;
         break;
       }
-      has_prev = true;
-      prev_u = u;
-      prev_rid = row_valid ? rec.x : -1;
-      prev_scale = l > 0.f ? __int_as_float(rec.y) / l : 0.f;
+      tc::tc_fence_after();
+      uint32_t sr[64];
+      {
+        uint32_t a[32], c[32];
+        tc::tmem_ld32(tg + bf * kChunk, a);
+        tc::tmem_ld32(tg + bf * kChunk + 32, c);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          sr[x] = a[x];
+          sr[32 + x] = c[x];
+        }
+      }
+      // keys after the query exist only in the own chunk: a warp-uniform branch
+      const bool masked = !__all_sync(0xffffffffu, nk == kChunk);
+      float m = -INFINITY;
+      if (!masked) {
+#pragma unroll
+        for (int x = 0; x < 64; ++x) m = fmaxf(m, __uint_as_float(sr[x]));
+      } else {
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x < nk) m = fmaxf(m, __uint_as_float(sr[x]));
+      }
+      const float mb = m * scale_log2;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int x = 0; x < 64; ++x) {
+        float e = tc::ex2_approx(fmaf(__uint_as_float(sr[x]), scale_log2, -mb));
+        if (masked) e = x < nk ? e : 0.f;
+        l4[x & 3] += e;
+        sr[x] = __float_as_uint(e);
+      }
+      const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      // P scaled by the fusion weight over l, so that P V is already this
+      // pair's share of the output
+      const float scale = (row_valid && l > 0.f) ? __int_as_float(rec.y) / l : 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        pk[x] = tc::pack_bf16x2(__uint_as_float(sr[2 * x]) * scale,
+                                __uint_as_float(sr[2 * x + 1]) * scale);
+      // P over the first 32 columns of the S buffer (the logits are in registers)
+      tc::tmem_st32(tg + bf * kChunk, pk);
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&sm_done[g][bf]);
     }
-    if (ok && has_prev && !epilogue(prev_u, prev_scale, prev_rid)) ok = false;
     if (!ok) *abort_v = 1;
   }
 

@@ -1,11 +1,12 @@
 // Prefill calibration, landmark scoring, selection and fusion weights (a1-a4)
 // for bf16 inputs, as two kernels:
 //
-//   calib_kernel (a1)   one thread per query row computes q~ = q + (qA)B in
-//       float32 and splits it into three bf16 terms hi + mid + lo (each the
-//       bf16 rounding of what is left, so q~ - (hi + mid + lo) is below
-//       2^-27 |q~|).  The terms are written as ready-made shared-memory
-//       images: per 128-row tile, three K-major 128-byte-swizzled tiles.
+//   calib_kernel (a1)   computes q~ = q + (qA)B in float32 per 128-row tile
+//       (t = qA first, then t B by column chunks) and splits it into three
+//       bf16 terms hi + mid + lo (each the bf16 rounding of what is left, so
+//       q~ - (hi + mid + lo) is below 2^-27 |q~|).  The terms are written as
+//       ready-made shared-memory images: per 128-row tile, three K-major
+//       128-byte-swizzled tiles.
 //   score_select_kernel (a2-a4)  persistent and warp-specialised; per
 //       128-row tile one bulk copy brings the three term tiles in, and for
 //       every block of 128 causally visible chunks S = sum over terms
@@ -49,16 +50,29 @@ struct ScoreLayout {
 };
 
 // ---- a1: calibration ------------------------------------------------------
-// RP = calibration rank rounded up (A staged as [D][RP] with zero columns).
-// Each thread computes NR rows (row tid of NR consecutive tiles), so every
-// 16-byte broadcast load of A or B feeds NR x 4 FMAs.
-template <int D, int RP, int NR>
+// RP = calibration rank rounded up (A staged as [D][RP] with zero columns, B as
+// [RP][D] with zero rows).  One CTA of 128 threads takes 128-row tiles in
+// turn, in two phases per tile:
+//   1. t = q A, float32: thread x computes, for rows x % 64 and x % 64 + 64,
+//      the half x / 64 of the RP columns (each 16-byte broadcast load of A
+//      feeds 8 FMAs), into shared memory.
+//   2. q~ = q + t B, and its split into three bf16 terms: thread (warp w,
+//      lane l) owns the 16-byte column chunk c = l % CPR of RPT rows, so one
+//      load of a B chunk feeds all of them, and the lanes of a warp store
+//      whole 128-byte rows of the swizzled images.
+template <int D, int RP>
 __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, int T,
                                                       int64_t n_tiles) {
   using Lay = ScoreLayout<D>;
+  constexpr int CPR = D / 8;          // 16-byte chunks per row: 8 or 16
+  constexpr int RG = kThrS / CPR;     // row groups in phase 2: 16 or 8
+  constexpr int RPT = kRowsS / RG;    // rows per thread in phase 2: 8 or 16
+  constexpr int HA = RP / 2;          // rank columns per thread in phase 1
+  constexpr int TS = RP + 4;          // padded row of t in shared memory
   extern __shared__ float smf[];
-  float* sA = smf;            // [D][RP]
-  float* sB = smf + D * RP;   // [RP][D]
+  float* sA = smf;                    // [D][RP]
+  float* sB = sA + D * RP;            // [RP][D]
+  float* sT = sB + RP * D;            // [kRowsS][TS]
   const int tid = threadIdx.x;
   for (int x = tid; x < D * RP; x += kThrS) {
     const int e = x / RP, a = x % RP;
@@ -66,107 +80,112 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
   }
   for (int x = tid; x < RP * D; x += kThrS) sB[x] = x < P.r * D ? P.Bm[x] : 0.f;
   __syncthreads();
-
-  const int64_t n_groups = (n_tiles + NR - 1) / NR;
-  for (int64_t gg = blockIdx.x; gg < n_groups; gg += gridDim.x) {
-    int64_t qoff[NR];
-    bool valid[NR];
+  const uint16_t* qb = reinterpret_cast<const uint16_t*>(P.q);
+  auto unpack = [](uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int v = 0; v < NR; ++v) {
-      const int64_t g = gg * NR + v;
-      const int t = (int)(g % T);
-      const int64_t bh = g / T;
-      const int h = (int)(bh % P.Hq), b = (int)(bh / P.Hq);
-      const int64_t i = (int64_t)t * kRowsS + tid;
-      valid[v] = g < n_tiles && i < P.L;
-      qoff[v] = valid[v] ? (((int64_t)b * P.L + i) * P.Hq + h) * D : 0;
+    for (int a = 0; a < 4; ++a) {
+      f[2 * a] = __uint_as_float(w[a] << 16);
+      f[2 * a + 1] = __uint_as_float(w[a] & 0xFFFF0000u);
     }
-    // t = q A: one accumulator chain per rank column, summed over e in order
-    float ta[NR][RP];
-#pragma unroll
-    for (int v = 0; v < NR; ++v)
-#pragma unroll
-      for (int a = 0; a < RP; ++a) ta[v][a] = 0.f;
-    // q is read 8 elements (16 bytes) at a time; the next group's load is
-    // issued before the current one is used, so its latency overlaps the FMAs
-    const uint16_t* qb = reinterpret_cast<const uint16_t*>(P.q);
-    auto ldq = [&](int v, int e) -> uint4 {
-      return valid[v] ? __ldg(reinterpret_cast<const uint4*>(qb + qoff[v] + e)) : make_uint4(0, 0, 0, 0);
+  };
+
+  for (int64_t gt = blockIdx.x; gt < n_tiles; gt += gridDim.x) {
+    const int t = (int)(gt % T);
+    const int64_t bh = gt / T;
+    const int h = (int)(bh % P.Hq), b = (int)(bh / P.Hq);
+    auto row_off = [&](int r, bool& valid) -> int64_t {
+      const int64_t i = (int64_t)t * kRowsS + r;
+      valid = i < P.L;
+      return valid ? (((int64_t)b * P.L + i) * P.Hq + h) * D : 0;
     };
-    auto unpack = [](uint4 u, float (&f)[8]) {
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        f[2 * a] = __uint_as_float(w[a] << 16);
-        f[2 * a + 1] = __uint_as_float(w[a] & 0xFFFF0000u);
-      }
-    };
+    // ---- phase 1: t = q A (rows r0 and r0 + 64, rank columns a0 .. a0 + HA)
     if (P.r > 0) {
-      uint4 qr[NR], qn[NR];
+      const int r0 = tid & 63, a0 = (tid >> 6) * HA;
+      bool v0, v1;
+      const int64_t o0 = row_off(r0, v0), o1 = row_off(r0 + 64, v1);
+      float ta[2][HA];
 #pragma unroll
-      for (int v = 0; v < NR; ++v) qr[v] = ldq(v, 0);
+      for (int a = 0; a < HA; ++a) ta[0][a] = ta[1][a] = 0.f;
+      auto ldq = [&](bool v, int64_t o, int e) -> uint4 {
+        return v ? __ldg(reinterpret_cast<const uint4*>(qb + o + e)) : make_uint4(0, 0, 0, 0);
+      };
+      uint4 q0 = ldq(v0, o0, 0), q1 = ldq(v1, o1, 0);
 #pragma unroll 1
       for (int e0 = 0; e0 < D; e0 += 8) {
-#pragma unroll
-        for (int v = 0; v < NR; ++v) qn[v] = e0 + 8 < D ? ldq(v, e0 + 8) : qr[v];
-        float qv[NR][8];
-#pragma unroll
-        for (int v = 0; v < NR; ++v) unpack(qr[v], qv[v]);
+        // the next 16 bytes are requested before these are used
+        const uint4 n0 = e0 + 8 < D ? ldq(v0, o0, e0 + 8) : q0;
+        const uint4 n1 = e0 + 8 < D ? ldq(v1, o1, e0 + 8) : q1;
+        float f0[8], f1[8];
+        unpack(q0, f0);
+        unpack(q1, f1);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
 #pragma unroll
-          for (int a = 0; a < RP; a += 4) {
-            const float4 av = *reinterpret_cast<const float4*>(sA + (e0 + u) * RP + a);
-#pragma unroll
-            for (int v = 0; v < NR; ++v) {
-              ta[v][a] = fmaf(qv[v][u], av.x, ta[v][a]);
-              ta[v][a + 1] = fmaf(qv[v][u], av.y, ta[v][a + 1]);
-              ta[v][a + 2] = fmaf(qv[v][u], av.z, ta[v][a + 2]);
-              ta[v][a + 3] = fmaf(qv[v][u], av.w, ta[v][a + 3]);
-            }
+          for (int a = 0; a < HA; a += 4) {
+            const float4 av = *reinterpret_cast<const float4*>(sA + (e0 + u) * RP + a0 + a);
+            ta[0][a] = fmaf(f0[u], av.x, ta[0][a]);
+            ta[0][a + 1] = fmaf(f0[u], av.y, ta[0][a + 1]);
+            ta[0][a + 2] = fmaf(f0[u], av.z, ta[0][a + 2]);
+            ta[0][a + 3] = fmaf(f0[u], av.w, ta[0][a + 3]);
+            ta[1][a] = fmaf(f1[u], av.x, ta[1][a]);
+            ta[1][a + 1] = fmaf(f1[u], av.y, ta[1][a + 1]);
+            ta[1][a + 2] = fmaf(f1[u], av.z, ta[1][a + 2]);
+            ta[1][a + 3] = fmaf(f1[u], av.w, ta[1][a + 3]);
           }
         }
+        q0 = n0;
+        q1 = n1;
+      }
 #pragma unroll
-        for (int v = 0; v < NR; ++v) qr[v] = qn[v];
+      for (int a = 0; a < HA; a += 4) {
+        *reinterpret_cast<float4*>(sT + r0 * TS + a0 + a) =
+            make_float4(ta[0][a], ta[0][a + 1], ta[0][a + 2], ta[0][a + 3]);
+        *reinterpret_cast<float4*>(sT + (r0 + 64) * TS + a0 + a) =
+            make_float4(ta[1][a], ta[1][a + 1], ta[1][a + 2], ta[1][a + 3]);
       }
     }
-    // q~ = q + t B (a ascending), then the three-term split, 8 elements at a time
-    uint4 xr[NR], xn[NR];
-#pragma unroll
-    for (int v = 0; v < NR; ++v) xr[v] = ldq(v, 0);
+    __syncthreads();
+    // ---- phase 2: q~ = q + t B for chunk c of rows rg, rg + RG, .. (8 at a time)
+    const int c = tid % CPR, rg = tid / CPR;
 #pragma unroll 1
-    for (int c = 0; c < D / 8; ++c) {
+    for (int j0 = 0; j0 < RPT; j0 += 8) {
+      float acc[8][8];
 #pragma unroll
-      for (int v = 0; v < NR; ++v) xn[v] = c + 1 < D / 8 ? ldq(v, (c + 1) * 8) : xr[v];
-      float x[NR][8];
+      for (int j = 0; j < 8; ++j) {
+        bool v;
+        const int64_t o = row_off(rg + RG * (j0 + j), v);
+        const uint4 u = v ? __ldg(reinterpret_cast<const uint4*>(qb + o + c * 8))
+                          : make_uint4(0, 0, 0, 0);
+        unpack(u, acc[j]);
+      }
+#pragma unroll 1
+      for (int a = 0; a < P.r; a += 4) {
+        float bv[4][8];
 #pragma unroll
-      for (int v = 0; v < NR; ++v) unpack(xr[v], x[v]);
+        for (int aa = 0; aa < 4; ++aa) {
+          const float4 b0 = *reinterpret_cast<const float4*>(sB + (a + aa) * D + c * 8);
+          const float4 b1 = *reinterpret_cast<const float4*>(sB + (a + aa) * D + c * 8 + 4);
+          bv[aa][0] = b0.x; bv[aa][1] = b0.y; bv[aa][2] = b0.z; bv[aa][3] = b0.w;
+          bv[aa][4] = b1.x; bv[aa][5] = b1.y; bv[aa][6] = b1.z; bv[aa][7] = b1.w;
+        }
 #pragma unroll
-      for (int a = 0; a < RP; ++a) {
-        if (a < P.r) {
-          const float4 b0 = *reinterpret_cast<const float4*>(sB + a * D + c * 8);
-          const float4 b1 = *reinterpret_cast<const float4*>(sB + a * D + c * 8 + 4);
+        for (int j = 0; j < 8; ++j) {
+          const float4 tv = *reinterpret_cast<const float4*>(sT + (rg + RG * (j0 + j)) * TS + a);
+          const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
-          for (int v = 0; v < NR; ++v) {
-            x[v][0] = fmaf(ta[v][a], b0.x, x[v][0]);
-            x[v][1] = fmaf(ta[v][a], b0.y, x[v][1]);
-            x[v][2] = fmaf(ta[v][a], b0.z, x[v][2]);
-            x[v][3] = fmaf(ta[v][a], b0.w, x[v][3]);
-            x[v][4] = fmaf(ta[v][a], b1.x, x[v][4]);
-            x[v][5] = fmaf(ta[v][a], b1.y, x[v][5]);
-            x[v][6] = fmaf(ta[v][a], b1.z, x[v][6]);
-            x[v][7] = fmaf(ta[v][a], b1.w, x[v][7]);
-          }
+          for (int aa = 0; aa < 4; ++aa)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[j][u] = fmaf(tt[aa], bv[aa][u], acc[j][u]);
         }
       }
-      const uint32_t off = (uint32_t)(c >> 3) * (kRowsS * 128) + tc::swz(tid, c & 7);
+      uint8_t* img = qimg + gt * (int64_t)Lay::kQimg + (uint32_t)(c >> 3) * (kRowsS * 128);
 #pragma unroll
-      for (int v = 0; v < NR; ++v) {
-        if (gg * NR + v >= n_tiles) continue;
+      for (int j = 0; j < 8; ++j) {
         uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          float x0 = x[v][2 * u], x1 = x[v][2 * u + 1];
+          float x0 = acc[j][2 * u], x1 = acc[j][2 * u + 1];
           hw[u] = tc::pack_bf16x2(x0, x1);
           x0 -= __uint_as_float(hw[u] << 16);
           x1 -= __uint_as_float(hw[u] & 0xFFFF0000u);
@@ -175,14 +194,13 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
           x1 -= __uint_as_float(mw[u] & 0xFFFF0000u);
           lw[u] = tc::pack_bf16x2(x0, x1);
         }
-        uint8_t* img = qimg + (gg * NR + v) * Lay::kQimg;
+        const uint32_t off = tc::swz(rg + RG * (j0 + j), c & 7);
         *reinterpret_cast<uint4*>(img + 0 * Lay::kQt + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(img + 1 * Lay::kQt + off) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
         *reinterpret_cast<uint4*>(img + 2 * Lay::kQt + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
-#pragma unroll
-      for (int v = 0; v < NR; ++v) xr[v] = xn[v];
     }
+    __syncthreads();   // t of the next tile goes where this one's was
   }
 }
 
@@ -764,23 +782,18 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
 template <int D, int RP>
 cudaError_t run_calib(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, int n_sm,
                       cudaStream_t s) {
-  constexpr int NR = RP <= 32 ? 2 : 1;
-  const size_t sm = sizeof(float) * 2 * D * RP;
-  cudaError_t e = set_smem(calib_kernel<D, RP, NR>, sm);
+  const size_t sm = sizeof(float) * (2 * D * RP + kRowsS * (RP + 4));
+  cudaError_t e = set_smem(calib_kernel<D, RP>, sm);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_kernel<D, RP, NR>, kThrS, sm);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_kernel<D, RP>, kThrS, sm);
   if (e != cudaSuccess) return e;
-  const int64_t grid = min((n_tiles + NR - 1) / NR, (int64_t)n_sm * max(1, per_sm));
+  const int64_t grid = min(n_tiles, (int64_t)n_sm * max(1, per_sm));
   HILS_PROFILE("prefill.calib", s);
-  calib_kernel<D, RP, NR><<<(unsigned)grid, kThrS, sm, s>>>(P, qimg, T, n_tiles);
+  calib_kernel<D, RP><<<(unsigned)grid, kThrS, sm, s>>>(P, qimg, T, n_tiles);
   return cudaGetLastError();
 }
 
-// The landmark tensor [B][max_chunks][Hkv][D] as a 4-d TMA map, innermost
-// first; one box = 64 dimensions x 128 chunks of one (sequence, KV head), in
-// the 128-byte swizzle the MMA descriptors expect.  Chunks past max_chunks
-// read as zeros.
 template <int D>
 cudaError_t landmark_tmap(const Params& P, CUtensorMap* tm) {
   const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hkv, (uint64_t)P.max_chunks, (uint64_t)P.B};

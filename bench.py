@@ -1,12 +1,14 @@
 #!/usr/bin/env python
 """Benchmark of the HiLS attention forward on B200 through the C-ABI library.
 
-A step is one pass of the whole hot path over one synthetic batch: the full
-prefill forward of the 128K-token GQA workload (B1, Hq32/Hkv8, d128, S64,
-k32, r32): calibration, landmark scoring, top-k selection, fusion weights,
-per-chunk attention and the fused merge.  The decode step (512K-token
-context, B1, H16, d64, k16) is timed in the same run and reported under
-"decode".
+A step is one pass of the whole hot path over one synthetic batch.  The
+headline line times the full prefill forward of the 128K-token GQA workload
+(B1, Hq32/Hkv8, d128, S64, k32, r32): calibration, landmark scoring, top-k
+selection, fusion weights, per-chunk attention and the fused merge.  The
+decode step at a 512K-token context (B1, H16, d64, k16) is timed in the same
+run under "decode", and the other workloads under "configs": the tiny float32
+problem, the 8K prefill, the decode of 32 sequences at 128K, and the decode at
+4M tokens (with the recall of its planted needle chunks).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,7 +38,7 @@ import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_KERNELS_PER_STEP = 7   # calib, score+select, bucket count, scan totals, scan, scatter, attend + merge (bf16)
-DECODE_KERNELS_PER_STEP = 2    # scan (append, calibration, scores, selection), attend (+merge)
+DECODE_KERNELS_PER_STEP = 1    # one kernel: append, calibration, scores, selection, attention
 
 
 def peaks():
@@ -323,6 +325,94 @@ def time_decode(hils, torch, wl, warmup_steps=8, n_steps=0):
     return times, phases
 
 
+def prefill_report(w: hi.Workload, ms: float, phases: dict, steps: int, n_ranks: int,
+                   clocks: dict) -> dict:
+    """Throughput and roofline of a timed prefill run.  The roofline is that of
+    the dominant kernel: its algorithmic flops per launch over its average
+    event-timed launch duration, against the measured dense bf16 peak (the
+    burst figure when the SM clock held its maximum during the run, the
+    sustained one otherwise)."""
+    pk, pk_src = peaks()
+    counts = prefill_counts(w)
+    dom_name, (dom_ms_total, dom_launches) = max(phases.items(), key=lambda kv: kv[1][0])
+    dom_ms = dom_ms_total / max(1, dom_launches)
+    if dom_name.startswith("prefill.score_select"):
+        work, what = counts["score_flop"], "useful landmark-scoring flop (q~ . landmark, causal chunks)"
+    else:
+        work, what = counts["attention_flop"], "useful attention flop (QK^T + PV over selected keys)"
+    at_max = bool(clocks.get("sm_mhz")) and clocks.get("sm_max_mhz") and \
+        clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"]
+    peak = pk["bf16_tflops"] if at_max else pk["bf16_tflops_sustained"]
+    achieved = work / (dom_ms / 1e3) / 1e12
+    traffic = attn_traffic(counts["pairs"]) if dom_name == "prefill.attend_tc" else None
+    bf16 = w.dtype == hi.DT_BF16
+    return {
+        "workload": w.name, "ms_per_step": ms,
+        "tok_per_s": weak_scaling_value(w.batch * w.seq_len, n_ranks, ms),
+        "kernels_ms_per_step": {k: v[0] / max(1, steps) for k, v in phases.items()},
+        "useful_attention_tflops": counts["attention_flop"] / (ms / 1e3) / 1e12,
+        "step_frac_of_peak": counts["attention_flop"] / (ms / 1e3) / 1e12 / peak,
+        "roofline": {"bound": "tensor" if bf16 else "alu", "kernel": dom_name,
+                     "achieved": achieved, "peak": peak if bf16 else None, "unit": "TFLOP/s",
+                     "frac": achieved / peak if bf16 else None, "traffic": traffic,
+                     "traffic_source": "ncu dram bytes scaled by (row, slot) pairs" if traffic else None,
+                     "work_per_launch": work, "work": what,
+                     "peak_source": (f"{pk_src} bf16 " + ("burst (SM clock at its maximum during the run)"
+                                                          if at_max else "sustained"))
+                     if bf16 else "float32 CUDA-core path: no tensor-core roofline"},
+    }
+
+
+def decode_report(dw: hi.Workload, times: list, phases: dict, n_ranks: int, maxreduce) -> dict:
+    """Step time and HBM roofline of a timed decode run: the step's algorithmic
+    bytes (every visible landmark, the selected K/V, q, out and the appended
+    k/v) over the graph-replayed step time, against the measured copy
+    bandwidth."""
+    pk, pk_src = peaks()
+    us = maxreduce(statistics.mean(times)) * 1e3
+    by = [decode_bytes(dw, s) for s in range(len(times))]
+    tot = statistics.mean(b["total"] for b in by)
+    kvb = statistics.mean(b["kv_bytes"] for b in by)
+    lmb = statistics.mean(b["landmark_bytes"] for b in by)
+    gbs = tot / (us / 1e6) / 1e9
+    return {
+        "workload": dw.name, "us_per_step": us, "us_per_step_median": statistics.median(times) * 1e3,
+        "steps": len(times), "batch": dw.batch, "context": dw.seq_len, "bytes_per_step": tot,
+        "landmark_bytes": lmb, "kv_bytes": kvb,
+        "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3 for k, v in phases.items()},
+        "roofline": {"bound": "hbm", "kernel": "decode step (one kernel)", "achieved": gbs,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                     "traffic": None, "peak_source": f"{pk_src} HBM copy bandwidth"},
+        "timing": "CUDA graph replay of one step; inputs staged and L2 flushed (256 MB write) "
+                  "before it; only the replay is timed",
+        "gpu_launches": DECODE_KERNELS_PER_STEP * len(times),
+    }
+
+
+def decode_needle_recall(hils, torch, wl) -> dict:
+    """Step 0 of a decode workload with planted needle chunks: the share of
+    (sequence, query head) selections that hold every needle."""
+    w = wl["workload"]
+    cfg = cfg_of(hils, w)
+    cache = make_cache(hils, wl)
+    nbytes = hils.workspace_size(cfg, hils.OP_DECODE, 1, wl["max_chunks"])
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    dt = torch.bfloat16 if w.dtype == hi.DT_BF16 else torch.float32
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=dt, device="cuda")
+    idx = torch.empty((w.batch, w.n_q_heads, w.top_k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.batch, w.n_q_heads, w.top_k), dtype=torch.float32, device="cuda")
+    seq0 = wl["seq_lens"].clone()
+    hils.decode(cfg, wl["q_dec"][0], wl["k_new"][0], wl["v_new"][0], wl["A"], wl["B"], cache, out,
+                idx, wt, ws, nbytes)
+    hils.device_status()
+    wl["seq_lens"].copy_(seq0)
+    sel = idx.cpu().numpy()
+    needles = set(int(c) for c in wl["needle_chunks"])
+    hit = [needles <= set(sel[b, h, 1:].tolist()) for b in range(w.batch) for h in range(w.n_q_heads)]
+    return {"needles": sorted(needles), "heads_with_all_needles": int(sum(hit)),
+            "heads": len(hit), "recall": sum(hit) / len(hit)}
+
+
 # ----------------------------------------------------------------- oracle (CPU)
 def oracle_prefill_sample(wl, budget_s: float, rng_seed: int = 0):
     """Time the CPU oracle on a sample of the prefill workload's rows for about
@@ -414,6 +504,10 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="timed decode steps (default: all of the workload's steps)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only the headline prefill and decode workloads")
+    ap.add_argument("--config-decode-steps", type=int, default=64,
+                    help="timed decode steps of the B=32 and 4M decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     args = ap.parse_args()
@@ -477,74 +571,69 @@ def main():
     torch.cuda.synchronize()
     ms, phases, clocks, _keep = time_prefill(hils, torch, wl, args.steps, args.warmup, barrier,
                                              maxreduce)
-    value = weak_scaling_value(tokens_per_rank, nworld, ms)
-    pk, pk_src = peaks()
-    # dominant kernel of the prefill step
-    dom = max(phases.items(), key=lambda kv: kv[1][0])
-    dom_name, (dom_ms_total, dom_launches) = dom
-    dom_ms = dom_ms_total / max(1, dom_launches)
-    if dom_name.startswith("prefill.attend"):
-        work, what = counts["attention_flop"], "useful attention flop (QK^T + PV over selected keys)"
-    elif dom_name.startswith("prefill.score_select"):
-        work, what = counts["score_flop"], "useful landmark-scoring flop (q~ . landmark, causal chunks)"
-    else:
-        work, what = counts["attention_flop"], "useful attention flop"
-    achieved = work / (dom_ms / 1e3) / 1e12
-    traffic = attn_traffic(counts["pairs"]) if dom_name == "prefill.attend_tc" else None
-    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
-                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,
-                "traffic_source": "ncu dram bytes on prefill_16k_gqa scaled by (row, slot) pairs"
-                                  if traffic else None,
-                "work_per_launch": work, "work": what,
-                "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)"}
+    rep = prefill_report(w, ms, phases, args.steps, nworld, clocks)
+    value = rep["tok_per_s"]
     result = {
         "metric": metric, "value": value, "unit": "tok/s", "n_gpus": nworld, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1), seeded", "config": config,
-        "clocks": clocks, "roofline": roofline,
+        "clocks": clocks, "roofline": rep["roofline"],
         "gpu_launches": PREFILL_KERNELS_PER_STEP * args.steps,
-        "kernels_ms_per_step": {k: v[0] / max(1, args.steps) for k, v in phases.items()},
-        "useful_attention_tflops": counts["attention_flop"] / (ms / 1e3) / 1e12,
+        "kernels_ms_per_step": rep["kernels_ms_per_step"],
+        "useful_attention_tflops": rep["useful_attention_tflops"],
+        "step_frac_of_peak": rep["step_frac_of_peak"],
     }
     del _keep
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = time_prefill_e2e(hils, torch, wl, max(1, min(args.steps, 3)), 1)
+        e2e_ms, h2d, d2h = time_prefill_e2e(hils, torch, wl, args.steps, 1)
         e2e_ms = maxreduce(e2e_ms)
         result["e2e"] = {"value": weak_scaling_value(tokens_per_rank, nworld, e2e_ms), "unit": "tok/s",
-                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                         "steps": args.steps}
     del wl
     torch.cuda.empty_cache()
+    configs = {}
     if not args.no_decode:
         dw = hi.WORKLOADS[args.decode_workload]
         dwl = hi.device_workload(dw, seed_offset=rank)
         times, dph = time_decode(hils, torch, dwl, n_steps=args.decode_steps)
-        us = maxreduce(statistics.mean(times)) * 1e3
-        by = [decode_bytes(dw, s) for s in range(len(times))]
-        tot = statistics.mean(b["total"] for b in by)
-        kvb = statistics.mean(b["kv_bytes"] for b in by)
-        lmb = statistics.mean(b["landmark_bytes"] for b in by)
-        result["decode"] = {
-            "workload": dw.name, "us_per_step": us, "steps": len(times),
-            "context": dw.seq_len, "bytes_per_step": tot, "landmark_bytes": lmb, "kv_bytes": kvb,
-            "step_gbs": tot / (us / 1e6) / 1e9,
-            "step_hbm_frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"],
-            "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3 for k, v in dph.items()},
-            # the step's kernels overlap (programmatic dependent launch), so the
-            # roofline is taken over the whole step: its algorithmic bytes / step time
-            "roofline": {"bound": "hbm", "kernel": "decode step (scan + attend, overlapped)",
-                         "achieved": tot / (us / 1e6) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": tot / (us / 1e6) / 1e9 / pk["hbm_gbs"], "traffic": None,
-                         "peak_source": f"{pk_src} HBM copy bandwidth"},
-            "timing": "CUDA graph replay of one step; inputs staged and L2 flushed (256 MB write) before it; only the replay is timed",
-            "gpu_launches": DECODE_KERNELS_PER_STEP * len(times),
-        }
+        result["decode"] = decode_report(dw, times, dph, nworld, maxreduce)
         del dwl
+        torch.cuda.empty_cache()
+    if not args.no_configs:
+        # the other workloads: a line each, same timing rules
+        for name in ("tiny_f32", "prefill_8k"):
+            pw = hi.WORKLOADS[name]
+            pwl = hi.device_workload(pw, seed_offset=rank)
+            pms, pph, pclk, keep = time_prefill(hils, torch, pwl, max(args.steps, 20), args.warmup,
+                                                barrier, maxreduce)
+            configs[name] = prefill_report(pw, pms, pph, max(args.steps, 20), nworld, pclk)
+            configs[name]["clocks"] = pclk
+            del keep, pwl
+            torch.cuda.empty_cache()
+        for name, n in (("decode_128k_b32", args.config_decode_steps),
+                        ("decode_4m", args.config_decode_steps)):
+            dw = hi.WORKLOADS[name]
+            dwl = hi.device_workload(dw, seed_offset=rank)
+            recall = decode_needle_recall(hils, torch, dwl) if dw.needles else None
+            times, dph = time_decode(hils, torch, dwl, n_steps=n)
+            configs[name] = decode_report(dw, times, dph, nworld, maxreduce)
+            if recall is not None:
+                configs[name]["needle_recall_step0"] = recall
+            del dwl
+            torch.cuda.empty_cache()
+        result["configs"] = configs
     if rank == 0 and nworld == 1 and not args.no_cpu_baseline:
+        from oracle import oracle
         wl = hi.device_workload(w)
         n, el, threads, sample = oracle_prefill_sample(wl, args.cpu_budget)
         result["cpu_baseline"] = {"value": n / el / w.n_q_heads, "unit": "tok/s", "cores": threads,
                                   "kind": "oracle", "sample": sample}
+        oracle.set_threads(1)
+        n1, el1, _, sample1 = oracle_prefill_sample(wl, max(2.0, args.cpu_budget / 3), rng_seed=1)
+        oracle.set_threads(threads)
+        result["cpu_baseline_1core"] = {"value": n1 / el1 / w.n_q_heads, "unit": "tok/s", "cores": 1,
+                                        "kind": "oracle", "sample": sample1}
     if rank == 0:
         print(json.dumps(result))
     if nworld > 1:

@@ -4,17 +4,18 @@
 // selection, and waits for the first before reading its results).
 //
 //   scan    grid (n_split, Hkv, B), 256 threads.  A CTA owns one KV head and a
-//           contiguous range of chunks of one sequence.  Every thread first
-//           issues the small loads (A, B, the group's queries, the own
-//           landmark), then its 256 bytes of landmark rows; q~ = q + (q A) B of
-//           the group's query heads is computed while the landmarks land, then
-//           every chunk of the range is scored.  Per query head, each warp
-//           sorts its part of the range with a bitonic network on 64-bit keys
-//           (score, then chunk) and the warps' sorted lists are merged pairwise
-//           (a tree of bitonic merges): the range's best k-1, best first.  The
-//           last CTA of a (sequence, KV head) -- one ticket per CTA -- merges
-//           the ranges' lists the same way, adds the own chunk (its score from
-//           the own landmark), writes the selection, the fusion weights and the
+//           contiguous range of chunks of one sequence.  One thread starts TMA
+//           copies of the range's landmark rows (64 KB, 128-byte swizzle) into
+//           shared memory; meanwhile every thread loads A, B, the group's
+//           queries and the own landmark, and q~ = q + (q A) B of the group's
+//           query heads is computed.  Every chunk of the range is then scored
+//           from shared memory.  Per query head, each warp sorts its part of
+//           the range with a bitonic network on 64-bit keys (score, then
+//           chunk) and the warps' sorted lists are merged pairwise: the range's
+//           best k-1, best first.  The last CTA of a (sequence, KV head) -- one
+//           ticket per CTA, taken with acquire-release ordering -- merges the
+//           ranges' lists the same way, adds the own chunk (its score from the
+//           own landmark), writes the selection, the fusion weights and the
 //           selected pages, and starts bringing those pages' K and V into L2.
 //           The first CTA of a (sequence, KV head) appends k_t and v_t.
 //   attend  grid (n_cta, Hq, B) in clusters of n_cta CTAs, one cluster per
@@ -42,8 +43,11 @@ namespace {
 
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kThreads = kScanThreads;
+constexpr int kWarps = kScanWarps;
 constexpr int kSlotThreads = 128;
 constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kLmBytes = 65536;   // landmark rows staged per scan CTA
 
 // Selection keys.  The high word is the score mapped to an unsigned order
 // (-0 taken as +0), the low word ~j, so a larger key ranks higher in (score
@@ -146,134 +150,155 @@ __device__ __forceinline__ int64_t decode_pos(const Params& P, int b, bool appen
   return t;
 }
 
-// Landmark work of one scan thread: 256 bytes of one KV head's landmark rows.
+// Ticket of the calling thread on `p`, with acquire-release ordering at device
+// scope: the writes this CTA made before it (published to this thread through
+// a CTA barrier) are visible to whoever takes a later ticket, and theirs to
+// this CTA.
+__device__ __forceinline__ int ticket(int32_t* p) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
+// Landmark geometry of one CTA: kLmBytes of landmark rows, CPS chunks of one KV
+// head, staged as NCB column blocks of CPS rows x 128 bytes (128-byte swizzle).
 template <int D, int EB>
-struct ScanGeo {
-  static constexpr int SLICE = 256 / EB;                  // landmark elements per thread
-  static constexpr int CPT = SLICE >= D ? SLICE / D : 1;  // chunks per thread
-  static constexpr int TPC = SLICE >= D ? 1 : D / SLICE;  // threads per chunk
-  static constexpr int EPT = SLICE >= D ? D : SLICE;      // elements per (thread, chunk)
-  static constexpr int CPS = kScanThreads * CPT / TPC;    // chunks per CTA
-  static constexpr int EPU = 16 / EB;                     // elements per 16-byte load
-  static constexpr int UPC = EPT / EPU;                   // 16-byte loads per (thread, chunk)
-  static constexpr int SEG = CPS / kScanWarps;            // chunks a warp sorts
-  static constexpr int V = SEG >= 32 ? SEG / 32 : 1;     // keys per lane in the warp sort
+struct Geo {
+  static constexpr int ROWB = D * EB;                // bytes of one landmark row
+  static constexpr int CPS = kLmBytes / ROWB;        // chunks per CTA: 512, 256 or 128
+  static constexpr int NCB = ROWB / 128;             // 128-byte column blocks per row
+  static constexpr int BOXR = CPS < 256 ? CPS : 256; // rows per TMA box
+  static constexpr int NRB = CPS / BOXR;             // boxes along the chunks
+  static constexpr int TPC = CPS >= kThreads ? 1 : kThreads / CPS;   // threads per chunk
+  static constexpr int CPT = CPS >= kThreads ? CPS / kThreads : 1;   // chunks per thread
+  static constexpr int UNITS = ROWB / 16;            // 16-byte units per row
+  static constexpr int UPT = UNITS / TPC;            // units per (thread, chunk)
+  static constexpr int EPU = 16 / EB;                // elements per unit
+  static constexpr int SEG = CPS / kWarps;           // chunks a warp sorts
+  static constexpr int V = SEG >= 32 ? SEG / 32 : 1; // keys per lane in the warp sort
 };
 
-// Dynamic shared memory of the scan, in this order: A [D][r], B [r][D] (float),
-// raw q [group][D], q~ [group][D + 4], q A [group][kMaxRank], scores
-// [CPS][group], own landmark [D], the warps' lists [kScanWarps][32] (64-bit),
-// and, for the last CTA, the ranges' lists of one head [n_split][k-1] (64-bit).
+// Dynamic shared memory of the scan after the 1024-byte-aligned landmark
+// block, in this order: A [D][r], B [r][D] (float), raw q [group][D], q~
+// [group][D + 4], q A [group][kMaxRank], scores [CPS][group], own landmark
+// [D], the warps' lists [kScanWarps][32] (64-bit), and, for the last CTA, the
+// ranges' lists of one head [n_split][k-1] (64-bit).
 struct ScanSmem {
-  int D, r, group, cps, n_split, K;
+  int D, r, group, cps, n_split, k;
   __host__ __device__ size_t floats() const {
     return (size_t)2 * D * r + (size_t)group * D + (size_t)group * (D + 4) +
            (size_t)group * kMaxRank + (size_t)cps * group + D;
   }
-  __host__ __device__ size_t lists_off() const { return (floats() * 4 + 15) & ~(size_t)15; }
+  __host__ __device__ size_t lists_off() const {
+    return kLmBytes + ((floats() * 4 + 15) & ~(size_t)15);
+  }
   __host__ __device__ size_t merge_off() const { return lists_off() + kScanWarps * 32 * 8; }
   __host__ __device__ size_t bytes() const {
-    return merge_off() + (size_t)n_split * (K > 0 ? K : 1) * 8;
+    return merge_off() + (size_t)n_split * (k > 1 ? k - 1 : 1) * 8 + 1024;   // + alignment slack
   }
 };
 
 template <int D, int EB>
-__global__ void __launch_bounds__(kScanThreads, 2)
-    scan_kernel(Params P, const void* k_new, const void* v_new, DecodeWs ws, int32_t* idx_out,
-                float* w_out) {
-  using G = ScanGeo<D, EB>;
+__global__ void __launch_bounds__(kThreads, 2)
+    scan_kernel(Params P, const __grid_constant__ CUtensorMap tm_lm, const void* k_new,
+                const void* v_new, DecodeWs ws, int32_t* idx_out, float* w_out) {
+  using G = Geo<D, EB>;
   // the attention grid may be scheduled now; it waits for this one before its reads
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int QS = D + 4;                        // padded q~ row
   const int group = P.group, K = P.k - 1;
-  const ScanSmem L{D, P.r, group, G::CPS, ws.n_split, K};
-  extern __shared__ __align__(16) uint8_t sraw[];
-  float* sA = reinterpret_cast<float*>(sraw);      // [D][r]
-  float* sB = sA + D * P.r;                        // [r][D]
-  float* sq = sB + P.r * D;                        // [group][D] raw q
-  float* sqt = sq + group * D;                     // [group][QS] q~
-  float* sT = sqt + group * QS;                    // [group][kMaxRank] q A
-  float* sS = sT + group * kMaxRank;               // [CPS][group] scores
-  float* slm = sS + G::CPS * group;                // [D] own chunk's landmark
-  uint64_t* wl = reinterpret_cast<uint64_t*>(sraw + L.lists_off());   // [kScanWarps][32]
-  uint64_t* ml = reinterpret_cast<uint64_t*>(sraw + L.merge_off());   // [n_split][K]
+  const ScanSmem L{D, P.r, group, G::CPS, ws.n_split, P.k};
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t lm_bar;
   __shared__ int last;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint8_t* lmb = smem;                                   // landmark rows (TMA destination)
+  float* sA = reinterpret_cast<float*>(smem + kLmBytes); // [D][r]
+  float* sB = sA + D * P.r;                              // [r][D]
+  float* sq = sB + P.r * D;                              // [group][D] raw q
+  float* sqt = sq + group * D;                           // [group][QS] q~
+  float* sT = sqt + group * QS;                          // [group][kMaxRank] q A
+  float* sS = sT + group * kMaxRank;                     // [CPS][group] scores
+  float* slm = sS + G::CPS * group;                      // [D] own chunk's landmark
+  uint64_t* wl = reinterpret_cast<uint64_t*>(smem + L.lists_off());   // [kWarps][32]
+  uint64_t* ml = reinterpret_cast<uint64_t*>(smem + L.merge_off());   // [n_split][K]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const bool append = ws.append != 0;
   const int64_t t = decode_pos(P, b, append, tid == 0 && split == 0 && g == 0);
   const int64_t own = t / kChunk;
-  const int cps = ws.chunks_per_split;                          // chunks of this range (<= CPS)
+  const int cps = ws.chunks_per_split;            // chunks of this range (<= CPS)
   const int64_t c0 = (int64_t)split * cps;
-  const int cl0 = G::TPC == 1 ? tid * G::CPT : tid / G::TPC;   // first local chunk
-  const int part = G::TPC == 1 ? 0 : tid % G::TPC;              // element part of the row
+  const bool any_cand = c0 < own;                 // the range holds a chunk before the own one
 
-  // ---- loads: the small ones first, then the landmark rows; q~ is computed
-  // while the landmark rows are still in flight ----------------------------------
-  constexpr int NQ = (64 * D / G::EPU + kScanThreads - 1) / kScanThreads;
-  const int nq = group * D / G::EPU;
-  uint4 rq[NQ], rl = make_uint4(0, 0, 0, 0);
+  // ---- loads: the landmark rows by TMA, the small inputs by every thread ------
+  if (tid == 0) {
+    tc::mbar_init(&lm_bar, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0 && any_cand) {
+    tc::mbar_arrive_expect_tx(&lm_bar, kLmBytes);
+#pragma unroll
+    for (int rb = 0; rb < G::NRB; ++rb)
+#pragma unroll
+      for (int cb = 0; cb < G::NCB; ++cb)
+        tc::tma_load_4d(tc::smem_u32(lmb + cb * (G::CPS * 128) + rb * (G::BOXR * 128)), &tm_lm,
+                        cb * (128 / EB), g, (int)(c0 + rb * G::BOXR), b, &lm_bar);
+  }
   {
-    const int na = D * P.r / 4;
+    constexpr int NQ = (64 * D / G::EPU + kThreads - 1) / kThreads;
+    const int na = D * P.r / 4, nq = group * D / G::EPU;
     // A and B straight into shared memory (asynchronous copies, no registers)
-    for (int x = tid; x < na; x += kScanThreads) {
+    for (int x = tid; x < na; x += kThreads) {
       tc::cp_async16(tc::smem_u32(sA + 4 * x), reinterpret_cast<const float4*>(P.A) + x, 16u);
       tc::cp_async16(tc::smem_u32(sB + 4 * x), reinterpret_cast<const float4*>(P.Bm) + x, 16u);
     }
     tc::cp_async_commit();
+    uint4 rq[NQ], rl = make_uint4(0, 0, 0, 0);
     const uint4* qsrc = reinterpret_cast<const uint4*>(
         reinterpret_cast<const uint8_t*>(P.q) + ((int64_t)b * P.Hq + (int64_t)g * group) * D * EB);
 #pragma unroll
     for (int u = 0; u < NQ; ++u) {
-      const int x = u * kScanThreads + tid;
+      const int x = u * kThreads + tid;
       if (x < nq) rq[u] = __ldg(qsrc + x);
     }
     if (tid < D / G::EPU)
       rl = __ldg(reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(P.landmarks) +
           (((int64_t)b * P.max_chunks + own) * P.Hkv + g) * D * EB) + tid);
-  }
-  uint4 lm[G::CPT][G::UPC];
+    // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
+    if (append && split == 0 && tid < 2 * (D / G::EPU)) {
+      const int64_t page = page_of(P, b, own);
+      if (page >= 0) {
+        const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x;
+        uint4* dst = reinterpret_cast<uint4*>(
+            reinterpret_cast<uint8_t*>(const_cast<void*>(P.pages)) +
+            page_offset(P, page, kind, g, (int)(t % kChunk)) * EB) + x;
+        *dst = __ldg(src);
+      }
+    }
 #pragma unroll
-  for (int ci = 0; ci < G::CPT; ++ci) {
-    const int64_t j = c0 + cl0 + ci;
-    const bool cand = cl0 + ci < cps && j < own;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        reinterpret_cast<const uint8_t*>(P.landmarks) +
-        ((((int64_t)b * P.max_chunks + (cand ? j : 0)) * P.Hkv + g) * D + part * G::EPT) * EB);
+    for (int u = 0; u < NQ; ++u) {
+      const int x = u * kThreads + tid;
+      if (x < nq) {
+        float v[G::EPU];
+        unpack16<EB>(rq[u], v);
 #pragma unroll
-    for (int u = 0; u < G::UPC; ++u) lm[ci][u] = cand ? __ldcs(src + u) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int u = 0; u < NQ; ++u) {
-    const int x = u * kScanThreads + tid;
-    if (x < nq) {
+        for (int e = 0; e < G::EPU; ++e) sq[x * G::EPU + e] = v[e];
+      }
+    }
+    if (tid < D / G::EPU) {
       float v[G::EPU];
-      unpack16<EB>(rq[u], v);
+      unpack16<EB>(rl, v);
 #pragma unroll
-      for (int e = 0; e < G::EPU; ++e) sq[x * G::EPU + e] = v[e];
+      for (int e = 0; e < G::EPU; ++e) slm[tid * G::EPU + e] = v[e];
     }
+    tc::cp_async_wait<0>();
   }
-  if (tid < D / G::EPU) {
-    float v[G::EPU];
-    unpack16<EB>(rl, v);
-#pragma unroll
-    for (int e = 0; e < G::EPU; ++e) slm[tid * G::EPU + e] = v[e];
-  }
-  // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
-  if (append && split == 0 && tid < 2 * (D / G::EPU)) {
-    const int64_t page = page_of(P, b, own);
-    if (page >= 0) {
-      const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
-      const uint4* src = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint8_t*>(kind ? v_new : k_new) + ((int64_t)b * P.Hkv + g) * D * EB) + x;
-      uint4* dst = reinterpret_cast<uint4*>(
-          reinterpret_cast<uint8_t*>(const_cast<void*>(P.pages)) +
-          page_offset(P, page, kind, g, (int)(t % kChunk)) * EB) + x;
-      *dst = __ldg(src);
-    }
-  }
-  tc::cp_async_wait<0>();
   __syncthreads();
 
   // ---- a1: q~ = q + (q A) B of the group's heads --------------------------------
@@ -281,8 +306,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     // t[h][a]: LP lanes per (h, a) pair, each summing a strided part over e
     const int pairs = group * P.r;
     int LP = 32;
-    while (LP > 1 && LP * pairs > kScanThreads) LP >>= 1;
-    for (int base = 0; base < pairs * LP; base += kScanThreads) {
+    while (LP > 1 && LP * pairs > kThreads) LP >>= 1;
+    for (int base = 0; base < pairs * LP; base += kThreads) {
       const int x = base + tid;
       const int pr = x / LP, sub = x % LP;
       float acc = 0.f;
@@ -295,7 +320,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     }
     __syncthreads();
   }
-  for (int x = tid; x < group * D; x += kScanThreads) {
+  for (int x = tid; x < group * D; x += kThreads) {
     const int h = x / D, e = x % D;
     float acc = sq[x];
     for (int a = 0; a < P.r; ++a) acc = fmaf(sT[h * kMaxRank + a], sB[a * D + e], acc);
@@ -303,30 +328,40 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   }
   __syncthreads();
 
-  // ---- a2: scores of the range ----------------------------------------------------
+  // ---- a2: scores of the range, from the staged landmark rows ---------------------
+  bool lm_ok = true;
+  if (any_cand) lm_ok = tc::mbar_wait(&lm_bar, 0);
+  if (!lm_ok && tid == 0) set_device_error(kErrTimeout);
 #pragma unroll
   for (int ci = 0; ci < G::CPT; ++ci) {
-    const int64_t j = c0 + cl0 + ci;
+    const int cl = G::TPC == 1 ? tid + ci * kThreads : tid / G::TPC;   // local chunk
+    const int part = G::TPC == 1 ? 0 : tid % G::TPC;
+    const int64_t j = c0 + cl;
+    const bool cand = lm_ok && cl < cps && j < own;
     for (int hh = 0; hh < group; ++hh) {
-      const float* qt = sqt + hh * QS + part * G::EPT;
       float acc = 0.f;
+      if (cand) {
+        const float* qt = sqt + hh * QS;
 #pragma unroll
-      for (int u = 0; u < G::UPC; ++u) {
-        float lv[G::EPU];
-        unpack16<EB>(lm[ci][u], lv);
+        for (int v = 0; v < G::UPT; ++v) {
+          const int u = part * G::UPT + v;
+          const uint4 w4 = *reinterpret_cast<const uint4*>(lmb + (u >> 3) * (G::CPS * 128) +
+                                                           tc::swz(cl, u & 7));
+          float lv[G::EPU];
+          unpack16<EB>(w4, lv);
 #pragma unroll
-        for (int e = 0; e < G::EPU; e += 4) {
-          const float4 q4 = *reinterpret_cast<const float4*>(qt + u * G::EPU + e);
-          acc = fmaf(q4.x, lv[e], acc);
-          acc = fmaf(q4.y, lv[e + 1], acc);
-          acc = fmaf(q4.z, lv[e + 2], acc);
-          acc = fmaf(q4.w, lv[e + 3], acc);
+          for (int e = 0; e < G::EPU; e += 4) {
+            const float4 q4 = *reinterpret_cast<const float4*>(qt + u * G::EPU + e);
+            acc = fmaf(q4.x, lv[e], acc);
+            acc = fmaf(q4.y, lv[e + 1], acc);
+            acc = fmaf(q4.z, lv[e + 2], acc);
+            acc = fmaf(q4.w, lv[e + 3], acc);
+          }
         }
       }
 #pragma unroll
       for (int o = 1; o < G::TPC; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
-      if (part == 0)
-        sS[(cl0 + ci) * group + hh] = (cl0 + ci < cps && j < own) ? acc * P.inv_sqrt_d : -INFINITY;
+      if (part == 0) sS[cl * group + hh] = cand ? acc * P.inv_sqrt_d : -INFINITY;
     }
   }
   __syncthreads();
@@ -344,7 +379,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     }
     wl[warp * 32 + lane] = warp_top32<G::V>(v);
 #pragma unroll
-    for (int step = 1; step < kScanWarps; step <<= 1) {
+    for (int step = 1; step < kWarps; step <<= 1) {
       __syncthreads();
       if ((warp & (2 * step - 1)) == 0)
         wl[warp * 32 + lane] = warp_merge32(wl[warp * 32 + lane], wl[(warp + step) * 32 + lane]);
@@ -355,13 +390,11 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     __syncthreads();
   }
 
-  // ---- a3/a4: the last CTA of the (sequence, KV head) merges the ranges -----------
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last = atomicAdd(&ws.tickets[b * P.Hkv + g], 1) == ws.n_split - 1;
+  // ---- the last CTA of the (sequence, KV head) takes over -------------------------
+  if (tid == 0) last = ticket(&ws.tickets[b * P.Hkv + g]) == ws.n_split - 1;
   __syncthreads();
   if (!last) return;
-  __threadfence();
+
   for (int hh = 0; hh < group; ++hh) {
     const int h = g * group + hh;
     const int64_t bh = (int64_t)b * P.Hq + h;
@@ -658,21 +691,25 @@ void attend_shape(int k, int* spc, int* n_cta) {
   *spc = (k + *n_cta - 1) / *n_cta;
 }
 
-size_t scan_smem(const Params& P, int D, int cps, int n_split) {
-  const ScanSmem L{D, P.r, P.group, cps, n_split, P.k - 1};
-  return L.bytes();
-}
-
 template <int D, int EB>
 cudaError_t run_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                        int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s) {
+  using G = Geo<D, EB>;
   cudaError_t e;
   {
-    const size_t smem = scan_smem(P, D, ScanGeo<D, EB>::CPS, ws.n_split);
+    CUtensorMap tm;
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hkv, (uint64_t)P.max_chunks, (uint64_t)P.B};
+    const uint64_t strides[3] = {(uint64_t)D * EB, (uint64_t)P.Hkv * D * EB,
+                                 (uint64_t)P.max_chunks * P.Hkv * D * EB};
+    const uint32_t box[4] = {128u / EB, 1, (uint32_t)G::BOXR, 1};
+    if ((e = encode_tmap(&tm, EB == 2 ? HILS_BF16 : HILS_F32, 4, P.landmarks, dims, strides,
+                         box)) != cudaSuccess)
+      return e;
+    const size_t smem = ScanSmem{D, P.r, P.group, G::CPS, ws.n_split, P.k}.bytes();
     if ((e = set_smem(scan_kernel<D, EB>, smem)) != cudaSuccess) return e;
     HILS_PROFILE("decode.scan", s);
     scan_kernel<D, EB><<<dim3(ws.n_split, P.Hkv, P.B), kScanThreads, smem, s>>>(
-        P, k_new, v_new, ws, idx_out, w_out);
+        P, tm, k_new, v_new, ws, idx_out, w_out);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
@@ -698,9 +735,9 @@ cudaError_t run_decode(const Params& P, const void* k_new, const void* v_new, vo
   return cudaGetLastError();
 }
 
-int chunks_per_split(const Params& P) {
-  if (P.dtype == HILS_BF16) return P.d == 64 ? ScanGeo<64, 2>::CPS : ScanGeo<128, 2>::CPS;
-  return P.d == 64 ? ScanGeo<64, 4>::CPS : ScanGeo<128, 4>::CPS;
+int chunks_per_cta(const Params& P) {
+  if (P.dtype == HILS_BF16) return P.d == 64 ? Geo<64, 2>::CPS : Geo<128, 2>::CPS;
+  return P.d == 64 ? Geo<64, 4>::CPS : Geo<128, 4>::CPS;
 }
 
 }  // namespace
@@ -710,7 +747,7 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
   DecodeWs w{};
   // as few ranges as the CTA geometry allows, then the chunks spread evenly over them
-  const int cps_max = chunks_per_split(P);
+  const int cps_max = chunks_per_cta(P);
   w.n_split = (P.max_chunks + cps_max - 1) / cps_max;
   if (w.n_split < 1) w.n_split = 1;
   w.chunks_per_split = (P.max_chunks + w.n_split - 1) / w.n_split;
@@ -730,6 +767,10 @@ size_t decode_ws_bytes(const Params& P, DecodeWs* out, char* base) {
   w.tickets = (int32_t*)take(w.ticket_bytes);
   if (out) *out = w;
   return off;
+}
+
+size_t decode_smem_bytes(const Params& P, const DecodeWs& ws) {
+  return ScanSmem{P.d, P.r, P.group, chunks_per_cta(P), ws.n_split, P.k}.bytes();
 }
 
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,

@@ -271,6 +271,10 @@ int decode_call(const hils_config* cfg, const void* q, const void* k_new, const 
   if (w.n_split > kMaxSplitLists)
     return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
                 kMaxSplitLists, P.max_chunks, w.n_split);
+  if (decode_smem_bytes(P, w) > 227 * 1024)
+    return fail(HILS_ERR_UNSUPPORTED,
+                "decode of %d query heads per KV head over %d chunk ranges needs more shared "
+                "memory than a CTA has", P.group, w.n_split);
   if (!ws || ws_bytes < need)
     return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
   if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");

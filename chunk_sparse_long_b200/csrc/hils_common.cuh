@@ -140,6 +140,9 @@ cudaError_t set_smem(F* func, size_t bytes) {
 // 128-byte swizzle, elements outside the tensor read as zeros.
 cudaError_t encode_tmap_bf16(CUtensorMap* tm, int rank, const void* base, const uint64_t* dims,
                              const uint64_t* strides, const uint32_t* box);
+// The same for a tensor of `dtype` (HILS_BF16 or HILS_F32).
+cudaError_t encode_tmap(CUtensorMap* tm, int dtype, int rank, const void* base,
+                        const uint64_t* dims, const uint64_t* strides, const uint32_t* box);
 
 // ---- launchers (each returns cudaError_t of its launches) -----------------
 cudaError_t launch_score(const Params& P, float* scores, int n_cols, cudaStream_t s);
@@ -185,6 +188,8 @@ struct DecodeWs {
   int append;          // k_new / v_new given
 };
 size_t decode_ws_bytes(const Params& P, DecodeWs* ws, char* base);
+// Dynamic shared memory of the decode kernel for this configuration.
+size_t decode_smem_bytes(const Params& P, const DecodeWs& ws);
 // hils_decode with its scratch at `ws`: validates every argument, lays the
 // workspace out, then (clear_counters) zeroes its completion counters on the
 // stream and launches the step.  Nothing is queued when a check fails.

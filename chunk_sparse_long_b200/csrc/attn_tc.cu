@@ -159,12 +159,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kb = n_item & 1;
       for (int t = 0; t < nt; ++t, ++m) {
         const int slot = m % kRing;
-        if (m >= kRing && !tc::warp_wait(&ring_free[slot], ((m / kRing) - 1) & 1)) {
+        if (m >= kRing && !tc::warp_wait(&ring_free[slot], ((m / kRing) - 1) & 1, wait_limit())) {
           ok = false;
           break;
         }
         if (t == 0) {
-          if (n_item >= 2 && !tc::warp_wait(&kv_empty[kb], ((n_item >> 1) - 1) & 1)) {
+          if (n_item >= 2 && !tc::warp_wait(&kv_empty[kb], ((n_item >> 1) - 1) & 1, wait_limit())) {
             ok = false;
             break;
           }
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // two end markers: one for each group
     for (int e = 0; e < 2 && ok; ++e, ++m) {
       const int slot = m % kRing;
-      if (m >= kRing && !tc::warp_wait(&ring_free[slot], ((m / kRing) - 1) & 1)) {
+      if (m >= kRing && !tc::warp_wait(&ring_free[slot], ((m / kRing) - 1) & 1, wait_limit())) {
         ok = false;
         break;
       }
@@ -227,9 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       if (lane == 0) *abort_v = 1;
       // let the copies already issued land before the CTA exits (bounded waits)
-      for (int x = max(0, m - kRing); x < m; ++x) tc::mbar_wait(&ring_full[x % kRing], (x / kRing) & 1);
+      for (int x = max(0, m - kRing); x < m; ++x)
+        tc::mbar_wait(&ring_full[x % kRing], (x / kRing) & 1, kDrainLimitNs);
       for (int x = max(0, kv_issued - 2); x < kv_issued; ++x)
-        tc::mbar_wait(&kv_full[x & 1], (x >> 1) & 1);
+        tc::mbar_wait(&kv_full[x & 1], (x >> 1) & 1, kDrainLimitNs);
     }
   } else if (warp >= kGatherWarp0 && warp < kEpiWarp0) {
     // ---------------------------------------------------------------- gathers
@@ -243,11 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0;; ++n) {
       const int st = n % NS, slot = n % kRing;
-      if (n >= NS && !tc::warp_wait(&q_empty[st], ((n / NS) - 1) & 1)) {
+      if (n >= NS && !tc::warp_wait(&q_empty[st], ((n / NS) - 1) & 1, wait_limit())) {
         ok = false;
         break;
       }
-      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1)) {
+      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1, wait_limit())) {
         ok = false;
         break;
       }
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t now = tc::globaltimer_ns();
           if (idle == 256) {
             t_idle = now;
-          } else if (now - t_idle > 2000000000ull) {
+          } else if (now - t_idle > wait_limit()) {
             *abort_v = 1;
             break;
           }
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every product issued has finished before the CTA frees its TMEM
       if (issued) {
         tc::mma_commit(&drain);
-        tc::mbar_wait(&drain, 0);
+        tc::mbar_wait(&drain, 0, kDrainLimitNs);
       }
     }
     __syncwarp();
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0;; ++n) {
       const int slot = n % kRing, g = n & 1, u = n >> 1;
-      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1) || *abort_v != 0) {
+      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1, wait_limit()) || *abort_v != 0) {
         ok = false;
         break;
       }
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t rid = row < d.n_valid ? meta[slot * kRows + row].x : -1;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
-      if (!tc::warp_wait(&o_full[g], u & 1)) {
+      if (!tc::warp_wait(&o_full[g], u & 1, wait_limit())) {
         ok = false;
         break;
       }
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every wait below is on an mbarrier whose phase the whole group (or
       // the MMA thread) completes, so each warp goes its own pace; a warp
       // whose wait ran out leaves, and the others follow once theirs do
-      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1) || *abort_v != 0) {
+      if (!tc::warp_wait(&ring_full[slot], (n / kRing) & 1, wait_limit()) || *abort_v != 0) {
         ok = false;
         break;
       }
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
       const int bf = u & 1;
-      if (!tc::warp_wait(&s_full[g][bf], (u >> 1) & 1)) {
+      if (!tc::warp_wait(&s_full[g][bf], (u >> 1) & 1, wait_limit())) {
         ok = false;
         break;
       }

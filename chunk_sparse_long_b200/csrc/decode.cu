@@ -330,7 +330,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // ---- a2: scores of the range, from the staged landmark rows ---------------------
   bool lm_ok = true;
-  if (any_cand) lm_ok = tc::mbar_wait(&lm_bar, 0);
+  if (any_cand) {
+    lm_ok = tc::mbar_wait(&lm_bar, 0, wait_limit());
+    // a CTA that gave up still lets its copies land before it goes on
+    if (!lm_ok) tc::mbar_wait(&lm_bar, 0, kDrainLimitNs);
+  }
   if (!lm_ok && tid == 0) set_device_error(kErrTimeout);
 #pragma unroll
   for (int ci = 0; ci < G::CPT; ++ci) {

@@ -216,9 +216,16 @@ int hils_device_status(void* stream) {
   const int zero = 0;
   e = cudaMemcpyToSymbol(hils::g_device_error, &zero, sizeof zero);
   if (e != cudaSuccess) return cuda_fail(e, "hils_device_status: clear");
-  return fail(HILS_ERR_DEVICE_CHECK, "device bounds check fired (bits 0x%x: %s%s%s)", word,
+  return fail((word & hils::kErrTimeout) ? HILS_ERR_TIMEOUT : HILS_ERR_DEVICE_CHECK,
+              "device check fired (bits 0x%x: %s%s%s)", word,
               (word & hils::kErrPage) ? "page " : "", (word & hils::kErrChunk) ? "chunk " : "",
-              (word & hils::kErrTimeout) ? "timeout" : "");
+              (word & hils::kErrTimeout) ? "a bounded wait ran out" : "");
+}
+
+int hils_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t v = ns == 0 ? hils::kDrainLimitNs : ns;
+  cudaError_t e = cudaMemcpyToSymbol(hils::g_wait_limit_ns, &v, sizeof v);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_set_wait_limit_ns");
 }
 
 const char* hils_last_error(void) { return g_last_error.c_str(); }

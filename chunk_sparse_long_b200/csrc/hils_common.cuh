@@ -36,6 +36,15 @@ extern __device__ int g_device_error;
 
 __device__ __forceinline__ void set_device_error(int bit) { atomicOr(&g_device_error, bit); }
 
+// How long a kernel's waits on its pipeline (one stage waiting for another)
+// last before the kernel gives up and reports a timeout: 2 s unless a test
+// lowers it (hils_set_wait_limit_ns).  The waits that let a kernel's own
+// asynchronous copies and products finish before it exits always use
+// kDrainLimitNs, so that a kernel that gives up never leaves work in flight.
+extern __constant__ uint64_t g_wait_limit_ns;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+__device__ __forceinline__ uint64_t wait_limit() { return g_wait_limit_ns; }
+
 // Plain parameters of one call, passed by value to every kernel.
 struct Params {
   int B, Hq, Hkv, d, k, r, dtype;

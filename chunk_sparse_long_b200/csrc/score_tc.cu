@@ -427,8 +427,8 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
           tc::tma_load_4d(dst + c * (kBlk * 128), &tm_lm, c * 64, g, s.blk * kBlk, b, &lm_bar[nb]);
       };
       // waits for the MMAs of step m
-      auto mma_done = [&](int m) {
-        return tc::mbar_wait_sleep(&s_full[m % kSBufs], (uint32_t)(m / kSBufs) & 1u);
+      auto mma_done = [&](int m, uint64_t limit) {
+        return tc::mbar_wait_sleep(&s_full[m % kSBufs], (uint32_t)(m / kSBufs) & 1u, limit);
       };
       Step st, pf;
       step_set(st, blockIdx.x, P, T, n_tiles);
@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
         }
         if (st.pass == 0 && st.blk == 0) {
           // the previous tile's MMAs must be done before its q~ terms are replaced
-          if (n > 0 && !mma_done(n - 1)) {
+          if (n > 0 && !mma_done(n - 1, wait_limit())) {
             ok = false;
             break;
           }
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
               tc::bulk_prefetch_l2(qimg + ((int64_t)nx.bh * T + nx.t) * (int64_t)Lay::kQimg,
                                    Lay::kQimg);
           }
-          if (!tc::mbar_wait_sleep(&qbar, qphase)) {
+          if (!tc::mbar_wait_sleep(&qbar, qphase, wait_limit())) {
             ok = false;
             break;
           }
@@ -470,11 +470,12 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
           qphase ^= 1;
         }
         const int sb = n % kSBufs;
-        if (n >= kSBufs && !tc::mbar_wait_sleep(&s_free[sb], (uint32_t)(n / kSBufs - 1) & 1u)) {
+        if (n >= kSBufs &&
+            !tc::mbar_wait_sleep(&s_free[sb], (uint32_t)(n / kSBufs - 1) & 1u, wait_limit())) {
           ok = false;
           break;
         }
-        if (!tc::mbar_wait_sleep(&lm_bar[n & 1], (uint32_t)(n >> 1) & 1u)) {
+        if (!tc::mbar_wait_sleep(&lm_bar[n & 1], (uint32_t)(n >> 1) & 1u, wait_limit())) {
           ok = false;
           break;
         }
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
         mma_issued = n + 1;
         // step n+1's landmark block goes where step n-1's was: its MMAs must be done
         if (pf.w < n_tiles) {
-          if (n > 0 && !mma_done(n - 1)) {
+          if (n > 0 && !mma_done(n - 1, wait_limit())) {
             ok = false;
             break;
           }
@@ -508,10 +509,10 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
       if (!ok) {
         *abort_v = 1;
         // let what was issued land before the CTA exits (bounded waits)
-        if (mma_issued > 0) mma_done(mma_issued - 1);
+        if (mma_issued > 0) mma_done(mma_issued - 1, kDrainLimitNs);
         for (int m = mma_issued; m < lm_issued; ++m)
-          tc::mbar_wait_sleep(&lm_bar[m & 1], (uint32_t)(m >> 1) & 1u);
-        if (q_pending) tc::mbar_wait_sleep(&qbar, qphase);
+          tc::mbar_wait_sleep(&lm_bar[m & 1], (uint32_t)(m >> 1) & 1u, kDrainLimitNs);
+        if (q_pending) tc::mbar_wait_sleep(&qbar, qphase, kDrainLimitNs);
       }
     }
   } else {
@@ -759,7 +760,7 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
     step_set(st, blockIdx.x, P, T, n_tiles);
     for (int n = 0; st.w < n_tiles; step_next(st, P, T, n_tiles), ++n) {
       const int sb = n % kSBufs;
-      const bool got = tc::mbar_wait_sleep(&s_full[sb], (uint32_t)(n / kSBufs) & 1u);
+      const bool got = tc::mbar_wait_sleep(&s_full[sb], (uint32_t)(n / kSBufs) & 1u, wait_limit());
       // the pair decides together, so neither is ever left alone at its named barrier
       if (tc::named_barrier_or(bar_id, 64, !got || *abort_v != 0)) {
         if (lane == 0) *abort_v = 1;

@@ -8,6 +8,7 @@
 namespace hils {
 
 __device__ int g_device_error = 0;
+__constant__ uint64_t g_wait_limit_ns = kDrainLimitNs;
 
 namespace {
 

@@ -192,8 +192,9 @@ __device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
 
 // Bounded wait of every lane of the warp; true only if it succeeded in all of
 // them, so the warp leaves the wait with one decision.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
-  const bool ok = mbar_wait(bar, parity);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = 2000000000ull) {
+  const bool ok = mbar_wait(bar, parity, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

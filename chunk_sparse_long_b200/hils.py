@@ -26,7 +26,7 @@ STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
 EXPORTED = ("hils_workspace_size", "hils_score", "hils_topk", "hils_prefill", "hils_decode",
             "hils_device_status", "hils_last_error", "hils_version", "hils_profile_enable",
             "hils_profile_collect", "hils_profile_read", "hils_profile_reset",
-            "hils_decode_noalloc", "hils_decode_noalloc_capacity")
+            "hils_decode_noalloc", "hils_decode_noalloc_capacity", "hils_set_wait_limit_ns")
 
 
 class HilsError(RuntimeError):
@@ -92,6 +92,8 @@ def load(path: str = LIB_PATH):
     L.hils_decode_noalloc.argtypes = [cfgp, P, P, P, P, P, cachep, P, P, P, P]
     L.hils_decode_noalloc_capacity.restype = ctypes.c_size_t
     L.hils_decode_noalloc_capacity.argtypes = []
+    L.hils_set_wait_limit_ns.restype = ctypes.c_int
+    L.hils_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     _lib = L
     return L
 
@@ -193,6 +195,12 @@ def decode_noalloc(cfg, q, k_new, v_new, A, B, cache: Cache, out, idx_out, w_out
 
 def decode_noalloc_capacity() -> int:
     return int(load().hils_decode_noalloc_capacity())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Testing hook: kernels give up on a pipeline wait after ``ns`` nanoseconds
+    (0 restores the default) and report HILS_ERR_TIMEOUT."""
+    _check(load().hils_set_wait_limit_ns(int(ns)), "hils_set_wait_limit_ns")
 
 
 def device_status(stream=None):

@@ -150,9 +150,19 @@ int hils_decode_noalloc(const hils_config* cfg, const void* q, const void* k_new
 size_t hils_decode_noalloc_capacity(void);
 
 /* Synchronises `stream`, then reports and clears the device error word set by
- * the kernels' bounds checks: HILS_OK or HILS_ERR_DEVICE_CHECK (HILS_ERR_CUDA if the
+ * the kernels' checks: HILS_OK; HILS_ERR_TIMEOUT if a kernel gave up on a bounded
+ * wait (the results of that call are undefined; later calls are unaffected);
+ * HILS_ERR_DEVICE_CHECK if only a bounds check fired (HILS_ERR_CUDA if the
  * synchronisation itself failed). */
 int hils_device_status(void* stream);
+
+/* Testing hook for the failure path: every kernel wait on another stage of its
+ * pipeline gives up after `ns` nanoseconds (0 restores the default, 2 s), after
+ * which the kernel lets its own asynchronous copies and products finish, exits
+ * and reports HILS_ERR_TIMEOUT through hils_device_status().  A short limit
+ * makes calls give up while their pipelines are still filling.  Applies to the
+ * current device; not meant for production use. */
+int hils_set_wait_limit_ns(uint64_t ns);
 
 /* Kernel timing with CUDA events, for benchmarking (not thread-safe).
  * hils_profile_enable(1): from now on every kernel the library launches is

@@ -1,10 +1,12 @@
 """Parity at the benchmark sizes, in the launch configuration bench.py times.
 
 The full workloads are generated on the device (hils_inputs.device_workload).
-The CUDA path runs on all rows. Sampled rows are then checked against the
-oracle, one by one: 64 prefill rows at 128K and 256 at 8K, every head of two
-512K decode steps, every head of four of the 32 sequences for two B=32 decode
-steps, and every head of one 4M decode step. The check applies the same rule
+The CUDA path runs on all rows. Rows are then checked against the oracle, one
+by one.  Selection and fusion weights: every row at 8K (131,072 rows), and at
+128K every row of the last 1024 positions plus one row in 64 of the rest
+(98,304 rows).  Outputs as well: 64 prefill rows at 128K and 256 at 8K, every
+head of two 512K decode steps, every head of four of the 32 sequences for two
+B=32 decode steps, and every head of one 4M decode step. The check applies the same rule
 as the small tests: selection exact wherever the oracle's score gap exceeds
 1e-5, weights within 1e-5, and outputs within 2e-2 (bf16).
 
@@ -105,6 +107,64 @@ def _prefill_sampled(name, n_random, seed):
     g_out = out[sel[:, 0], sel[:, 1], sel[:, 2]].float().cpu().numpy()
     rep, _ = _check_rows(torch, hi, oracle, gu, wl, oc, rows_q, bb, heads, pos, g_idx, g_w, g_out)
     print(name, rep)
+
+
+def _prefill_selection_rows(name, pick):
+    """Selection and fusion weights of many rows (selection-only oracle: a few
+    flops per landmark, so every row at 8K and a dense share at 128K fit in
+    one test).  ``pick(L, Hq)`` gives the (position, head) rows to check."""
+    torch, hi, hils, oracle, gu = _libs()
+    w = hi.WORKLOADS[name]
+    wl = hi.device_workload(w)
+    cfg, oc = _cfgs(hils, oracle, w)
+    L, Hq, k = w.seq_len, w.n_q_heads, w.top_k
+    cache = hils.Cache(wl["pages"], wl["num_pages"], wl["block_table"], wl["max_chunks"],
+                       wl["landmarks"])
+    out = torch.empty_like(wl["q"])
+    idx = torch.empty((w.batch, L, Hq, k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((w.batch, L, Hq, k), dtype=torch.float32, device="cuda")
+    nbytes = hils.workspace_size(cfg, hils.OP_PREFILL, L, wl["max_chunks"])
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    hils.prefill(cfg, wl["q"], L, 0, wl["A"], wl["B"], cache, out, idx, wts, ws, nbytes)
+    hils.device_status()
+    del ws, out
+    pos, heads = pick(L, Hq)
+    bb = np.zeros(len(pos), dtype=np.int32)
+    sel = torch.from_numpy(np.stack([bb, pos, heads], 1)).to("cuda")
+    rows_q = _host(wl["q"][sel[:, 0], sel[:, 1], sel[:, 2]], w.dtype, hi)
+    g_idx = idx[sel[:, 0], sel[:, 1], sel[:, 2]].cpu().numpy()
+    g_w = wts[sel[:, 0], sel[:, 1], sel[:, 2]].cpu().numpy()
+    A, B = wl["A"].cpu().numpy(), wl["B"].cpu().numpy()
+    lm = _host(wl["landmarks"], w.dtype, hi)
+    bt = wl["block_table"].cpu().numpy()
+    orc = oracle.hils_rows(oc, rows_q, bb, heads, pos, A, B, None, bt, lm)
+
+    def rerun(ids, forced):
+        return oracle.hils_rows(oc, rows_q[ids], bb[ids], heads[ids], pos[ids], A, B, None, bt, lm,
+                                forced_idx=forced)
+
+    rep = gu.compare(g_idx, g_w, None, orc, rerun, w.dtype)
+    print(name, len(pos), "rows", rep)
+    return len(pos)
+
+
+def test_prefill_8k_selection_of_every_row_matches_oracle():
+    def every_row(L, Hq):
+        p, h = np.meshgrid(np.arange(L), np.arange(Hq), indexing="ij")
+        return p.reshape(-1).astype(np.int64), h.reshape(-1).astype(np.int32)
+    assert _prefill_selection_rows("prefill_8k", every_row) == 8192 * 16
+
+
+def test_prefill_128k_gqa_selection_of_dense_rows_matches_oracle():
+    """Every row of the last 1024 positions (the 8 tiles with the most landmark
+    blocks, 16 each) and one row in 64 over the whole sequence."""
+    def dense(L, Hq):
+        p1, h1 = np.meshgrid(np.arange(L - 1024, L), np.arange(Hq), indexing="ij")
+        r = np.arange(0, L * Hq, 64)
+        pos = np.concatenate([p1.reshape(-1), r // Hq]).astype(np.int64)
+        heads = np.concatenate([h1.reshape(-1), r % Hq]).astype(np.int32)
+        return pos, heads
+    assert _prefill_selection_rows("prefill_128k_gqa", dense) == 1024 * 32 + 131072 * 32 // 64
 
 
 def test_prefill_128k_gqa_sampled_rows_match_oracle():

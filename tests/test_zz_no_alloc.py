@@ -73,3 +73,48 @@ def test_noalloc_rejects_configurations_beyond_its_scratch():
     with pytest.raises(hils.HilsError) as e:
         hils.decode_noalloc(cfg, fake, None, None, fake, fake, cache, fake, None, None)
     assert e.value.status == 3 and "built-in" in str(e.value)
+
+
+def test_noalloc_clears_counters_left_by_a_larger_configuration():
+    """Every call starts from what the previous call left in the built-in
+    scratch.  A large configuration fills the start of the array with its
+    candidate lists; a small one that follows keeps its completion counters at
+    an offset inside that region, so it is correct only because the call
+    clears them first.  Its results must equal hils_decode on a zeroed
+    workspace."""
+    import gpu_util as gu
+    from chunk_sparse_long_b200 import hils
+    big = random_problem(batch=2, n_q_heads=32, n_kv_heads=4, head_dim=64, chunk_size=64,
+                         top_k=32, calib_rank=8, seq_len=36000, dtype=hi.DT_BF16, seed=33,
+                         spare_pages=2)
+    small = random_problem(batch=1, n_q_heads=2, n_kv_heads=2, head_dim=64, chunk_size=64,
+                           top_k=4, calib_rank=8, seq_len=300, dtype=hi.DT_BF16, seed=34,
+                           spare_pages=2)
+    nb_big = hils.workspace_size(gu.cfg_of(big), hils.OP_DECODE, 1, big.max_chunks)
+    nb_small = hils.workspace_size(gu.cfg_of(small), hils.OP_DECODE, 1, small.max_chunks)
+    assert nb_small < nb_big // 8 < hils.decode_noalloc_capacity()
+
+    def one_step(p, dp, noalloc):
+        t = p.seq_len - 1
+        dp.seq_lens.fill_(t + 1)
+        B, Hq, d, k = p.batch, p.n_q_heads, p.head_dim, p.top_k
+        q = dp.q[:, t].contiguous()
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device="cuda")
+        idx = torch.empty((B, Hq, k), dtype=torch.int32, device="cuda")
+        w = torch.empty((B, Hq, k), dtype=torch.float32, device="cuda")
+        if noalloc:
+            hils.decode_noalloc(dp.cfg, q, None, None, dp.A, dp.B, dp.cache, out, idx, w)
+        else:
+            nb = hils.workspace_size(dp.cfg, hils.OP_DECODE, 1, p.max_chunks)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+            hils.decode(dp.cfg, q, None, None, dp.A, dp.B, dp.cache, out, idx, w, ws, nb)
+        hils.device_status()
+        return idx.cpu().numpy(), w.cpu().numpy(), gu.to_f64(out)
+
+    one_step(big, gu.DevProblem(big), noalloc=True)     # leaves candidate keys in the scratch
+    dps = gu.DevProblem(small)
+    i1, w1, o1 = one_step(small, dps, noalloc=True)
+    i0, w0, o0 = one_step(small, dps, noalloc=False)
+    np.testing.assert_array_equal(i1, i0)
+    np.testing.assert_allclose(w1, w0, rtol=0, atol=1e-5)
+    assert np.abs(o1 - o0).max() <= 2e-2

@@ -38,7 +38,7 @@ import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_KERNELS_PER_STEP = 7   # calib, score+select, bucket count, scan totals, scan, scatter, attend + merge (bf16)
-DECODE_KERNELS_PER_STEP = 1    # one kernel: append, calibration, scores, selection, attention
+DECODE_KERNELS_PER_STEP = 2    # scan (append, calibration, scores, selection) + attend, overlapped by PDL
 
 
 def peaks():
@@ -51,12 +51,13 @@ def peaks():
 
 # ----------------------------------------------------------------- work counts
 # DRAM traffic of the attention kernel from one ncu capture on prefill_16k_gqa
-# (dram__bytes_read.sum + dram__bytes_write.sum = 4.391 GB for 15.76M pairs),
-# per (row, slot) pair; it grows with the pairs.  Valid only for the kernel
-# source it was taken on (sha256 below); otherwise the bench reports null.
+# (dram__bytes_read.sum + dram__bytes_write.sum = 697.8 MB + 115.3 MB for
+# 15.76M (row, slot) pairs), per pair; it grows with the pairs.  Valid only
+# for the kernel source it was taken on (sha256 below); otherwise the bench
+# reports null.
 ATTN_TRAFFIC = {"file": "chunk_sparse_long_b200/csrc/attn_tc.cu",
-                "sha256": "726b33a4854ca776577f02fa71415dc0a3b058fce348c6832b982bf4ea3a8afe",
-                "bytes_per_pair": (394345216 + 3976426752) / 15.76e6}
+                "sha256": "50c909ba895377dcaa23c4273998ef78fa7a7f1761ac1aeab87cc68af1f7e790",
+                "bytes_per_pair": (697821184 + 115285760) / 15761408}
 
 
 def attn_traffic(pairs: float):
@@ -380,7 +381,7 @@ def decode_report(dw: hi.Workload, times: list, phases: dict, n_ranks: int, maxr
         "steps": len(times), "batch": dw.batch, "context": dw.seq_len, "bytes_per_step": tot,
         "landmark_bytes": lmb, "kv_bytes": kvb,
         "kernels_us_per_step_serialized": {k: v[0] / max(1, v[1]) * 1e3 for k, v in phases.items()},
-        "roofline": {"bound": "hbm", "kernel": "decode step (one kernel)", "achieved": gbs,
+        "roofline": {"bound": "hbm", "kernel": "decode step (scan + attend, overlapped)", "achieved": gbs,
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                      "traffic": None, "peak_source": f"{pk_src} HBM copy bandwidth"},
         "timing": "CUDA graph replay of one step; inputs staged and L2 flushed (256 MB write) "

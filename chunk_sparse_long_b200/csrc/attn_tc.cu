@@ -296,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O = P V of tile np once its softmax is done and the group's O is free
         if (np < ns) {
           const int g = np & 1, u = np >> 1, bf = u & 1;
-          if (tc::mbar_try_wait(&sm_done[g][bf], (u >> 1) & 1) &&
-              (u == 0 || tc::mbar_try_wait(&o_free[g], (u - 1) & 1))) {
+          if (tc::mbar_test_wait(&sm_done[g][bf], (u >> 1) & 1) &&
+              (u == 0 || tc::mbar_test_wait(&o_free[g], (u - 1) & 1))) {
             tc::tc_fence_after();
             const TileDesc d = desc[np % kRing];
             const uint32_t vb = sbase + Lay::kV + d.kb * Lay::kKVBytes;
@@ -320,15 +320,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P V (which reads P from the buffer) was issued before this
         if (!s_done) {
           const int st = ns % NS;
-          if (tc::mbar_try_wait(&q_full[st], (ns / NS) & 1) &&
-              tc::mbar_try_wait(&ring_full[ns % kRing], (ns / kRing) & 1)) {
+          if (tc::mbar_test_wait(&q_full[st], (ns / NS) & 1) &&
+              tc::mbar_test_wait(&ring_full[ns % kRing], (ns / kRing) & 1)) {
             const TileDesc d = desc[ns % kRing];
             const int g = ns & 1, u = ns >> 1, bf = u & 1;
             if (d.end) {
               s_done = true;
-            } else if ((!d.first || tc::mbar_try_wait(&kv_full[d.kb], d.kv_phase)) &&
+            } else if ((!d.first || tc::mbar_test_wait(&kv_full[d.kb], d.kv_phase)) &&
                        (u < 2 || (np > ns - 4 &&
-                                  tc::mbar_try_wait(&sm_done[g][bf], ((u >> 1) - 1) & 1)))) {
+                                  tc::mbar_test_wait(&sm_done[g][bf], ((u >> 1) - 1) & 1)))) {
               tc::tc_fence_after();
               const uint32_t qst = sbase + Lay::kQ + st * Lay::kQBytes;
               const uint32_t kbuf = sbase + Lay::kK + d.kb * Lay::kKVBytes;

@@ -197,6 +197,10 @@ WORKLOADS = {
     # the 128K GQA shape at 16K tokens: a profiling-size case (a few GB on the device)
     "prefill_16k_gqa": Workload("prefill_16k_gqa", 1, 32, 8, 128, 64, 32, 32, DT_BF16, 16384, 3,
                                 "prefill"),
+    # the 128K GQA shape at 512K tokens: a long prefill in one call (about 26 GB
+    # of workspace, 43 GB on the device in all)
+    "prefill_512k_gqa": Workload("prefill_512k_gqa", 1, 32, 8, 128, 64, 32, 32, DT_BF16,
+                                 524288, 6, "prefill"),
     "decode_512k": Workload("decode_512k", 1, 16, 16, 64, 64, 16, 16, DT_BF16, 524288, 4,
                             "decode", decode_steps=256),
     "decode_128k_b32": Workload("decode_128k_b32", 32, 16, 16, 64, 64, 16, 16, DT_BF16, 131072,

@@ -139,11 +139,14 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
  * every GPU that loads the library holds until the process exits; a
  * configuration that needs more returns HILS_ERR_WORKSPACE (use hils_decode).
  * The first call on each device looks up the array's device address; make
- * that first call before any stream capture.  Each call clears the array's
+ * that first call before any stream capture, and make no call after
+ * cudaDeviceReset (the looked-up address is kept for the life of the
+ * process).  Each call that passes its argument checks clears the array's
  * completion counters (a cudaMemsetAsync on `stream`) and otherwise reuses
- * what the previous call left there.  All calls on one device share the array:
- * calls that overlap on the GPU (other streams, other threads) race and give
- * wrong results, so serialise them.  Allocates no memory. */
+ * what the previous call left there; a rejected call queues nothing.  All
+ * calls on one device share the array: calls that overlap on the GPU (other
+ * streams, other threads) race and give wrong results, so serialise them.
+ * Allocates no memory. */
 int hils_decode_noalloc(const hils_config* cfg, const void* q, const void* k_new,
                         const void* v_new, const float* A, const float* B, hils_kv_cache* cache,
                         void* out, int32_t* idx_out, float* w_out, void* stream);

@@ -4,10 +4,10 @@ The full workloads are generated on the device (hils_inputs.device_workload).
 The CUDA path runs on all rows. Rows are then checked against the oracle, one
 by one.  Selection and fusion weights: every row at 8K (131,072 rows), and at
 128K every row of the last 1024 positions plus one row in 64 of the rest
-(98,304 rows).  Outputs as well: 64 prefill rows at 128K and 256 at 8K, every
-head of two 512K decode steps, every head of four of the 32 sequences for two
-B=32 decode steps, and every head of one 4M decode step. The check applies the same rule
-as the small tests: selection exact wherever the oracle's score gap exceeds
+(98,304 rows).  Outputs as well: 64 prefill rows at 128K and at 512K, 256 at
+8K, every head of two 512K decode steps, every head of four of the 32
+sequences for two B=32 decode steps, and every head of one 4M decode step.
+The check applies the same rule as the small tests: selection exact wherever the oracle's score gap exceeds
 1e-5, weights within 1e-5, and outputs within 2e-2 (bf16).
 
 The oracle is given a compact page pool. It holds only the chunks that a
@@ -173,6 +173,13 @@ def test_prefill_128k_gqa_sampled_rows_match_oracle():
 
 def test_prefill_8k_sampled_rows_match_oracle():
     _prefill_sampled("prefill_8k", 240, 2025)
+
+
+def test_prefill_512k_gqa_in_one_call_sampled_rows_match_oracle():
+    """A 512K-token prefill at the 128K GQA shape in one call: its workspace
+    (selection, pair records, q~ images; no per-pair partial outputs) fits on
+    one GPU next to the inputs."""
+    _prefill_sampled("prefill_512k_gqa", 48, 2026)
 
 
 def _decode_steps(torch, hils, wl, cfg, n_steps):

@@ -8,8 +8,8 @@
 // per SM runs a warp-specialised pipeline over its items' tiles:
 //
 //   warp 0 (producer)  takes items in a fixed order.  Per tile a bulk copy of
-//       its 128 pair records (query row, fusion weight, visible keys) into a
-//       ring of kRing slots; per item one TMA copy of K and one of V (3-d
+//       its 128 pair records (query row; fusion weight with the visible keys
+//       in its lowest bits) into a ring of kRing slots; per item one TMA copy of K and one of V (3-d
 //       tensor map over the page pool) into one of two buffers.
 //   warps 10-11 (gathers)  per tile, the pairs' query rows into one of NS
 //       stages with 16-byte cp.async, 128-byte swizzled, 64 rows per warp.
@@ -50,6 +50,10 @@ constexpr int kEpiWarp0 = 12;     // warps 12-15: epilogue, one per TMEM lane qu
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRing = 8;          // tiles whose descriptors and pair records are in flight
+// One ring slot of 8-byte pair records: the tile's 128, copied from the
+// 16-byte boundary at or before its first, with room for the one before it
+// and the rounding of the copy to 16 bytes.
+constexpr uint32_t kMetaSlot = (kRows + 2) * 8;
 constexpr uint32_t kStageRowBytes = 128;  // epilogue staging: 64 bf16 of one row
 
 template <int D>
@@ -62,8 +66,8 @@ struct AttnLayout {
   static constexpr uint32_t kV = kK + 2 * kKVBytes;     // two V buffers
   static constexpr uint32_t kStage = kV + 2 * kKVBytes; // 4 warps x 32 rows x 128 bytes
   static constexpr uint32_t kStageWarp = 32 * kStageRowBytes;
-  static constexpr uint32_t kMeta = kStage + 4 * kStageWarp;   // [kRing][128] pair records
-  static constexpr uint32_t kEnd = kMeta + kRing * kRows * 16;
+  static constexpr uint32_t kMeta = kStage + 4 * kStageWarp;   // [kRing] slots of pair records
+  static constexpr uint32_t kEnd = kMeta + kRing * kMetaSlot;
   static constexpr uint32_t kSmem = kEnd + 1024;                // + slack for 1024-byte alignment
   static_assert(kSmem + 1024 <= 232448, "dynamic + static shared memory above 227 KB");
   static constexpr uint32_t kTmemCols = 512;
@@ -78,6 +82,7 @@ struct TileDesc {
   int32_t kb;         // K/V buffer
   int32_t kv_phase;   // parity of that buffer's fill
   int32_t first, last, end;
+  int32_t rec0;       // record of tile row 0 in the ring slot (0 or 1)
 };
 
 template <int D>
@@ -95,7 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t sbase = tc::smem_u32(smem);
-  const int4* meta = reinterpret_cast<const int4*>(smem + Lay::kMeta);
+  // pair records of ring slot x, tile row r: meta[x * (kMetaSlot / 8) + desc[x].rec0 + r]
+  const int2* meta = reinterpret_cast<const int2*>(smem + Lay::kMeta);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_v = &abort_sh;
 
@@ -198,10 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           d.kv_phase = (n_item >> 1) & 1;
           d.first = t == 0;
           d.last = t == nt - 1;
+          // the copy starts at the 16-byte boundary at or before the tile's
+          // first record and covers whole 16-byte units (the workspace has
+          // room after the last record)
+          d.rec0 = d.tile_base & 1;
+          const uint32_t bytes = ((uint32_t)(d.rec0 + d.n_valid) * 8u + 15u) & ~15u;
           desc[slot] = d;
-          tc::mbar_arrive_expect_tx(&ring_full[slot], (uint32_t)d.n_valid * 16u);
-          tc::bulk_g2s_hint(sbase + Lay::kMeta + (uint32_t)slot * (kRows * 16),
-                            ws.pinfo + d.tile_base, (uint32_t)d.n_valid * 16u, &ring_full[slot],
+          tc::mbar_arrive_expect_tx(&ring_full[slot], bytes);
+          tc::bulk_g2s_hint(sbase + Lay::kMeta + (uint32_t)slot * kMetaSlot,
+                            ws.pinfo + (d.tile_base - d.rec0), bytes, &ring_full[slot],
                             stream_policy);
         }
       }
@@ -258,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive(&q_full[st]);
         break;
       }
-      const int4* rec = meta + slot * kRows;
+      const int2* rec = meta + slot * (kMetaSlot / 8) + d.rec0;
       const uint32_t qdst = sbase + Lay::kQ + st * Lay::kQBytes;
       const uint16_t* qb = reinterpret_cast<const uint16_t*>(P.q);
 #pragma unroll
@@ -392,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const TileDesc d = desc[slot];
       if (d.end) break;
-      const int32_t rid = row < d.n_valid ? meta[slot * kRows + row].x : -1;
+      const int32_t rid = row < d.n_valid ? meta[slot * (kMetaSlot / 8) + d.rec0 + row].x : -1;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
       if (!tc::warp_wait(&o_full[g], u & 1, wait_limit())) {
@@ -467,8 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileDesc d = desc[slot];
       if (d.end) break;
       const bool row_valid = row < d.n_valid;
-      const int4 rec = meta[slot * kRows + row];
-      const int nk = row_valid ? rec.z : kChunk;
+      const int2 rec = meta[slot * (kMetaSlot / 8) + d.rec0 + row];
+      const int nk = row_valid ? (rec.y & 63) + 1 : kChunk;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&ring_free[slot]);
       const int bf = u & 1;
@@ -512,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
       // P scaled by the fusion weight over l, so that P V is already this
       // pair's share of the output
-      const float scale = (row_valid && l > 0.f) ? __int_as_float(rec.y) / l : 0.f;
+      const float scale = (row_valid && l > 0.f) ? __int_as_float(rec.y & ~63) / l : 0.f;
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)

@@ -166,8 +166,8 @@ struct PrefillWs {
   int32_t* tile_off; // [n_keys + 1] tile offsets
   int32_t* cursor;   // [n_keys]
   int32_t* pairs;    // float32 path: [rows * k] pair ids (row * k + slot) in bucket order
-  int4* pinfo;       // bf16 path: [rows * k] (query row, fusion weight bits, visible keys, 0)
-                     // in bucket order
+  int2* pinfo;       // bf16 path: [rows * k] (query row, fusion weight bits with the visible
+                     // keys - 1 in the 6 lowest) in bucket order
   float* acc;        // [rows][d] float32 accumulator (CUDA-core attention)
   void* qimg;        // bf16: per 128-row tile the three q~ term tiles (shared-memory images)
   int4* items;       // [max_tiles] (key, first pair, end pair, 0) of every work item

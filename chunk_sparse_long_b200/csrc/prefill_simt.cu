@@ -175,13 +175,15 @@ __device__ __forceinline__ int64_t pair_key(const Params& P, Windows W, int64_t 
   return bucket_key(P, W, (int)(bi / P.L), h / P.group, bi % P.L, j);
 }
 
-// The record of pair (query row, chunk j) for the tensor-core attention:
-// (row, fusion weight bits, keys of chunk j visible to the row, 0).  The
-// visible keys are 64 except in the row's own chunk, where they end at the
-// row's position.
-__device__ __forceinline__ int4 pair_record(int32_t row, float w, int64_t pos, int32_t j) {
+// The 8-byte record of pair (query row, chunk j) for the tensor-core
+// attention: the row, and the fusion weight w with its 6 lowest mantissa bits
+// replaced by the number of keys of chunk j visible to the row, minus one.
+// The visible keys are 64 except in the row's own chunk, where they end at
+// the row's position.  The change to w, below 2^-17 of w, is far below the
+// bf16 rounding of the probabilities that w scales.
+__device__ __forceinline__ int2 pair_record(int32_t row, float w, int64_t pos, int32_t j) {
   const int nk = pos / kChunk == j ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
-  return make_int4(row, __float_as_int(w), nk, 0);
+  return make_int2(row, (int)((__float_as_uint(w) & ~63u) | (uint32_t)(nk - 1)));
 }
 
 // One CTA per (sequence b, KV head g, block of kBucketRows query positions):
@@ -198,6 +200,10 @@ struct SmallDiv {
   __device__ __forceinline__ uint32_t div(uint32_t x) const { return d > 1 ? __umulhi(x, m) : x; }
 };
 
+// Pairs a thread takes per round of the bucketing loops: their loads are all
+// issued before the first is used.
+constexpr int kBucketUnroll = 8;
+
 __device__ __forceinline__ void block_hist(const Params& P, const int32_t* idx, int32_t* hist,
                                            int nvis, int64_t i0, int64_t i1, int b, int g,
                                            bool check) {
@@ -206,15 +212,23 @@ __device__ __forceinline__ void block_hist(const Params& P, const int32_t* idx, 
   const int n = (int)(i1 - i0) * per_i;
   const int32_t* base = idx + (((int64_t)b * P.L + i0) * P.Hq + g * P.group) * P.k;
   const int64_t row_stride = (int64_t)P.Hq * P.k;   // idx entries from one position to the next
-  for (int f = threadIdx.x; f < n; f += blockDim.x) {
-    const int ii = (int)dv.div((uint32_t)f);
-    const int32_t j = base[ii * row_stride + (f - ii * per_i)];
-    if (j < 0) continue;
-    if (j >= nvis) {
-      if (check) set_device_error(kErrChunk);
-      continue;
+  for (int f0 = threadIdx.x; f0 < n; f0 += blockDim.x * kBucketUnroll) {
+    int32_t j[kBucketUnroll];
+#pragma unroll
+    for (int u = 0; u < kBucketUnroll; ++u) {
+      const int f = f0 + u * blockDim.x;
+      const int ii = (int)dv.div((uint32_t)f);
+      j[u] = f < n ? __ldg(base + ii * row_stride + (f - ii * per_i)) : -1;
     }
-    atomicAdd(&hist[j], 1);
+#pragma unroll
+    for (int u = 0; u < kBucketUnroll; ++u) {
+      if (j[u] < 0) continue;
+      if (j[u] >= nvis) {
+        if (check) set_device_error(kErrChunk);
+        continue;
+      }
+      atomicAdd(&hist[j[u]], 1);
+    }
   }
 }
 
@@ -235,9 +249,9 @@ __global__ void __launch_bounds__(256) bucket_count_kernel(Params P, const int32
 
 // Same blocks: one global atomic per nonzero bin reserves the block's range of
 // each bucket, shared-memory atomics place the pairs inside it.
-__global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int32_t* idx,
+__global__ void __launch_bounds__(256, 3) bucket_scatter_kernel(Params P, const int32_t* idx,
                                                              const float* wts, int32_t* cursor,
-                                                             int32_t* pairs, int4* pinfo,
+                                                             int32_t* pairs, int2* pinfo,
                                                              Windows W) {
   extern __shared__ int32_t hist[];
   const int b = blockIdx.z, g = blockIdx.y;
@@ -259,19 +273,31 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(Params P, const int
   const SmallDiv dv(per_i), dk(P.k);
   const int n = (int)(i1 - i0) * per_i;
   const bool rows_out = pinfo != nullptr;   // tensor-core path: a record per pair
-  for (int f = threadIdx.x; f < n; f += blockDim.x) {
-    const int ii = (int)dv.div((uint32_t)f);
-    const int q = f - ii * per_i;                                        // head-in-group * k + slot
-    const int64_t i = i0 + ii;
-    const int64_t row0 = ((int64_t)b * P.L + i) * P.Hq + g * P.group;   // first row of the group
-    const int64_t p = row0 * P.k + q;
-    const int32_t j = idx[p];
-    if (j < 0 || j >= nvis) continue;
-    const int32_t at = base[j] + atomicAdd(&hist[j], 1);
-    if (rows_out)
-      pinfo[at] = pair_record((int32_t)(row0 + dk.div((uint32_t)q)), wts[p], P.pos0 + i, j);
-    else
-      pairs[at] = (int32_t)p;
+  for (int f0 = threadIdx.x; f0 < n; f0 += blockDim.x * kBucketUnroll) {
+    int32_t j[kBucketUnroll];
+    float wv[kBucketUnroll];
+#pragma unroll
+    for (int u = 0; u < kBucketUnroll; ++u) {
+      const int f = f0 + u * blockDim.x;
+      const int ii = (int)dv.div((uint32_t)f);
+      const int64_t p = (((int64_t)b * P.L + i0 + ii) * P.Hq + g * P.group) * P.k + (f - ii * per_i);
+      j[u] = f < n ? __ldg(idx + p) : -1;
+      wv[u] = (f < n && rows_out) ? __ldg(wts + p) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBucketUnroll; ++u) {
+      if (j[u] < 0 || j[u] >= nvis) continue;
+      const int f = f0 + u * blockDim.x;
+      const int ii = (int)dv.div((uint32_t)f);
+      const int q = f - ii * per_i;                                        // head-in-group * k + slot
+      const int64_t i = i0 + ii;
+      const int64_t row0 = ((int64_t)b * P.L + i) * P.Hq + g * P.group;   // first row of the group
+      const int32_t at = base[j[u]] + atomicAdd(&hist[j[u]], 1);
+      if (rows_out)
+        pinfo[at] = pair_record((int32_t)(row0 + dk.div((uint32_t)q)), wv[u], P.pos0 + i, j[u]);
+      else
+        pairs[at] = (int32_t)(row0 * P.k + q);
+    }
   }
 }
 
@@ -290,7 +316,7 @@ __global__ void count_kernel(Params P, const int32_t* idx, int32_t* counts, int6
 }
 
 __global__ void scatter_kernel(Params P, const int32_t* idx, const float* wts, int32_t* cursor,
-                               int32_t* pairs, int4* pinfo, int64_t n_pairs, Windows W) {
+                               int32_t* pairs, int2* pinfo, int64_t n_pairs, Windows W) {
   const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= n_pairs) return;
   const int32_t j = idx[p];
@@ -593,7 +619,7 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
   w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
   if (P.dtype == HILS_BF16)
-    w.pinfo = (int4*)take(sizeof(int4) * n_pairs);
+    w.pinfo = (int2*)take(sizeof(int2) * n_pairs + 16);   // + 16: tiles are copied in 16-byte units
   else
     w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
   if (P.dtype == HILS_BF16) {

@@ -33,8 +33,7 @@ constexpr int kThrS = 128;
 constexpr int kTerms = 3;
 constexpr int kEpiWarps = 8;          // epilogue warps; warp 8 issues the MMAs and loads
 constexpr int kSBufs = 3;             // S buffers of 128 TMEM columns
-constexpr uint32_t kTmemColsS = 512;  // the S buffers, then the class maxima
-constexpr uint32_t kCmaxCol = kSBufs * 128;   // selection pass 0: 128 class maxima per row
+constexpr uint32_t kTmemColsS = 512;  // the S buffers (allocations are powers of two)
 constexpr int kLmBufs = 2;            // landmark blocks in flight: prefetch distance 1
 constexpr int kHalfCap = 32;          // selection pass 1: collected candidates per row and column half
 
@@ -204,6 +203,316 @@ __global__ void __launch_bounds__(kThrS) calib_kernel(Params P, uint8_t* qimg, i
   }
 }
 
+// ---- a1 on the tensor cores ------------------------------------------------
+// calib_tc_kernel writes the same q~ images as calib_kernel (rank r <= 32),
+// with both small products on the tensor cores.  Per 128-row tile:
+//   1. TMA brings the q tile in (K-major, 128-byte swizzle), a tile ahead.
+//   2. T = q A.  A is split once per CTA into three bf16 terms (A = A0 + A1
+//      + A2 up to 2^-27 |A|); q is bf16, so every product q A_i is exact and
+//      T = sum_i q A_i accumulates in float32 in TMEM.
+//   3. The epilogue splits T into three bf16 terms T_i and stores them back
+//      into TMEM, where the next product reads them as its A operand.
+//   4. U = T B = sum over i + j <= 2 of T_i B_j (B split like A; the products
+//      left out are below 2^-23 of the largest), float32 in TMEM.
+//   5. The epilogue adds q (from the staged tile) to U, splits q~ = q + U
+//      into its three bf16 terms and writes them into the tile's three images
+//      in shared memory, which one bulk copy stores.
+// Warps 0-3: epilogue (TMEM lane quarter w, one query row per thread); warp
+// 4: TMA and MMA issue (one thread).
+constexpr int kCalibRank = 32;   // rank the tensor-core calibration is built for (r <= 32)
+constexpr int kCalibThreads = 160;
+
+template <int D>
+struct CalibLayout {
+  static constexpr uint32_t kQB = kRowsS * D * 2;        // one q tile = one term image
+  static constexpr uint32_t kOpB = kCalibRank * D * 2;   // one term of A (or B) as an operand
+  static constexpr uint32_t kQ = 0;                      // two q buffers
+  static constexpr uint32_t kA = 2 * kQB;                // A terms: [32 rank rows][D], K-major
+  static constexpr uint32_t kB = kA + 3 * kOpB;          // B terms: [32 rank rows][D], MN-major
+  static constexpr uint32_t kOut = kB + 3 * kOpB;        // the tile's three q~ term images
+  static constexpr uint32_t kSmem = kOut + 3 * kQB + 1024;   // + base alignment
+  static_assert(kSmem + 1024 <= 232448, "shared memory above 227 KB");
+  // TMEM columns: T (32), its three bf16 terms (16 each), U (D)
+  static constexpr uint32_t kT = 0, kTt = 32, kU = 128, kCols = 256;
+};
+
+// (x0, x1) -> three packed bf16 pairs, each the rounding of what is left.
+__device__ __forceinline__ void split3(float x0, float x1, uint32_t& h, uint32_t& m, uint32_t& l) {
+  h = tc::pack_bf16x2(x0, x1);
+  x0 -= __uint_as_float(h << 16);
+  x1 -= __uint_as_float(h & 0xFFFF0000u);
+  m = tc::pack_bf16x2(x0, x1);
+  x0 -= __uint_as_float(m << 16);
+  x1 -= __uint_as_float(m & 0xFFFF0000u);
+  l = tc::pack_bf16x2(x0, x1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCalibThreads, 1) calib_tc_kernel(
+    Params P, const __grid_constant__ CUtensorMap tm_q, uint8_t* qimg, int T, int n_tiles) {
+  using Lay = CalibLayout<D>;
+  constexpr int KB = D / 64;   // 128-byte blocks in a row of D bf16
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t q_full[2], t_full, tt_ready, u_full, out_ready, out_free, drain;
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // A and B as three bf16 terms each, zero beyond the rank
+  for (int x = tid; x < kCalibRank * (D / 8); x += kCalibThreads) {
+    const int a = x / (D / 8), c = x % (D / 8);   // rank row, 16-byte chunk along D
+    float va[8], vb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = c * 8 + u;
+      va[u] = a < P.r ? P.A[e * P.r + a] : 0.f;
+      vb[u] = a < P.r ? P.Bm[a * D + e] : 0.f;
+    }
+    uint32_t ha[4], ma[4], la[4], hb[4], mb[4], lb[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      split3(va[2 * q], va[2 * q + 1], ha[q], ma[q], la[q]);
+      split3(vb[2 * q], vb[2 * q + 1], hb[q], mb[q], lb[q]);
+    }
+    const uint32_t off = (uint32_t)(c >> 3) * (kCalibRank * 128) + tc::swz(a, c & 7);
+    *reinterpret_cast<uint4*>(smem + Lay::kA + 0 * Lay::kOpB + off) = make_uint4(ha[0], ha[1], ha[2], ha[3]);
+    *reinterpret_cast<uint4*>(smem + Lay::kA + 1 * Lay::kOpB + off) = make_uint4(ma[0], ma[1], ma[2], ma[3]);
+    *reinterpret_cast<uint4*>(smem + Lay::kA + 2 * Lay::kOpB + off) = make_uint4(la[0], la[1], la[2], la[3]);
+    *reinterpret_cast<uint4*>(smem + Lay::kB + 0 * Lay::kOpB + off) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+    *reinterpret_cast<uint4*>(smem + Lay::kB + 1 * Lay::kOpB + off) = make_uint4(mb[0], mb[1], mb[2], mb[3]);
+    *reinterpret_cast<uint4*>(smem + Lay::kB + 2 * Lay::kOpB + off) = make_uint4(lb[0], lb[1], lb[2], lb[3]);
+  }
+  tc::fence_proxy_async();   // the terms are read by the tensor cores
+  if (tid == 0) {
+    tc::mbar_init(&q_full[0], 1);
+    tc::mbar_init(&q_full[1], 1);
+    tc::mbar_init(&t_full, 1);
+    tc::mbar_init(&tt_ready, 4);
+    tc::mbar_init(&u_full, 1);
+    tc::mbar_init(&out_ready, 4);
+    tc::mbar_init(&out_free, 1);
+    tc::mbar_init(&drain, 1);
+    tc::fence_mbar_init();
+    abort_sh = 0;
+  }
+  if (warp == 4) {
+    tc::tmem_alloc(&tmem_sh, Lay::kCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+  volatile int* abort_v = &abort_sh;
+  // this CTA's tiles: blockIdx.x, + gridDim.x, ...
+  const int my_tiles = ((int)blockIdx.x < n_tiles)
+                           ? (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                           : 0;
+  auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
+
+  if (warp == 4) {
+    if (lane == 0 && my_tiles > 0) {
+      constexpr uint32_t kId1 = tc::idesc_bf16(kRowsS, kCalibRank, 0);
+      constexpr uint32_t kId2 = tc::idesc_bf16(kRowsS, D, 1);
+      auto load_q = [&](int n) {
+        const int gt = tile_of(n), t = gt % T, bh = gt / T;
+        const int h = bh % P.Hq, b = bh / P.Hq;
+        uint64_t* bar = &q_full[n & 1];
+        tc::mbar_arrive_expect_tx(bar, Lay::kQB);
+#pragma unroll
+        for (int c = 0; c < KB; ++c)
+          tc::tma_load_4d(sbase + Lay::kQ + (n & 1) * Lay::kQB + c * (kRowsS * 128), &tm_q,
+                          c * 64, h, t * kRowsS, b, bar);
+      };
+      auto mma1 = [&](int n) {   // T = sum_i q A_i
+        const uint32_t qb = sbase + Lay::kQ + (n & 1) * Lay::kQB;
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = tc::smem_desc(qb + (kk >> 2) * (kRowsS * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::smem_desc(
+                sbase + Lay::kA + term * Lay::kOpB + (kk >> 2) * (kCalibRank * 128) + (kk & 3) * 32,
+                16, 1024);
+            tc::mma_bf16(tmem + Lay::kT, a, bd, kId1, (term | kk) != 0);
+          }
+        }
+        tc::mma_commit(&t_full);
+      };
+      auto mma2 = [&]() {   // U = sum over i + j <= 2 of T_i B_j
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+#pragma unroll
+          for (int j = 0; j + i < 3; ++j) {
+#pragma unroll
+            for (int kk = 0; kk < kCalibRank / 16; ++kk) {
+              const uint64_t bd = tc::smem_desc(sbase + Lay::kB + j * Lay::kOpB + kk * 2048,
+                                                kCalibRank * 128, 1024);
+              tc::mma_bf16_tmem_a(tmem + Lay::kU, tmem + Lay::kTt + i * 16 + kk * 8, bd, kId2, acc);
+              acc = 1;
+            }
+          }
+        }
+        tc::mma_commit(&u_full);
+      };
+      int loads = 0, landed = 0;   // q loads issued / waited for
+      bool ok = true, any_mma = false;
+      load_q(0);
+      loads = 1;
+      if (my_tiles > 1) {
+        load_q(1);
+        loads = 2;
+      }
+      if (tc::mbar_wait_sleep(&q_full[0], 0, wait_limit())) {
+        landed = 1;
+        tc::tc_fence_after();
+        mma1(0);
+        any_mma = true;
+      } else {
+        ok = false;
+      }
+      for (int n = 0; ok && n < my_tiles; ++n) {
+        // T's terms are in TMEM (and T itself was read): U of tile n
+        if (!tc::mbar_wait_sleep(&tt_ready, n & 1, wait_limit()) || *abort_v) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        mma2();
+        if (n + 1 < my_tiles) {
+          if (!tc::mbar_wait_sleep(&q_full[(n + 1) & 1], ((n + 1) >> 1) & 1, wait_limit())) {
+            ok = false;
+            break;
+          }
+          landed = n + 2;
+          tc::tc_fence_after();
+          mma1(n + 1);
+        }
+        // the epilogue has written tile n's images (and read its q tile)
+        if (!tc::mbar_wait_sleep(&out_ready, n & 1, wait_limit())) {
+          ok = false;
+          break;
+        }
+        tc::bulk_s2g(qimg + (int64_t)tile_of(n) * (3 * Lay::kQB), sbase + Lay::kOut, 3 * Lay::kQB);
+        tc::bulk_commit();
+        if (n + 2 < my_tiles) {
+          load_q(n + 2);
+          loads = n + 3;
+        }
+        tc::bulk_wait_read();
+        tc::mbar_arrive(&out_free);
+      }
+      if (!ok) {
+        *abort_v = 1;
+        // let what was issued land before the CTA exits (bounded waits)
+        for (int x = landed; x < loads; ++x)
+          tc::mbar_wait_sleep(&q_full[x & 1], (x >> 1) & 1, kDrainLimitNs);
+        if (any_mma) {
+          tc::mma_commit(&drain);
+          tc::mbar_wait_sleep(&drain, 0, kDrainLimitNs);
+        }
+      }
+      tc::bulk_wait_all();
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: warp w owns TMEM lanes 32 w .. 32 w + 31 (tile rows) ----
+    const int row = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
+    for (int n = 0; n < my_tiles; ++n) {
+      // T -> three bf16 terms, back into TMEM as the next product's A operand
+      if (!tc::warp_wait(&t_full, n & 1, wait_limit()) || *abort_v) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      {
+        uint32_t tv[32];
+        tc::tmem_ld32(tmem + lane_off + Lay::kT, tv);
+        tc::tmem_ld_wait();
+        uint32_t th[16], tm[16], tl[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          split3(__uint_as_float(tv[2 * x]), __uint_as_float(tv[2 * x + 1]), th[x], tm[x], tl[x]);
+        tc::tmem_st16(tmem + lane_off + Lay::kTt, th);
+        tc::tmem_st16(tmem + lane_off + Lay::kTt + 16, tm);
+        tc::tmem_st16(tmem + lane_off + Lay::kTt + 32, tl);
+        tc::tmem_st_wait();
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tt_ready);
+      // q~ = q + U, split into three terms, into the output images
+      if (!tc::warp_wait(&u_full, n & 1, wait_limit()) ||
+          (n > 0 && !tc::warp_wait(&out_free, (n - 1) & 1, wait_limit()))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint8_t* qt = smem + Lay::kQ + (n & 1) * Lay::kQB;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t uv[32];
+        tc::tmem_ld32(tmem + lane_off + Lay::kU + c0, uv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = c0 / 8 + cc;   // 16-byte chunk of the row
+          const uint32_t off = (uint32_t)(c >> 3) * (kRowsS * 128) + tc::swz(row, c & 7);
+          const uint4 qv = *reinterpret_cast<const uint4*>(qt + off);
+          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+          uint32_t h[4], m[4], l[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            split3(__uint_as_float(qw[q] << 16) + __uint_as_float(uv[cc * 8 + 2 * q]),
+                   __uint_as_float(qw[q] & 0xFFFF0000u) + __uint_as_float(uv[cc * 8 + 2 * q + 1]),
+                   h[q], m[q], l[q]);
+          *reinterpret_cast<uint4*>(smem + Lay::kOut + 0 * Lay::kQB + off) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(smem + Lay::kOut + 1 * Lay::kQB + off) = make_uint4(m[0], m[1], m[2], m[3]);
+          *reinterpret_cast<uint4*>(smem + Lay::kOut + 2 * Lay::kQB + off) = make_uint4(l[0], l[1], l[2], l[3]);
+        }
+      }
+      tc::tc_fence_before();
+      tc::fence_proxy_async();   // the images are read by the bulk copy
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&out_ready);
+    }
+    if (!ok) *abort_v = 1;
+  }
+  if (tid == 0 && *abort_v) set_device_error(kErrTimeout);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 4) tc::tmem_dealloc(tmem, Lay::kCols);
+}
+
+template <int D>
+cudaError_t run_calib_tc(const Params& P, uint8_t* qimg, int T, int64_t n_tiles, int n_sm,
+                         cudaStream_t s) {
+  using Lay = CalibLayout<D>;
+  CUtensorMap tm;
+  {
+    // q [B][L][Hq][D] as (D, head, position, sequence); a box is 64 elements of
+    // 128 consecutive positions of one head
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hq, (uint64_t)P.L, (uint64_t)P.B};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)P.Hq * D * 2,
+                                 (uint64_t)P.L * P.Hq * D * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)kRowsS, 1};
+    cudaError_t e = encode_tmap_bf16(&tm, 4, P.q, dims, strides, box);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = set_smem(calib_tc_kernel<D>, Lay::kSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = min(n_tiles, (int64_t)n_sm);
+  HILS_PROFILE("prefill.calib", s);
+  calib_tc_kernel<D><<<(unsigned)grid, kCalibThreads, Lay::kSmem, s>>>(P, tm, qimg, T, (int)n_tiles);
+  return cudaGetLastError();
+}
+
 // ---- a2-a4: landmark scores, selection and weights, fused -------------------
 // Keys: a larger key ranks higher in (score desc, index asc).  The high word
 // is the score's bits mapped to an unsigned order (-0 taken as +0), the low
@@ -350,8 +659,8 @@ __device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int n
 // Selection in two passes over the tile's blocks, so that no per-score work
 // depends on earlier scores:
 //   pass 0  per row and column half, the maximum score of each column class
-//           of candidates j < own, kept in TMEM between blocks: over both
-//           halves, the maxima of the 128 classes j mod 128.  The K-th
+//           of candidates j < own, kept in registers between blocks: over
+//           both halves, the maxima of the 128 classes j mod 128.  The K-th
 //           largest of these maxima (K = k-1) is a lower bound tau on the
 //           row's K-th best score: the K classes it comes from hold K
 //           distinct candidates scoring at least tau.  The two halves swap
@@ -365,8 +674,9 @@ __device__ __forceinline__ void step_next(Step& s, const Params& P, int T, int n
 // second's: the best K are the selection, best first.  A candidate left out
 // scores below tau, or below a half's bar, so at least K collected ones rank
 // above it.  The softmax of the own and selected scores gives the weights.
-// Pass 0 compares raw accumulator values; tau is scaled once, and rounding is
-// monotone, so the bound holds for the scaled scores of pass 1.
+// Both passes compare raw accumulator values; pass 1's bound is lowered by a
+// few ulps, so every score whose scaled value could round up to the bound's
+// is collected, and the keys (scaled scores) then decide exactly.
 template <int D>
 __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
     Params P, const __grid_constant__ CUtensorMap tm_lm, const uint8_t* qimg, int T, int n_tiles,
@@ -531,9 +841,10 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
     uint64_t* const buf = reinterpret_cast<uint64_t*>(smem + Lay::kBuf);
     uint64_t* Bf = buf + hf * kHalfCap * kThrS + row;         // this half, stride kThrS
     uint64_t* Bo = buf + (1 - hf) * kHalfCap * kThrS + row;   // the partner's half
-    float thr_f = -INFINITY;   // pass 1: candidates scoring below this are left out
+    float thr_f = -INFINITY;   // pass 1: raw scores below this are left out
     uint64_t thr_key = 0;      // pass 1: and keys must exceed this (set once the buffer was cut)
     int cnt = 0;               // pass 1: keys in this half's buffer
+    const float sqrt_d = sqrtf((float)P.d);
 
     auto append = [&](uint64_t key) {
       Bf[cnt * kThrS] = key;
@@ -541,7 +852,9 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
         keep_best(Bf, cnt, K);
         cnt = K;
         thr_key = Bf[0];
-        thr_f = key_score(thr_key);
+        // the bar in raw units, lowered by a few ulps: the keys decide exactly
+        const float r = key_score(thr_key) * sqrt_d;
+        thr_f = fmaxf(thr_f, r - fabsf(r) * 0x1p-20f);
       }
     };
 
@@ -623,6 +936,9 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
 
     // S buffer sb, this half's 64 columns: tile st's rows against chunks
     // st.blk * 128 + co ..
+    // Pass 0 keeps this half's 64 class maxima in registers from block to
+    // block (raw accumulator values).
+    float cmx[64];
     auto drain = [&](int sb, const Step& st) {
       const int i = st.t * kRowsS + row;
       const int i_last = min((st.t + 1) * kRowsS, (int)P.L) - 1;
@@ -631,57 +947,35 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
       const int own_max = (int)((P.pos0 + i_last) / kChunk);
       const int jb = st.blk * kBlk + co;
       const uint32_t ta = tmem + sb * kBlk + co + lane_off;
-      const uint32_t tc_max = tmem + kCmaxCol + co + lane_off;
       if (st.pass == 0) {
         if (K == 0) return;
-        // class maxima: TMEM -> registers for this block only, read together
-        // with the 64 scores (one wait); the previous block's store of them is
-        // waited for here, not right after it was issued
-        uint32_t cmu[2][32];
-        tc::tmem_st_wait();
+        if (st.blk == 0) {
+#pragma unroll
+          for (int x = 0; x < 64; ++x) cmx[x] = -INFINITY;
+        }
         if (jb < own_max) {
           uint32_t s0[32], s1[32];
-          if (st.blk != 0) {
-            tc::tmem_ld32(tc_max, cmu[0]);
-            tc::tmem_ld32(tc_max + 32, cmu[1]);
-          }
           tc::tmem_ld32(ta, s0);
           tc::tmem_ld32(ta + 32, s1);
           tc::tmem_ld_wait();
-          if (st.blk == 0) {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
-          }
           if (jb + 64 <= own_min) {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              cmu[0][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[0][x]), __uint_as_float(s0[x])));
-              cmu[1][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[1][x]), __uint_as_float(s1[x])));
+              cmx[x] = fmaxf(cmx[x], __uint_as_float(s0[x]));
+              cmx[32 + x] = fmaxf(cmx[32 + x], __uint_as_float(s1[x]));
             }
           } else {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              cmu[0][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[0][x]),
-                                                jb + x < own ? __uint_as_float(s0[x]) : -INFINITY));
-              cmu[1][x] = __float_as_uint(fmaxf(__uint_as_float(cmu[1][x]),
-                                                jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY));
+              cmx[x] = fmaxf(cmx[x], jb + x < own ? __uint_as_float(s0[x]) : -INFINITY);
+              cmx[32 + x] = fmaxf(cmx[32 + x], jb + 32 + x < own ? __uint_as_float(s1[x]) : -INFINITY);
             }
           }
-        } else if (st.blk != 0) {
-          tc::tmem_ld32(tc_max, cmu[0]);
-          tc::tmem_ld32(tc_max + 32, cmu[1]);
-          tc::tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) cmu[0][x] = cmu[1][x] = __float_as_uint(-INFINITY);
         }
         if (st.blk == st.nblk - 1) {
           float cm[64];
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            cm[x] = __uint_as_float(cmu[0][x]);
-            cm[32 + x] = __uint_as_float(cmu[1][x]);
-          }
+          for (int x = 0; x < 64; ++x) cm[x] = cmx[x];
           sort_desc<64>(cm);
           // the two halves' best 32 maxima meet in the (empty) collection
           // buffers: the K-th largest of all 128 class maxima is the bound
@@ -699,10 +993,10 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
           float tau = top[0];
 #pragma unroll
           for (int p = 1; p < 32; ++p) tau = (p == K - 1) ? top[p] : tau;
-          thr_f = tau * P.inv_sqrt_d;
-        } else {
-          tc::tmem_st32(tc_max, cmu[0]);
-          tc::tmem_st32(tc_max + 32, cmu[1]);
+          // pass 1 compares raw scores with this bound, lowered by a few
+          // ulps so that every score whose scaled value could round to the
+          // bound's scaled value is collected too
+          thr_f = tau - fabsf(tau) * 0x1p-20f;
         }
         return;
       }
@@ -714,12 +1008,12 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
         float v0[32], v1[32];
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          v0[x] = __uint_as_float(sv[0][x]) * P.inv_sqrt_d;
-          v1[x] = __uint_as_float(sv[1][x]) * P.inv_sqrt_d;
+          v0[x] = __uint_as_float(sv[0][x]);
+          v1[x] = __uint_as_float(sv[1][x]);
         }
         const int od = own - jb;
-        if (od >= 0 && od < 32) s_own_sh[row] = pick32(v0, od);
-        if (od >= 32 && od < 64) s_own_sh[row] = pick32(v1, od - 32);
+        if (od >= 0 && od < 32) s_own_sh[row] = pick32(v0, od) * P.inv_sqrt_d;
+        if (od >= 32 && od < 64) s_own_sh[row] = pick32(v1, od - 32) * P.inv_sqrt_d;
         if (K > 0 && jb < own_max) {
           uint32_t m0 = 0, m1 = 0;
           if (jb + 64 <= own_min) {
@@ -736,18 +1030,19 @@ __global__ void __launch_bounds__(2 * kThrS + 32, 1) score_select_kernel(
             }
           }
           // per round one candidate of each 32 columns per lane: lanes do not
-          // serialise each other, and the two extractions are independent
+          // serialise each other, and the two extractions are independent;
+          // keys hold the scaled scores
           while (__any_sync(0xffffffffu, (m0 | m1) != 0)) {
             if (m0) {
               const int x = __ffs(m0) - 1;
               m0 &= m0 - 1;
-              const uint64_t key = make_key(pick32(v0, x), jb + x);
+              const uint64_t key = make_key(pick32(v0, x) * P.inv_sqrt_d, jb + x);
               if (key > thr_key) append(key);
             }
             if (m1) {
               const int x = __ffs(m1) - 1;
               m1 &= m1 - 1;
-              const uint64_t key = make_key(pick32(v1, x), jb + 32 + x);
+              const uint64_t key = make_key(pick32(v1, x) * P.inv_sqrt_d, jb + 32 + x);
               if (key > thr_key) append(key);
             }
           }
@@ -817,13 +1112,9 @@ cudaError_t run_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, fl
   const int64_t n_tiles = (int64_t)P.B * P.Hq * T;
   uint8_t* qimg = reinterpret_cast<uint8_t*>(ws.qimg);
 
-  const int rp = P.r <= 8 ? 8 : P.r <= 16 ? 16 : P.r <= 32 ? 32 : 64;
-  switch (rp) {
-    case 8: e = run_calib<D, 8>(P, qimg, T, n_tiles, n_sm, s); break;
-    case 16: e = run_calib<D, 16>(P, qimg, T, n_tiles, n_sm, s); break;
-    case 32: e = run_calib<D, 32>(P, qimg, T, n_tiles, n_sm, s); break;
-    default: e = run_calib<D, 64>(P, qimg, T, n_tiles, n_sm, s); break;
-  }
+  // ranks up to 32 on the tensor cores, larger ones (up to 64) on the CUDA cores
+  e = P.r <= kCalibRank ? run_calib_tc<D>(P, qimg, T, n_tiles, n_sm, s)
+                        : run_calib<D, 64>(P, qimg, T, n_tiles, n_sm, s);
   if (e != cudaSuccess) return e;
 
   CUtensorMap tm;

@@ -51,13 +51,13 @@ def peaks():
 
 # ----------------------------------------------------------------- work counts
 # DRAM traffic of the attention kernel from one ncu capture on prefill_16k_gqa
-# (dram__bytes_read.sum + dram__bytes_write.sum = 697.8 MB + 115.3 MB for
+# (dram__bytes_read.sum + dram__bytes_write.sum = 562.5 MB + 114.6 MB for
 # 15.76M (row, slot) pairs), per pair; it grows with the pairs.  Valid only
 # for the kernel source it was taken on (sha256 below); otherwise the bench
 # reports null.
 ATTN_TRAFFIC = {"file": "chunk_sparse_long_b200/csrc/attn_tc.cu",
-                "sha256": "50c909ba895377dcaa23c4273998ef78fa7a7f1761ac1aeab87cc68af1f7e790",
-                "bytes_per_pair": (697821184 + 115285760) / 15761408}
+                "sha256": "dabe3af0a52ce023f9d3543722daa5c44a3f1d2ea727ee1a539c700fff426add",
+                "bytes_per_pair": (562519040 + 114627328) / 15761408}
 
 
 def attn_traffic(pairs: float):

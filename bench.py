@@ -215,38 +215,63 @@ def time_prefill(hils, torch, wl, steps, warmup, barrier, maxreduce):
 
 
 def time_prefill_e2e(hils, torch, wl, steps, warmup):
-    """Same step through host buffers: pinned host inputs copied in, the result
-    copied out, every step, inside the timed region."""
+    """Same step through host buffers: every step copies all of its inputs in
+    from pinned host memory and its result out, inside the timed region.  The
+    steps are pipelined over three streams, as a serving loop would run them:
+    while step n computes, step n+1's inputs are copied in and step n-1's
+    result is copied out (device inputs and outputs double-buffered; the
+    host-to-device and device-to-host copies use the link's two directions at
+    once).  The timed region runs from the first step's first copy in to the
+    last step's copy out, so the pipeline's fill and drain are included."""
     w = wl["workload"]
     cfg = cfg_of(hils, w)
-    stream = torch.cuda.current_stream()
-    host = {k: wl[k].cpu().pin_memory() for k in ("q", "pages", "landmarks", "block_table", "A", "B")}
-    dev = {k: torch.empty_like(wl[k]) for k in host}
+    keys = ("q", "pages", "landmarks", "block_table", "A", "B")
+    host = {k: wl[k].cpu().pin_memory() for k in keys}
+    dev = [{k: torch.empty_like(wl[k]) for k in keys} for _ in range(2)]
     L = w.seq_len
-    out = torch.empty_like(wl["q"])
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    out = [torch.empty_like(wl["q"]) for _ in range(2)]
+    out_host = [torch.empty(out[0].shape, dtype=out[0].dtype).pin_memory() for _ in range(2)]
     nbytes = hils.workspace_size(cfg, hils.OP_PREFILL, L, wl["max_chunks"])
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    cache = hils.Cache(dev["pages"], wl["num_pages"], dev["block_table"], wl["max_chunks"],
-                       dev["landmarks"])
+    caches = [hils.Cache(d["pages"], wl["num_pages"], d["block_table"], wl["max_chunks"],
+                         d["landmarks"]) for d in dev]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out.numel() * out.element_size()
+    d2h = out[0].numel() * out[0].element_size()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
-        hils.prefill(cfg, dev["q"], L, 0, dev["A"], dev["B"], cache, out, None, None, ws, nbytes,
-                     stream)
-        out_host.copy_(out, non_blocking=True)
+    def run(n_steps):
+        ev_in, ev_run, ev_out = [], [], []
+        for n in range(n_steps):
+            b = n % 2
+            ev_in.append(torch.cuda.Event())
+            ev_run.append(torch.cuda.Event())
+            ev_out.append(torch.cuda.Event())
+            with torch.cuda.stream(s_in):
+                if n >= 2:
+                    s_in.wait_event(ev_run[n - 2])     # step n-2 has read buffer b's inputs
+                for k in keys:
+                    dev[b][k].copy_(host[k], non_blocking=True)
+                ev_in[n].record(s_in)
+            s_run.wait_event(ev_in[n])
+            if n >= 2:
+                s_run.wait_event(ev_out[n - 2])        # buffer b's previous result is out
+            d = dev[b]
+            hils.prefill(cfg, d["q"], L, 0, d["A"], d["B"], caches[b], out[b], None, None, ws,
+                         nbytes, s_run)
+            ev_run[n].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_run[n])
+                out_host[b].copy_(out[b], non_blocking=True)
+                ev_out[n].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    run(warmup)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
+    e0.record(s_in)
+    s_run.wait_event(e0)
+    s_out.wait_event(e0)
+    run(steps)
+    e1.record(s_out)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps, h2d, d2h
 

@@ -140,12 +140,16 @@ __device__ __forceinline__ void unpack16(const uint4& u, float* v) {
 }
 
 // Decode position of sequence b: seq_lens[b] when appending, else the last
-// token; clamped (and flagged) if it falls outside the block table.
-__device__ __forceinline__ int64_t decode_pos(const Params& P, int b, bool append, bool report) {
+// token; clamped (and flagged) if it falls outside [0, limit).  The limit is
+// the block table's capacity, or none (kNoLimit) for the global positions of
+// context-parallel decode.
+constexpr int64_t kNoLimit = INT64_MAX;
+__device__ __forceinline__ int64_t decode_pos(const Params& P, int b, bool append, bool report,
+                                              int64_t limit) {
   int64_t t = append ? (int64_t)P.seq_lens[b] : (int64_t)P.seq_lens[b] - 1;
-  if (t < 0 || t >= (int64_t)P.max_chunks * kChunk) {
+  if (t < 0 || t >= limit) {
     if (report) set_device_error(kErrChunk);
-    t = t < 0 ? 0 : (int64_t)P.max_chunks * kChunk - 1;
+    t = t < 0 ? 0 : limit - 1;
   }
   return t;
 }
@@ -226,8 +230,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const bool append = ws.append != 0;
-  const int64_t t = decode_pos(P, b, append, tid == 0 && split == 0 && g == 0);
-  const int64_t own = t / kChunk;
+  // context-parallel mode: ws.cp_own set (read from the parameter where used)
+  const bool report = tid == 0 && split == 0 && g == 0;
+  const int64_t t =
+      decode_pos(P, b, append, report, ws.cp_own ? kNoLimit : (int64_t)P.max_chunks * kChunk);
+  // the own chunk, local to this cache; in context-parallel mode it may lie
+  // outside (below 0, or past the cache, where max_chunks stands for it), and
+  // the candidates are the local chunks before it in either case
+  int64_t own = t / kChunk - ws.chunk_base;
+  if (own > P.max_chunks) own = P.max_chunks;
   const int cps = ws.chunks_per_split;            // chunks of this range (<= CPS)
   const int64_t c0 = (int64_t)split * cps;
   const bool any_cand = c0 < own;                 // the range holds a chunk before the own one
@@ -264,12 +275,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int x = u * kThreads + tid;
       if (x < nq) rq[u] = __ldg(qsrc + x);
     }
-    if (tid < D / G::EPU)
+    if (own >= 0 && own < P.max_chunks && tid < D / G::EPU)
       rl = __ldg(reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(P.landmarks) +
           (((int64_t)b * P.max_chunks + own) * P.Hkv + g) * D * EB) + tid);
     // the append: the first CTA of each (sequence, KV head) writes its head's k_t and v_t
-    if (append && split == 0 && tid < 2 * (D / G::EPU)) {
+    if (append && own >= 0 && own < P.max_chunks && split == 0 && tid < 2 * (D / G::EPU)) {
       const int64_t page = page_of(P, b, own);
       if (page >= 0) {
         const int kind = tid / (D / G::EPU), x = tid % (D / G::EPU);
@@ -379,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int q = 0; q < G::V; ++q) {
       const int x = q * 32 + lane;
       const int cl = warp * G::SEG + x;
-      v[q] = x < G::SEG ? sel_key(sS[cl * group + hh], c0 + cl) : 0ull;
+      v[q] = x < G::SEG ? sel_key(sS[cl * group + hh], ws.chunk_base + c0 + cl) : 0ull;
     }
     wl[warp * 32 + lane] = warp_top32<G::V>(v);
 #pragma unroll
@@ -425,33 +436,39 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) so += __shfl_xor_sync(kFull, so, o);
       so *= P.inv_sqrt_d;
-      // a4: slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
-      const uint64_t sh = shfl64(key, (lane + 31) & 31);
-      const float my_s = lane == 0 ? so : key_score(sh);
-      const int my_j = lane == 0 ? (int)own : key_chunk(sh);
-      const bool live = lane < P.k && my_j >= 0;
-      float m = live ? my_s : -INFINITY;
+      if (ws.cp_own) {
+        // the merged list and the own score leave for the gather across GPUs
+        if (K > 0 && lane < K) ws.cp_keys[bh * K + lane] = key;
+        if (lane == 0) ws.cp_own[bh] = (own >= 0 && own < P.max_chunks) ? so : -INFINITY;
+      } else {
+        // a4: slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
+        const uint64_t sh = shfl64(key, (lane + 31) & 31);
+        const float my_s = lane == 0 ? so : key_score(sh);
+        const int my_j = lane == 0 ? (int)own : key_chunk(sh);
+        const bool live = lane < P.k && my_j >= 0;
+        float m = live ? my_s : -INFINITY;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-      const float ex = live ? __expf(my_s - m) : 0.f;
-      float z = ex;
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        const float ex = live ? __expf(my_s - m) : 0.f;
+        float z = ex;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-      if (lane < P.k) {
-        const int jv = live ? my_j : -1;
-        const float wv = live ? ex / z : 0.f;
-        const int64_t page = live ? page_of(P, b, jv) : -1;
-        const int64_t o = bh * P.k + lane;
-        ws.idx[o] = jv;
-        ws.w[o] = wv;
-        ws.page[o] = (int32_t)page;
-        if (idx_out) idx_out[o] = jv;
-        if (w_out) w_out[o] = wv;
-        // the attention kernel reads these pages next: start bringing them into L2
-        if (page >= 0 && lane > 0) {
-          const uint8_t* base = reinterpret_cast<const uint8_t*>(P.pages);
-          tc::bulk_prefetch_l2(base + page_offset(P, page, 0, g, 0) * EB, kChunk * D * EB);
-          tc::bulk_prefetch_l2(base + page_offset(P, page, 1, g, 0) * EB, kChunk * D * EB);
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+        if (lane < P.k) {
+          const int jv = live ? my_j : -1;
+          const float wv = live ? ex / z : 0.f;
+          const int64_t page = live ? page_of(P, b, jv) : -1;
+          const int64_t o = bh * P.k + lane;
+          ws.idx[o] = jv;
+          ws.w[o] = wv;
+          ws.page[o] = (int32_t)page;
+          if (idx_out) idx_out[o] = jv;
+          if (w_out) w_out[o] = wv;
+          // the attention kernel reads these pages next: start bringing them into L2
+          if (page >= 0 && lane > 0) {
+            const uint8_t* base = reinterpret_cast<const uint8_t*>(P.pages);
+            tc::bulk_prefetch_l2(base + page_offset(P, page, 0, g, 0) * EB, kChunk * D * EB);
+            tc::bulk_prefetch_l2(base + page_offset(P, page, 1, g, 0) * EB, kChunk * D * EB);
+          }
         }
       }
     }
@@ -581,8 +598,11 @@ __global__ void __launch_bounds__(kSlotThreads * 2)
   // none of this depends on the scan: the query, the position, and the own chunk
   for (int e = tid; e < D; e += blockDim.x)
     sq[e] = load_elem(P.q, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + e);
-  const int64_t t = decode_pos(P, b, append, false);
-  const int64_t own = t / kChunk;
+  const bool cp = ws.cp_partial != nullptr;       // context-parallel mode
+  const int64_t t =
+      decode_pos(P, b, append, false, cp ? kNoLimit : (int64_t)P.max_chunks * kChunk);
+  const int64_t own = t / kChunk;                  // global chunk index
+  const int64_t own_l = own - ws.chunk_base;       // in this cache
   const int tr = (int)(t % kChunk);
   if (rank == 0 && tid == 0) {
     tc::mbar_init(&cpart_bar, n_cta > 1 ? n_cta - 1 : 1);
@@ -592,8 +612,8 @@ __global__ void __launch_bounds__(kSlotThreads * 2)
   cluster.sync();
   float acc = 0.f, l = 0.f;
   bool have = false;
-  if (active && slot == 0) {
-    const int64_t page = page_of(P, b, own);
+  if (active && slot == 0 && own_l >= 0 && own_l < P.max_chunks) {
+    const int64_t page = page_of(P, b, own_l);
     if (page >= 0) {
       stage_tiles<D, EB>(P, page, g, kv, st);
       tc::named_barrier(bar_id, kSlotThreads);
@@ -616,9 +636,13 @@ __global__ void __launch_bounds__(kSlotThreads * 2)
   if (active) {
     wj = __ldcg(ws.w + bh * P.k + slot);
     if (slot > 0) {
-      const int32_t page = __ldcg(ws.page + bh * P.k + slot);
+      const int32_t j = __ldcg(ws.idx + bh * P.k + slot);
+      int64_t page = -1;
+      if (!cp)
+        page = __ldcg(ws.page + bh * P.k + slot);
+      else if (j >= 0 && j - ws.chunk_base >= 0 && j - ws.chunk_base < P.max_chunks)
+        page = page_of(P, b, j - ws.chunk_base);   // a selected chunk held here
       if (page >= 0) {
-        const int32_t j = __ldcg(ws.idx + bh * P.k + slot);
         stage_tiles<D, EB>(P, page, g, kv, st);
         tc::named_barrier(bar_id, kSlotThreads);
         l = chunk_attend<D, EB>(sq, kv, j == own ? tr + 1 : kChunk, P.inv_sqrt_d, sp[sg],
@@ -652,10 +676,13 @@ __global__ void __launch_bounds__(kSlotThreads * 2)
   if (tid < D) {
     float o = 0.f;
     for (int r = 0; r < n_cta; ++r) o += cpart[r][tid];
-    store_elem(out, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + tid, o);
+    if (cp)
+      ws.cp_partial[bh * D + tid] = o;
+    else
+      store_elem(out, EB == 2 ? HILS_BF16 : HILS_F32, bh * D + tid, o);
   }
   // every kernel of the step has read seq_lens: the last head of the sequence advances it
-  if (tid == 0 && append) {
+  if (tid == 0 && append && !cp) {
     __threadfence();
     int32_t* done = ws.tickets + P.B * P.Hkv + b;
     if (atomicAdd(done, 1) == P.Hq - 1) {
@@ -695,48 +722,115 @@ void attend_shape(int k, int* spc, int* n_cta) {
   *spc = (k + *n_cta - 1) / *n_cta;
 }
 
+// The scan (a1-a4): one CTA per (chunk range, KV head, sequence).
+template <int D, int EB>
+cudaError_t launch_scan(const Params& P, const void* k_new, const void* v_new, const DecodeWs& ws,
+                        int32_t* idx_out, float* w_out, cudaStream_t s) {
+  using G = Geo<D, EB>;
+  cudaError_t e;
+  CUtensorMap tm;
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hkv, (uint64_t)P.max_chunks, (uint64_t)P.B};
+  const uint64_t strides[3] = {(uint64_t)D * EB, (uint64_t)P.Hkv * D * EB,
+                               (uint64_t)P.max_chunks * P.Hkv * D * EB};
+  const uint32_t box[4] = {128u / EB, 1, (uint32_t)G::BOXR, 1};
+  if ((e = encode_tmap(&tm, EB == 2 ? HILS_BF16 : HILS_F32, 4, P.landmarks, dims, strides, box)) !=
+      cudaSuccess)
+    return e;
+  const size_t smem = ScanSmem{D, P.r, P.group, G::CPS, ws.n_split, P.k}.bytes();
+  if ((e = set_smem(scan_kernel<D, EB>, smem)) != cudaSuccess) return e;
+  HILS_PROFILE(ws.cp_own ? "decode_cp.candidates" : "decode.scan", s);
+  scan_kernel<D, EB><<<dim3(ws.n_split, P.Hkv, P.B), kScanThreads, smem, s>>>(P, tm, k_new, v_new,
+                                                                             ws, idx_out, w_out);
+  return cudaGetLastError();
+}
+
+// The attention (a5, a6): one cluster of CTAs per (query head, sequence),
+// launched early (programmatic dependent launch) behind the previous kernel.
+template <int D, int EB>
+cudaError_t launch_attend(const Params& P, const DecodeWs& ws, const void* k_new,
+                          const void* v_new, void* out, cudaStream_t s) {
+  int spc, n_cta;
+  attend_shape(P.k, &spc, &n_cta);
+  const size_t kv_bytes = (size_t)spc * SlotTiles<D, EB>::kBytes;
+  cudaError_t e;
+  if ((e = set_smem(attend_kernel<D, EB>, kv_bytes)) != cudaSuccess) return e;
+  if (n_cta > 8) {
+    static bool np_set[2][2] = {};   // one flag per instantiation
+    bool& done = np_set[D == 128][EB == 4];
+    if (!done) {
+      e = cudaFuncSetAttribute(attend_kernel<D, EB>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      done = true;
+    }
+  }
+  HILS_PROFILE(ws.cp_partial ? "decode_cp.attend" : "decode.attend", s);
+  e = launch_pdl(attend_kernel<D, EB>, dim3(n_cta, P.Hq, P.B), dim3(kSlotThreads * spc), kv_bytes,
+                 n_cta, s, P, ws, k_new, v_new, out, spc);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int D, int EB>
 cudaError_t run_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                        int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s) {
-  using G = Geo<D, EB>;
-  cudaError_t e;
-  {
-    CUtensorMap tm;
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)P.Hkv, (uint64_t)P.max_chunks, (uint64_t)P.B};
-    const uint64_t strides[3] = {(uint64_t)D * EB, (uint64_t)P.Hkv * D * EB,
-                                 (uint64_t)P.max_chunks * P.Hkv * D * EB};
-    const uint32_t box[4] = {128u / EB, 1, (uint32_t)G::BOXR, 1};
-    if ((e = encode_tmap(&tm, EB == 2 ? HILS_BF16 : HILS_F32, 4, P.landmarks, dims, strides,
-                         box)) != cudaSuccess)
-      return e;
-    const size_t smem = ScanSmem{D, P.r, P.group, G::CPS, ws.n_split, P.k}.bytes();
-    if ((e = set_smem(scan_kernel<D, EB>, smem)) != cudaSuccess) return e;
-    HILS_PROFILE("decode.scan", s);
-    scan_kernel<D, EB><<<dim3(ws.n_split, P.Hkv, P.B), kScanThreads, smem, s>>>(
-        P, tm, k_new, v_new, ws, idx_out, w_out);
-  }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
-    int spc, n_cta;
-    attend_shape(P.k, &spc, &n_cta);
-    const size_t kv_bytes = (size_t)spc * SlotTiles<D, EB>::kBytes;
-    if ((e = set_smem(attend_kernel<D, EB>, kv_bytes)) != cudaSuccess) return e;
-    if (n_cta > 8) {
-      static bool np_set[2][2] = {};   // one flag per instantiation
-      bool& done = np_set[D == 128][EB == 4];
-      if (!done) {
-        e = cudaFuncSetAttribute(attend_kernel<D, EB>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        done = true;
-      }
-    }
-    HILS_PROFILE("decode.attend", s);
-    e = launch_pdl(attend_kernel<D, EB>, dim3(n_cta, P.Hq, P.B), dim3(kSlotThreads * spc),
-                   kv_bytes, n_cta, s, P, ws, k_new, v_new, out, spc);
-  }
+  cudaError_t e = launch_scan<D, EB>(P, k_new, v_new, ws, idx_out, w_out, s);
   if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_attend<D, EB>(P, ws, k_new, v_new, out, s);
+}
+
+// ---- context-parallel decode ---------------------------------------------
+// One sequence's chunks spread over several GPUs: this GPU holds the chunks
+// chunk_base .. chunk_base + P.max_chunks - 1 (its block table, pages and
+// landmarks are indexed by local chunk); seq_lens holds the global positions.
+// The selection exchanges only each GPU's best k-1 keys and the own chunk's
+// score; the output, only each GPU's weighted sum over the selected chunks it
+// holds.  The scan and the attention are the kernels above in their
+// context-parallel mode; the selection from the gathered lists and the final
+// cast are below.
+
+// Per (query head, sequence), one warp: the global selection from the
+// gathered lists [world][B][Hq][k-1] and own scores [world][B][Hq] -- the
+// same slot order and weights as hils_decode.
+__global__ void __launch_bounds__(32) cp_select_kernel(Params P, int world, const uint64_t* keys,
+                                                       const float* own_scores, bool append,
+                                                       int32_t* idx, float* w) {
+  const int h = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
+  const int K = P.k - 1;
+  const int64_t bh = (int64_t)b * P.Hq + h, nbh = (int64_t)P.B * P.Hq;
+  const int64_t own = decode_pos(P, b, append, lane == 0, kNoLimit) / kChunk;
+  uint64_t c = 0ull;
+  float so = -INFINITY;
+  for (int r = 0; r < world; ++r) {
+    const uint64_t x = (K > 0 && lane < K) ? keys[(r * nbh + bh) * K + lane] : 0ull;
+    c = r == 0 ? x : warp_merge32(c, x);
+    so = fmaxf(so, own_scores[r * nbh + bh]);
+  }
+  if (so == -INFINITY && lane == 0) set_device_error(kErrChunk);   // no GPU holds the own chunk
+  // slot 0 = own chunk, slots 1.. = the merged list; lane a holds slot a
+  const uint64_t sh = shfl64(c, (lane + 31) & 31);
+  const float my_s = lane == 0 ? so : key_score(sh);
+  const int64_t my_j = lane == 0 ? own : key_chunk(sh);
+  const bool live = lane < P.k && my_j >= 0 && my_s != -INFINITY;
+  float m = live ? my_s : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  const float ex = live ? __expf(my_s - m) : 0.f;
+  float z = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+  if (lane < P.k) {
+    idx[bh * P.k + lane] = live ? (int32_t)my_j : -1;
+    w[bh * P.k + lane] = live ? ex / z : 0.f;
+  }
+}
+
+// The summed outputs in the storage dtype; seq_lens advanced when appending.
+__global__ void cp_finish_kernel(Params P, const float* sum, void* out, bool append, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) store_elem(out, P.dtype, i, sum[i]);
+  if (append && blockIdx.x == 0)
+    for (int b = threadIdx.x; b < P.B; b += blockDim.x) P.seq_lens[b] += 1;
 }
 
 int chunks_per_cta(const Params& P) {
@@ -786,6 +880,50 @@ cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new,
                      : run_decode<128, 2>(P, k_new, v_new, out, idx_out, w_out, ws, s);
   return P.d == 64 ? run_decode<64, 4>(P, k_new, v_new, out, idx_out, w_out, ws, s)
                    : run_decode<128, 4>(P, k_new, v_new, out, idx_out, w_out, ws, s);
+}
+
+cudaError_t launch_cp_candidates(const Params& P, const void* k_new, const void* v_new,
+                                 const DecodeWs& ws_in, cudaStream_t s) {
+  DecodeWs ws = ws_in;
+  ws.append = k_new != nullptr;
+  if (P.dtype == HILS_BF16)
+    return P.d == 64 ? launch_scan<64, 2>(P, k_new, v_new, ws, nullptr, nullptr, s)
+                     : launch_scan<128, 2>(P, k_new, v_new, ws, nullptr, nullptr, s);
+  return P.d == 64 ? launch_scan<64, 4>(P, k_new, v_new, ws, nullptr, nullptr, s)
+                   : launch_scan<128, 4>(P, k_new, v_new, ws, nullptr, nullptr, s);
+}
+
+cudaError_t launch_cp_select(const Params& P, int world, const uint64_t* keys,
+                             const float* own_scores, bool append, int32_t* idx, float* w,
+                             cudaStream_t s) {
+  HILS_PROFILE("decode_cp.select", s);
+  cp_select_kernel<<<dim3(P.Hq, P.B), 32, 0, s>>>(P, world, keys, own_scores, append, idx, w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cp_attend(const Params& P, int64_t chunk_base, const void* k_new,
+                             const void* v_new, const int32_t* idx, const float* w, float* partial,
+                             cudaStream_t s) {
+  DecodeWs ws{};   // no workspace: the selection comes from idx and w, the pages from the cache
+  ws.idx = const_cast<int32_t*>(idx);
+  ws.w = const_cast<float*>(w);
+  ws.append = k_new != nullptr;
+  ws.chunk_base = chunk_base;
+  ws.cp_partial = partial;
+  if (P.dtype == HILS_BF16)
+    return P.d == 64 ? launch_attend<64, 2>(P, ws, k_new, v_new, nullptr, s)
+                     : launch_attend<128, 2>(P, ws, k_new, v_new, nullptr, s);
+  return P.d == 64 ? launch_attend<64, 4>(P, ws, k_new, v_new, nullptr, s)
+                   : launch_attend<128, 4>(P, ws, k_new, v_new, nullptr, s);
+}
+
+cudaError_t launch_cp_finish(const Params& P, const float* sum, void* out, bool append,
+                             cudaStream_t s) {
+  const int64_t n = (int64_t)P.B * P.Hq * P.d;
+  HILS_PROFILE("decode_cp.finish", s);
+  const unsigned blocks = (unsigned)((n + 255) / 256 > 0 ? (n + 255) / 256 : 1);
+  cp_finish_kernel<<<blocks, 256, 0, s>>>(P, sum, out, append, n);
+  return cudaGetLastError();
 }
 
 }  // namespace hils

@@ -206,6 +206,111 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
                            false, stream);
 }
 
+namespace {
+// Lays the decode scratch out at `ws` after checking that the configuration
+// fits the kernels and that the buffer is large enough and 256-byte aligned.
+int decode_layout(const hils::Params& P, void* ws, size_t ws_bytes, hils::DecodeWs* w) {
+  if (P.Hq > 64) return fail(HILS_ERR_UNSUPPORTED, "decode supports up to 64 query heads");
+  const size_t need = hils::decode_ws_bytes(P, w, nullptr);
+  if (w->n_split > hils::kMaxSplitLists)
+    return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
+                hils::kMaxSplitLists, P.max_chunks, w->n_split);
+  if (hils::decode_smem_bytes(P, *w) > 227 * 1024)
+    return fail(HILS_ERR_UNSUPPORTED,
+                "decode of %d query heads per KV head over %d chunk ranges needs more shared "
+                "memory than a CTA has", P.group, w->n_split);
+  if (!ws || ws_bytes < need)
+    return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
+  if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  hils::decode_ws_bytes(P, w, (char*)ws);
+  return HILS_OK;
+}
+}  // namespace
+
+// ---- context-parallel decode ----
+namespace {
+int cp_common(const hils_config* cfg, const void* q, const void* k_new, const void* v_new,
+              hils::Params* P) {
+  if (!q || !aligned16(q)) return fail(HILS_ERR_INVALID_ARG, "q is NULL or misaligned");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  P->q = q;
+  P->L = 1;
+  return HILS_OK;
+}
+}  // namespace
+
+int hils_decode_cp_candidates(const hils_config* cfg, const void* q, const void* k_new,
+                              const void* v_new, const float* A, const float* B,
+                              hils_kv_cache* shard, int64_t chunk_base, uint64_t* keys,
+                              float* own_score, void* ws, size_t ws_bytes, void* stream) {
+  hils::Params P{};
+  int st;
+  if ((st = check_config(cfg, &P)) || (st = check_calib(cfg, A, B, &P)) ||
+      (st = check_pages(shard, &P)) || (st = cp_common(cfg, q, k_new, v_new, &P)))
+    return st;
+  if (!shard->seq_lens) return fail(HILS_ERR_INVALID_ARG, "shard->seq_lens is required");
+  if (chunk_base < 0) return fail(HILS_ERR_INVALID_ARG, "chunk_base must be >= 0");
+  if ((cfg->top_k > 1 && !keys) || !own_score)
+    return fail(HILS_ERR_INVALID_ARG, "keys and own_score are required");
+  hils::DecodeWs w{};
+  if ((st = decode_layout(P, ws, ws_bytes, &w))) return st;
+  w.chunk_base = chunk_base;
+  w.cp_keys = keys;
+  w.cp_own = own_score;
+  if (P.B == 0) return HILS_OK;
+  cudaError_t e = hils::launch_cp_candidates(P, k_new, v_new, w, (cudaStream_t)stream);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode_cp_candidates");
+}
+
+int hils_decode_cp_select(const hils_config* cfg, int32_t world, const uint64_t* keys,
+                          const float* own_scores, const int32_t* seq_lens, int32_t append,
+                          int32_t* idx, float* w, void* stream) {
+  hils::Params P{};
+  int st;
+  if ((st = check_config(cfg, &P))) return st;
+  if (world < 1) return fail(HILS_ERR_INVALID_ARG, "world must be positive");
+  if ((cfg->top_k > 1 && !keys) || !own_scores || !seq_lens || !idx || !w)
+    return fail(HILS_ERR_INVALID_ARG, "keys, own_scores, seq_lens, idx and w are required");
+  P.seq_lens = const_cast<int32_t*>(seq_lens);
+  if (P.B == 0) return HILS_OK;
+  cudaError_t e = hils::launch_cp_select(P, world, keys, own_scores, append != 0, idx, w,
+                                         (cudaStream_t)stream);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode_cp_select");
+}
+
+int hils_decode_cp_attend(const hils_config* cfg, const void* q, const void* k_new,
+                          const void* v_new, const hils_kv_cache* shard, int64_t chunk_base,
+                          const int32_t* idx, const float* w, float* partial, void* stream) {
+  hils::Params P{};
+  int st;
+  if ((st = check_config(cfg, &P)) || (st = check_pages(shard, &P)) ||
+      (st = cp_common(cfg, q, k_new, v_new, &P)))
+    return st;
+  if (!shard->seq_lens) return fail(HILS_ERR_INVALID_ARG, "shard->seq_lens is required");
+  if (chunk_base < 0) return fail(HILS_ERR_INVALID_ARG, "chunk_base must be >= 0");
+  if (!idx || !w || !partial) return fail(HILS_ERR_INVALID_ARG, "idx, w and partial are required");
+  if (P.B == 0) return HILS_OK;
+  cudaError_t e = hils::launch_cp_attend(P, chunk_base, k_new, v_new, idx, w, partial,
+                                         (cudaStream_t)stream);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode_cp_attend");
+}
+
+int hils_decode_cp_finish(const hils_config* cfg, const float* sum, void* out, int32_t* seq_lens,
+                          int32_t append, void* stream) {
+  hils::Params P{};
+  int st;
+  if ((st = check_config(cfg, &P))) return st;
+  if (!sum || !out) return fail(HILS_ERR_INVALID_ARG, "sum and out are required");
+  if (append && !seq_lens) return fail(HILS_ERR_INVALID_ARG, "seq_lens is required to append");
+  P.seq_lens = seq_lens;
+  if (P.B == 0) return HILS_OK;
+  cudaError_t e = hils::launch_cp_finish(P, sum, out, append != 0, (cudaStream_t)stream);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_decode_cp_finish");
+}
+
 int hils_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "hils_device_status: stream synchronize");
@@ -269,23 +374,11 @@ int decode_call(const hils_config* cfg, const void* q, const void* k_new, const 
   if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
     return fail(HILS_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (!cache->seq_lens) return fail(HILS_ERR_INVALID_ARG, "cache->seq_lens is required for decode");
-  if (P.Hq > 64) return fail(HILS_ERR_UNSUPPORTED, "decode supports up to 64 query heads");
   P.q = q;
   P.L = 1;
   P.pos0 = 0;
   DecodeWs w{};
-  const size_t need = decode_ws_bytes(P, &w, nullptr);
-  if (w.n_split > kMaxSplitLists)
-    return fail(HILS_ERR_UNSUPPORTED, "decode supports up to %d chunk ranges (max_chunks %d needs %d)",
-                kMaxSplitLists, P.max_chunks, w.n_split);
-  if (decode_smem_bytes(P, w) > 227 * 1024)
-    return fail(HILS_ERR_UNSUPPORTED,
-                "decode of %d query heads per KV head over %d chunk ranges needs more shared "
-                "memory than a CTA has", P.group, w.n_split);
-  if (!ws || ws_bytes < need)
-    return fail(HILS_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws_bytes);
-  if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  decode_ws_bytes(P, &w, (char*)ws);
+  if ((st = decode_layout(P, ws, ws_bytes, &w))) return st;
   if (P.B == 0) return HILS_OK;
   cudaError_t e;
   if (clear_counters &&

@@ -195,6 +195,17 @@ struct DecodeWs {
   size_t ticket_bytes;
   int n_split, chunks_per_split;
   int append;          // k_new / v_new given
+  // context-parallel mode (cp_keys or cp_partial set): the cache holds the
+  // chunks chunk_base .. chunk_base + max_chunks - 1 of every sequence and
+  // seq_lens the global positions.  The scan then leaves the merged keys
+  // [B][Hq][k-1] and the own chunk's score [B][Hq] (-inf where not held)
+  // instead of the weights; the attention reads idx and w (global chunks),
+  // looks the pages up itself and writes float32 weighted sums to cp_partial
+  // without advancing seq_lens.
+  int64_t chunk_base;
+  uint64_t* cp_keys;
+  float* cp_own;
+  float* cp_partial;
 };
 size_t decode_ws_bytes(const Params& P, DecodeWs* ws, char* base);
 // Dynamic shared memory of the decode kernel for this configuration.
@@ -207,5 +218,20 @@ int decode_call(const hils_config* cfg, const void* q, const void* k_new, const 
                 float* w_out, void* ws, size_t ws_bytes, bool clear_counters, void* stream);
 cudaError_t launch_decode(const Params& P, const void* k_new, const void* v_new, void* out,
                           int32_t* idx_out, float* w_out, const DecodeWs& ws, cudaStream_t s);
+
+// Context-parallel decode (this GPU holds chunks chunk_base .. chunk_base +
+// P.max_chunks - 1 of every sequence); see hils_decode_cp_* in hils.h.
+// The scan over this GPU's chunks; ws laid out by decode_ws_bytes for the
+// shard, with chunk_base, cp_keys and cp_own set.
+cudaError_t launch_cp_candidates(const Params& P, const void* k_new, const void* v_new,
+                                 const DecodeWs& ws, cudaStream_t s);
+cudaError_t launch_cp_select(const Params& P, int world, const uint64_t* keys,
+                             const float* own_scores, bool append, int32_t* idx, float* w,
+                             cudaStream_t s);
+cudaError_t launch_cp_attend(const Params& P, int64_t chunk_base, const void* k_new,
+                             const void* v_new, const int32_t* idx, const float* w, float* partial,
+                             cudaStream_t s);
+cudaError_t launch_cp_finish(const Params& P, const float* sum, void* out, bool append,
+                             cudaStream_t s);
 
 }  // namespace hils

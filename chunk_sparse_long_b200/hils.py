@@ -26,7 +26,9 @@ STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
 EXPORTED = ("hils_workspace_size", "hils_score", "hils_topk", "hils_prefill", "hils_decode",
             "hils_device_status", "hils_last_error", "hils_version", "hils_profile_enable",
             "hils_profile_collect", "hils_profile_read", "hils_profile_reset",
-            "hils_decode_noalloc", "hils_decode_noalloc_capacity", "hils_set_wait_limit_ns")
+            "hils_decode_noalloc", "hils_decode_noalloc_capacity", "hils_set_wait_limit_ns",
+            "hils_decode_cp_candidates", "hils_decode_cp_select", "hils_decode_cp_attend",
+            "hils_decode_cp_finish")
 
 
 class HilsError(RuntimeError):
@@ -94,6 +96,15 @@ def load(path: str = LIB_PATH):
     L.hils_decode_noalloc_capacity.argtypes = []
     L.hils_set_wait_limit_ns.restype = ctypes.c_int
     L.hils_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.hils_decode_cp_candidates.restype = ctypes.c_int
+    L.hils_decode_cp_candidates.argtypes = [cfgp, P, P, P, P, P, cachep, I64, P, P, P,
+                                            ctypes.c_size_t, P]
+    L.hils_decode_cp_select.restype = ctypes.c_int
+    L.hils_decode_cp_select.argtypes = [cfgp, I32, P, P, P, I32, P, P, P]
+    L.hils_decode_cp_attend.restype = ctypes.c_int
+    L.hils_decode_cp_attend.argtypes = [cfgp, P, P, P, cachep, I64, P, P, P, P]
+    L.hils_decode_cp_finish.restype = ctypes.c_int
+    L.hils_decode_cp_finish.argtypes = [cfgp, P, P, P, I32, P]
     _lib = L
     return L
 
@@ -191,6 +202,40 @@ def decode_noalloc(cfg, q, k_new, v_new, A, B, cache: Cache, out, idx_out, w_out
                                       _ptr(A), _ptr(B), ctypes.byref(cache.c()), _ptr(out),
                                       _ptr(idx_out), _ptr(w_out), _stream(stream)),
            "hils_decode_noalloc")
+
+
+def decode_cp_candidates(cfg, q, k_new, v_new, A, B, shard: Cache, chunk_base, keys, own_score,
+                         ws, ws_bytes, stream=None):
+    """Context-parallel decode, step 1 (include/hils.h): this shard's best k-1
+    selection keys (int64 tensor holding the 64-bit keys) and own-chunk score;
+    ws is the shard's zeroed decode workspace."""
+    _check(load().hils_decode_cp_candidates(ctypes.byref(cfg.c()), _ptr(q), _ptr(k_new),
+                                            _ptr(v_new), _ptr(A), _ptr(B),
+                                            ctypes.byref(shard.c()), chunk_base, _ptr(keys),
+                                            _ptr(own_score), _ptr(ws), ws_bytes, _stream(stream)),
+           "hils_decode_cp_candidates")
+
+
+def decode_cp_select(cfg, world, keys, own_scores, seq_lens, append, idx, w, stream=None):
+    """Context-parallel decode, step 3: the selection from the gathered lists."""
+    _check(load().hils_decode_cp_select(ctypes.byref(cfg.c()), world, _ptr(keys), _ptr(own_scores),
+                                        _ptr(seq_lens), int(bool(append)), _ptr(idx), _ptr(w),
+                                        _stream(stream)), "hils_decode_cp_select")
+
+
+def decode_cp_attend(cfg, q, k_new, v_new, shard: Cache, chunk_base, idx, w, partial,
+                     stream=None):
+    """Context-parallel decode, step 4: this shard's weighted outputs (float32)."""
+    _check(load().hils_decode_cp_attend(ctypes.byref(cfg.c()), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                        ctypes.byref(shard.c()), chunk_base, _ptr(idx), _ptr(w),
+                                        _ptr(partial), _stream(stream)), "hils_decode_cp_attend")
+
+
+def decode_cp_finish(cfg, total, out, seq_lens, append, stream=None):
+    """Context-parallel decode, step 6: the output from the summed partials."""
+    _check(load().hils_decode_cp_finish(ctypes.byref(cfg.c()), _ptr(total), _ptr(out),
+                                        _ptr(seq_lens), int(bool(append)), _stream(stream)),
+           "hils_decode_cp_finish")
 
 
 def decode_noalloc_capacity() -> int:

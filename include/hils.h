@@ -128,6 +128,57 @@ int hils_decode(const hils_config* cfg, const void* q, const void* k_new, const 
                 const float* A, const float* B, hils_kv_cache* cache, void* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Context-parallel decode: one sequence's chunks spread over several GPUs
+ * (the decode step beyond one GPU's memory).  Each GPU ("rank") holds the
+ * chunks chunk_base .. chunk_base + shard->max_chunks - 1 of every sequence:
+ * `shard` is a cache of its own (pages, block table and landmarks indexed by
+ * local chunk, j - chunk_base), and shard->seq_lens holds the global token
+ * counts, the same on every rank.  t = seq_lens[b] when appending (k_new and
+ * v_new given), else seq_lens[b] - 1; the own chunk is t / chunk_size.  One
+ * step is four calls around two collectives that the caller runs (NCCL, for
+ * instance); the pieces follow the paper's fusion (review, 二: each chunk's
+ * attention weighted by its retrieval score; digest, 局限: every landmark is
+ * scored at every step), split so that only the candidate lists and the
+ * d-vectors of the weighted outputs cross between GPUs:
+ *   1. hils_decode_cp_candidates: this shard's best k-1 chunks before the
+ *      own one, per (sequence, query head), as 64-bit selection keys, best
+ *      first, into keys [B][Hq][k-1] (key 0 = none; a larger key ranks higher
+ *      in (score desc, chunk asc): the high word is the float32 score mapped
+ *      to an unsigned order, the low word is the complement of the global
+ *      chunk index), and the own chunk's score into own_score [B][Hq] on the
+ *      rank holding it (-inf elsewhere).  That rank appends k_new, v_new.
+ *      ws: the shard's decode workspace, at least hils_workspace_size(cfg,
+ *      HILS_OP_DECODE, 1, shard->max_chunks) bytes, 256-byte aligned, zeroed
+ *      once before the first call and kept (as for hils_decode).
+ *   2. all-gather of keys and own_score over the ranks, in rank order.
+ *   3. hils_decode_cp_select: the global selection and fusion weights from
+ *      the gathered keys [world][B][Hq][k-1] and own scores [world][B][Hq],
+ *      into idx and w [B][Hq][k] (global chunk indices; the same on every
+ *      rank, and the same slot order and weights as hils_decode).
+ *   4. hils_decode_cp_attend: the weighted outputs of the selected chunks
+ *      this shard holds, float32 partial [B][Hq][d] (zero where none).
+ *   5. all-reduce (sum) of partial.
+ *   6. hils_decode_cp_finish: out [B][Hq][d] in cfg->dtype from the sum;
+ *      seq_lens advanced by one when `append` (call it on every rank, each
+ *      with its own seq_lens).
+ * All arrays are device memory; nothing is allocated.  Steps 1 and 4 run
+ * the kernels of hils_decode (the chunk ranges of the scan spread over CTAs,
+ * the selected chunks over a cluster of CTAs per head) on the shard.  A step's calls go to
+ * one stream per rank, in this order.  The own chunk must be held by exactly
+ * one rank; hils_device_status() reports HILS_ERR_DEVICE_CHECK otherwise. */
+int hils_decode_cp_candidates(const hils_config* cfg, const void* q, const void* k_new,
+                              const void* v_new, const float* A, const float* B,
+                              hils_kv_cache* shard, int64_t chunk_base, uint64_t* keys,
+                              float* own_score, void* ws, size_t ws_bytes, void* stream);
+int hils_decode_cp_select(const hils_config* cfg, int32_t world, const uint64_t* keys,
+                          const float* own_scores, const int32_t* seq_lens, int32_t append,
+                          int32_t* idx, float* w, void* stream);
+int hils_decode_cp_attend(const hils_config* cfg, const void* q, const void* k_new,
+                          const void* v_new, const hils_kv_cache* shard, int64_t chunk_base,
+                          const int32_t* idx, const float* w, float* partial, void* stream);
+int hils_decode_cp_finish(const hils_config* cfg, const float* sum, void* out, int32_t* seq_lens,
+                          int32_t append, void* stream);
+
 /* The decode step without a workspace argument, for callers that cannot
  * allocate device memory: plugins run by a host engine that owns every device
  * allocation and passes kernels only their inputs and outputs, and services

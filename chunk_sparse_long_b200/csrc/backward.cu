@@ -1,0 +1,399 @@
+// Prefill backward of HiLS attention with the chunk selection held fixed: the
+// gradients of sum(dout * out) with respect to q, the K/V page pool, the
+// landmarks and the calibration matrices A, B.  The pages train the model end
+// to end under the language-modelling loss, with the retrieval scores inside
+// the forward pass so that gradients reach them (ai-feeds.com digest,
+// "关键模块" item 1: the scores are fully differentiable, item 3: native
+// sparse training, and "输出与训练"; chatpaper abstract: chunk selection
+// learned end to end).  Which chunks are selected is a discrete choice and
+// carries no gradient.
+//
+// Notation as in the forward: row (b, i, h) at position t = pos0 + i, KV head
+// g, selected chunks j with fusion weights w_j, per-chunk probabilities P_j
+// and outputs O_j, out = sum_j w_j O_j.
+//   attention  one CTA per work item of the key-major buckets (up to 128
+//              pairs of one chunk and KV head): K_j and V_j are staged once;
+//              per pair, P_j and O_j are recomputed exactly (a chunk has 64
+//              keys, so no softmax statistics need to be kept), dw_j =
+//              dout . O_j is kept per pair, and with G = w_j dout:
+//                dS = P_j (G V_j^T - G . O_j),  dq += dS K_j / sqrt(d);
+//              dK_j += dS^T q / sqrt(d) and dV_j += P_j^T G are products over
+//              the item's pairs, added into the pool's gradient once per item.
+//   scores     per row: ds_j = w_j (dw_j - sum_l w_l dw_l) (softmax
+//              derivative), dq~ = sum_j ds_j lm_j / sqrt(d), dlm_j += ds_j q~ /
+//              sqrt(d), and through q~ = q + (qA)B: dq += dq~ + (dq~ B^T) A^T,
+//              dA += q^T (dq~ B^T), dB += (qA)^T dq~, the last two as products
+//              over groups of 32 rows, added once per CTA.
+// All arithmetic is float32 on CUDA cores.  Every gradient output is added
+// into (the caller zeroes it first); the order of the float additions into
+// dq, the pool and the landmarks is not fixed.
+#include "hils_common.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSub = 16;        // pairs per sub-tile of an attention item: two per warp
+constexpr int kRowGroup = 32;   // rows per group of the score backward: four per warp
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// Shared memory of the attention backward, in floats.
+template <int D>
+struct AttnSmem {
+  static constexpr int LD = D + 1;                  // K and V row stride: conflict-free rows
+  static constexpr int kK = 0;                      // [64][LD]
+  static constexpr int kV = kK + kChunk * LD;       // [64][LD]
+  static constexpr int kQ = kV + kChunk * LD;       // [kSub][D] the pairs' raw q rows
+  static constexpr int kG = kQ + kSub * D;          // [kSub][D] G = w dout
+  static constexpr int kP = kG + kSub * D;          // [kSub][64] probabilities
+  static constexpr int kS = kP + kSub * kChunk;     // [kSub][64] dS
+  static constexpr size_t kBytes = (size_t)(kS + kSub * kChunk) * sizeof(float);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) attn_bwd_kernel(Params P, PrefillWs ws,
+                                                            const float* wts, const void* dout,
+                                                            float* dq, float* dpages, float* dw) {
+  using L = AttnSmem<D>;
+  constexpr int LD = L::LD;
+  constexpr int EPL = D / 32;             // row elements per lane: e = lane + 32 c
+  constexpr int NRG = kThreads / D;       // row groups of the dK / dV products
+  constexpr int RPT = kChunk / NRG;       // K / V rows per thread in those products
+  extern __shared__ float sm[];
+  float* sK = sm + L::kK;
+  float* sV = sm + L::kV;
+  float* sQ = sm + L::kQ;
+  float* sG = sm + L::kG;
+  float* sP = sm + L::kP;
+  float* sS = sm + L::kS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x;
+  if (tile >= ws.tile_off[ws.n_keys]) return;
+  const int4 item = ws.items[tile];
+  const int key = item.x;
+  const int j = key % P.max_chunks;
+  const int bg = key / P.max_chunks / ws.n_win;
+  const int g = bg % P.Hkv, b = bg / P.Hkv;
+  const int64_t page = page_of(P, b, j);
+  if (page < 0) return;
+  for (int x = tid; x < kChunk * (D / 8); x += kThreads) {
+    const int s = x / (D / 8), e8 = (x % (D / 8)) * 8;
+    float v[8];
+    load8(P.pages, P.dtype, page_offset(P, page, 0, g, s) + e8, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sK[s * LD + e8 + u] = v[u];
+    load8(P.pages, P.dtype, page_offset(P, page, 1, g, s) + e8, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sV[s * LD + e8 + u] = v[u];
+  }
+  // this thread's part of dK and dV: column ce, rows rg + NRG m
+  const int ce = tid % D, rg = tid / D;
+  float aK[RPT], aV[RPT];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) aK[m] = aV[m] = 0.f;
+  const float sc = P.inv_sqrt_d;
+  __syncthreads();
+  for (int sb = item.y; sb < item.z; sb += kSub) {
+    const int n = min(kSub, item.z - sb);
+    for (int ps = warp; ps < n; ps += kWarps) {
+      const int32_t pid = ws.pairs[sb + ps];
+      const int64_t r = pid / P.k;
+      const int64_t pos = P.pos0 + (r / P.Hq) % P.L;
+      const int nk = pos / kChunk == j ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
+      const float wj = __ldg(wts + pid);
+      float* q = sQ + ps * D;
+      float* G = sG + ps * D;
+      float go[EPL];
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) {
+        const int e = lane + 32 * c;
+        q[e] = load_elem(P.q, P.dtype, r * D + e);
+        go[c] = load_elem(dout, P.dtype, r * D + e);
+      }
+      __syncwarp();
+      // logits of keys lane and lane + 32, then the chunk's probabilities
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < D; ++e) {
+        s0 = fmaf(q[e], sK[lane * LD + e], s0);
+        s1 = fmaf(q[e], sK[(lane + 32) * LD + e], s1);
+      }
+      s0 = lane < nk ? s0 * sc : -INFINITY;
+      s1 = lane + 32 < nk ? s1 * sc : -INFINITY;
+      const float mx = warp_max(fmaxf(s0, s1));
+      float p0 = __expf(s0 - mx), p1 = __expf(s1 - mx);
+      const float inv_l = 1.f / warp_sum(p0 + p1);
+      p0 *= inv_l;
+      p1 *= inv_l;
+      // O_j and dw_j = dout . O_j
+      float o[EPL];
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) o[c] = 0.f;
+      for (int t = 0; t < kChunk; ++t) {
+        const float pt = __shfl_sync(kFull, t < 32 ? p0 : p1, t & 31);
+#pragma unroll
+        for (int c = 0; c < EPL; ++c) o[c] = fmaf(pt, sV[t * LD + lane + 32 * c], o[c]);
+      }
+      float part = 0.f;
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) part = fmaf(go[c], o[c], part);
+      const float dwj = warp_sum(part);
+      if (lane == 0) dw[pid] = dwj;
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) G[lane + 32 * c] = wj * go[c];
+      __syncwarp();
+      // dP = G V^T at keys lane and lane + 32; dS = P (dP - G . O) with G . O = w dw
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < D; ++e) {
+        d0 = fmaf(G[e], sV[lane * LD + e], d0);
+        d1 = fmaf(G[e], sV[(lane + 32) * LD + e], d1);
+      }
+      const float go_o = wj * dwj;
+      const float ds0 = p0 * (d0 - go_o), ds1 = p1 * (d1 - go_o);
+      sP[ps * kChunk + lane] = p0;
+      sP[ps * kChunk + lane + 32] = p1;
+      sS[ps * kChunk + lane] = ds0;
+      sS[ps * kChunk + lane + 32] = ds1;
+      // dq += dS K / sqrt(d)
+      float aq[EPL];
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) aq[c] = 0.f;
+      for (int t = 0; t < kChunk; ++t) {
+        const float st = __shfl_sync(kFull, t < 32 ? ds0 : ds1, t & 31);
+#pragma unroll
+        for (int c = 0; c < EPL; ++c) aq[c] = fmaf(st, sK[t * LD + lane + 32 * c], aq[c]);
+      }
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) atomicAdd(dq + r * D + lane + 32 * c, aq[c] * sc);
+    }
+    __syncthreads();
+    // dK += dS^T q and dV += P^T G over the sub-tile's pairs
+    for (int ps = 0; ps < n; ++ps) {
+      const float qe = sQ[ps * D + ce], ge = sG[ps * D + ce];
+      const float* srow = sS + ps * kChunk;
+      const float* prow = sP + ps * kChunk;
+#pragma unroll
+      for (int m = 0; m < RPT; ++m) {
+        const int t = rg + NRG * m;
+        aK[m] = fmaf(srow[t], qe, aK[m]);
+        aV[m] = fmaf(prow[t], ge, aV[m]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const int t = rg + NRG * m;
+    atomicAdd(dpages + page_offset(P, page, 0, g, t) + ce, aK[m] * sc);
+    atomicAdd(dpages + page_offset(P, page, 1, g, t) + ce, aV[m]);
+  }
+}
+
+// Shared memory of the score backward, in floats: A [D][r + 1], B [r][D + 1]
+// (padded rows), then per group of rows q [32][D], dq~ [32][D], qA [32][r]
+// and dq~ B^T [32][r].
+template <int D>
+size_t score_bwd_smem(int r) {
+  const int rr = r > 0 ? r : 1;
+  return sizeof(float) * ((size_t)D * (r + 1) + (size_t)r * (D + 1) + 2 * kRowGroup * D +
+                          2 * kRowGroup * rr);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) score_bwd_kernel(Params P, const int32_t* idx,
+                                                             const float* wts, const float* dw,
+                                                             float* dq, float* dlm, float* dA,
+                                                             float* dB) {
+  constexpr int EPL = D / 32;
+  constexpr int NA = kThreads / D;         // rank groups of the dA / dB products
+  constexpr int MAXA = kMaxRank / NA;      // rank entries per thread, at most
+  const int R = P.r;
+  const int RA = R + 1, RB = D + 1, RR = R > 0 ? R : 1;
+  extern __shared__ float sm[];
+  float* sA = sm;                          // [D][RA]
+  float* sB = sA + D * RA;                 // [R][RB]
+  float* sq = sB + R * RB;                 // [kRowGroup][D]
+  float* sdqt = sq + kRowGroup * D;        // [kRowGroup][D]
+  float* st = sdqt + kRowGroup * D;        // [kRowGroup][RR]  q A
+  float* su = st + kRowGroup * RR;         // [kRowGroup][RR]  dq~ B^T
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int x = tid; x < D * R; x += kThreads) sA[(x / R) * RA + x % R] = P.A[x];
+  for (int x = tid; x < R * D; x += kThreads) sB[(x / D) * RB + x % D] = P.Bm[x];
+  const int ce = tid % D, a0 = tid / D;    // this thread's dA column e = ce, ranks a0 + NA m
+  float gA[MAXA], gB[MAXA];
+#pragma unroll
+  for (int m = 0; m < MAXA; ++m) gA[m] = gB[m] = 0.f;
+  const float sc = P.inv_sqrt_d;
+  const int64_t rows = (int64_t)P.B * P.L * P.Hq;
+  const int64_t n_groups = (rows + kRowGroup - 1) / kRowGroup;
+  __syncthreads();
+  for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+    for (int lr = warp; lr < kRowGroup; lr += kWarps) {
+      const int64_t row = grp * kRowGroup + lr;
+      float* q = sq + lr * D;
+      float* dqt = sdqt + lr * D;
+      float* t = st + lr * RR;
+      float* u = su + lr * RR;
+      if (row >= rows) {   // past the last row: contributes nothing to dA, dB
+#pragma unroll
+        for (int c = 0; c < EPL; ++c) q[lane + 32 * c] = dqt[lane + 32 * c] = 0.f;
+        for (int a = lane; a < RR; a += 32) t[a] = u[a] = 0.f;
+        continue;
+      }
+      const int h = (int)(row % P.Hq);
+      const int b = (int)(row / P.Hq / P.L);
+      const int g = h / P.group;
+      // lane s holds slot s: the softmax derivative ds = w (dw - sum w dw)
+      int32_t js = -1;
+      float wv = 0.f, dwv = 0.f;
+      if (lane < P.k) {
+        js = idx[row * P.k + lane];
+        if (js >= 0) {
+          wv = wts[row * P.k + lane];
+          dwv = dw[row * P.k + lane];
+        }
+      }
+      const float dsum = warp_sum(wv * dwv);
+      const float ds = wv * (dwv - dsum);
+      // q, then t = q A
+      float qe[EPL];
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) {
+        qe[c] = load_elem(P.q, P.dtype, row * D + lane + 32 * c);
+        q[lane + 32 * c] = qe[c];
+      }
+      __syncwarp();
+      for (int a = lane; a < R; a += 32) {
+        float acc = 0.f;
+        for (int e = 0; e < D; ++e) acc = fmaf(q[e], sA[e * RA + a], acc);
+        t[a] = acc;
+      }
+      __syncwarp();
+      // q~ = q + t B; dq~ = sum_j ds_j lm_j / sqrt(d); dlm_j += ds_j q~ / sqrt(d)
+      float qt[EPL], gq[EPL];
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) {
+        float acc = qe[c];
+        for (int a = 0; a < R; ++a) acc = fmaf(t[a], sB[a * RB + lane + 32 * c], acc);
+        qt[c] = acc;
+        gq[c] = 0.f;
+      }
+      for (int s = 0; s < P.k; ++s) {
+        const int32_t j = __shfl_sync(kFull, js, s);
+        const float dss = __shfl_sync(kFull, ds, s);
+        if (j < 0) continue;
+        if (j >= P.max_chunks) {
+          if (lane == 0) set_device_error(kErrChunk);
+          continue;
+        }
+        const int64_t lrow = (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * D;
+#pragma unroll
+        for (int c = 0; c < EPL; ++c) {
+          const int e = lane + 32 * c;
+          gq[c] = fmaf(dss, load_elem(P.landmarks, P.dtype, lrow + e), gq[c]);
+          atomicAdd(dlm + lrow + e, dss * qt[c] * sc);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) {
+        gq[c] *= sc;
+        dqt[lane + 32 * c] = gq[c];
+      }
+      __syncwarp();
+      // u = dq~ B^T, then dq += dq~ + A u
+      for (int a = lane; a < R; a += 32) {
+        float acc = 0.f;
+        for (int e = 0; e < D; ++e) acc = fmaf(sB[a * RB + e], dqt[e], acc);
+        u[a] = acc;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < EPL; ++c) {
+        const int e = lane + 32 * c;
+        float acc = gq[c];
+        for (int a = 0; a < R; ++a) acc = fmaf(sA[e * RA + a], u[a], acc);
+        dq[row * D + e] += acc;
+      }
+    }
+    __syncthreads();
+    // dA += q^T u and dB += t^T dq~ over the group's rows
+    if (R > 0) {
+      for (int lr = 0; lr < kRowGroup; ++lr) {
+        const float qv = sq[lr * D + ce], gv = sdqt[lr * D + ce];
+#pragma unroll
+        for (int m = 0; m < MAXA; ++m) {
+          const int a = a0 + NA * m;
+          if (a < R) {
+            gA[m] = fmaf(qv, su[lr * RR + a], gA[m]);
+            gB[m] = fmaf(st[lr * RR + a], gv, gB[m]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (R > 0) {
+#pragma unroll
+    for (int m = 0; m < MAXA; ++m) {
+      const int a = a0 + NA * m;
+      if (a < R) {
+        atomicAdd(dA + ce * R + a, gA[m]);
+        atomicAdd(dB + a * D + ce, gB[m]);
+      }
+    }
+  }
+}
+
+template <int D>
+cudaError_t run_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
+                         float* dq, float* dpages, float* dlm, float* dA, float* dB,
+                         const PrefillWs& ws, float* dw, cudaStream_t s) {
+  const int64_t rows = (int64_t)P.B * P.L * P.Hq;
+  cudaError_t e;
+  // every pair's dw is written by the attention pass; zero first, so that a
+  // pair the bucketing rejected (its chunk out of range) reads as 0
+  if ((e = cudaMemsetAsync(dw, 0, sizeof(float) * rows * P.k, s)) != cudaSuccess) return e;
+  if ((e = launch_bucketing(P, idx, w, ws, false, kBackwardTilePairs, "backward.bucket", s)) != cudaSuccess) return e;
+  constexpr size_t asm_ = AttnSmem<D>::kBytes;
+  if ((e = set_smem(attn_bwd_kernel<D>, asm_)) != cudaSuccess) return e;
+  {
+    HILS_PROFILE("backward.attention", s);
+    attn_bwd_kernel<D><<<(unsigned)ws.max_tiles, kThreads, asm_, s>>>(P, ws, w, dout, dq, dpages,
+                                                                      dw);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t ssm = score_bwd_smem<D>(P.r);
+  if ((e = set_smem(score_bwd_kernel<D>, ssm)) != cudaSuccess) return e;
+  const int64_t n_groups = (rows + kRowGroup - 1) / kRowGroup;
+  const unsigned nb = (unsigned)(n_groups < 2 * 148 ? n_groups : 2 * 148);
+  {
+    HILS_PROFILE("backward.scores", s);
+    score_bwd_kernel<D><<<nb, kThreads, ssm, s>>>(P, idx, w, dw, dq, dlm, dA, dB);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
+                            float* dq, float* dpages, float* dlm, float* dA, float* dB,
+                            const PrefillWs& ws, float* dw, cudaStream_t s) {
+  if (P.L == 0 || P.B == 0) return cudaSuccess;
+  return P.d == 64 ? run_backward<64>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, dw, s)
+                   : run_backward<128>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, dw, s);
+}
+
+}  // namespace hils

@@ -178,6 +178,23 @@ struct PrefillWs {
   int64_t max_tiles;
 };
 size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base);
+// Key-major bucketing of the (row, slot) pairs of idx [B][L][Hq][k] by
+// (sequence, KV head, query window, chunk) into ws: counts, offsets, the work
+// items (up to tile_pairs pairs of one key each) and, per pair in bucket
+// order, either its id row * k + slot (ws.pairs) or, with records, its
+// tensor-core record (ws.pinfo).
+cudaError_t launch_bucketing(const Params& P, const int32_t* idx, const float* w,
+                             const PrefillWs& ws, bool records, int tile_pairs, const char* label,
+                             cudaStream_t s);
+
+// Prefill backward with the selection fixed (hils_prefill_backward): the
+// bucketing arrays of ws (pair ids, tiles of kBackwardTilePairs) and dw, one
+// float per pair.  With base == nullptr only the size is computed.
+constexpr int kBackwardTilePairs = 128;
+size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base);
+cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
+                            float* dq, float* dpages, float* dlm, float* dA, float* dB,
+                            const PrefillWs& ws, float* dw, cudaStream_t s);
 cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
                            const PrefillWs& ws, cudaStream_t s);
 cudaError_t launch_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, float* w,

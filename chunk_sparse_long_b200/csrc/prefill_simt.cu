@@ -531,44 +531,9 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // bucket by (sequence, KV head, chunk)
-  if ((e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ws.n_keys, s)) != cudaSuccess) return e;
-  {
-    HILS_PROFILE("prefill.bucket", s);
-    const int tile_pairs = P.dtype == HILS_BF16 ? kItemPairs : kTilePairs;
-    const int64_t nvis_max = min((int64_t)P.max_chunks, (P.pos0 + P.L - 1) / kChunk + 1);
-    const size_t hsm = sizeof(int32_t) * 2 * (size_t)nvis_max;
-    if (nvis_max <= kHistMax) {
-      if ((e = set_smem(bucket_scatter_kernel, hsm)) !=
-          cudaSuccess)
-        return e;
-      if ((e = set_smem(bucket_count_kernel, hsm)) !=
-          cudaSuccess)
-        return e;
-      const dim3 bgrid((unsigned)((P.L + kBucketRows - 1) / kBucketRows), P.Hkv, P.B);
-      const Windows W{ws.n_win, ws.win_rows};
-      bucket_count_kernel<<<bgrid, 256, hsm / 2, s>>>(P, ws.idx, ws.counts, W);
-      {
-        const unsigned nb = (unsigned)((ws.n_keys + kScanBlock - 1) / kScanBlock);
-        scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
-        scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
-                                              ws.offsets, ws.tile_off, ws.cursor, ws.items);
-      }
-      bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, ws.idx, ws.w, ws.cursor, ws.pairs,
-                                                    P.dtype == HILS_BF16 ? ws.pinfo : nullptr, W);
-    } else {
-      const unsigned pb = (unsigned)((n_pairs + 255) / 256);
-      const Windows W{ws.n_win, ws.win_rows};
-      count_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.counts, n_pairs, W);
-      {
-        const unsigned nb = (unsigned)((ws.n_keys + kScanBlock - 1) / kScanBlock);
-        scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
-        scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
-                                              ws.offsets, ws.tile_off, ws.cursor, ws.items);
-      }
-      scatter_kernel<<<pb, 256, 0, s>>>(P, ws.idx, ws.w, ws.cursor, ws.pairs,
-                                        P.dtype == HILS_BF16 ? ws.pinfo : nullptr, n_pairs, W);
-    }
-  }
+  e = launch_bucketing(P, ws.idx, ws.w, ws, P.dtype == HILS_BF16,
+                       P.dtype == HILS_BF16 ? kItemPairs : kTilePairs, "prefill.bucket", s);
+  if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // a5 + a6
   if (P.dtype == HILS_BF16) return launch_attn_tc(P, out, ws, s);
@@ -591,19 +556,57 @@ cudaError_t run_prefill(const Params& P, void* out, const PrefillWs& ws, cudaStr
 
 }  // namespace
 
+cudaError_t launch_bucketing(const Params& P, const int32_t* idx, const float* wts,
+                             const PrefillWs& ws, bool records, int tile_pairs, const char* label,
+                             cudaStream_t s) {
+  const int64_t n_pairs = (int64_t)P.B * P.L * P.Hq * P.k;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ws.n_keys, s)) != cudaSuccess) return e;
+  HILS_PROFILE(label, s);
+  const Windows W{ws.n_win, ws.win_rows};
+  const int64_t nvis_max = min((int64_t)P.max_chunks, (P.pos0 + P.L - 1) / kChunk + 1);
+  const size_t hsm = sizeof(int32_t) * 2 * (size_t)nvis_max;
+  const unsigned nb = (unsigned)((ws.n_keys + kScanBlock - 1) / kScanBlock);
+  int2* rec = records ? ws.pinfo : nullptr;
+  if (nvis_max <= kHistMax) {
+    if ((e = set_smem(bucket_scatter_kernel, hsm)) != cudaSuccess) return e;
+    if ((e = set_smem(bucket_count_kernel, hsm)) != cudaSuccess) return e;
+    const dim3 bgrid((unsigned)((P.L + kBucketRows - 1) / kBucketRows), P.Hkv, P.B);
+    bucket_count_kernel<<<bgrid, 256, hsm / 2, s>>>(P, idx, ws.counts, W);
+    scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
+    scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
+                                          ws.offsets, ws.tile_off, ws.cursor, ws.items);
+    bucket_scatter_kernel<<<bgrid, 256, hsm, s>>>(P, idx, wts, ws.cursor, ws.pairs, rec, W);
+  } else {
+    const unsigned pb = (unsigned)((n_pairs + 255) / 256);
+    count_kernel<<<pb, 256, 0, s>>>(P, idx, ws.counts, n_pairs, W);
+    scan_totals_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals);
+    scan_kernel<<<nb, kScanBlock, 0, s>>>(ws.counts, ws.n_keys, tile_pairs, ws.scan_totals,
+                                          ws.offsets, ws.tile_off, ws.cursor, ws.items);
+    scatter_kernel<<<pb, 256, 0, s>>>(P, idx, wts, ws.cursor, ws.pairs, rec, n_pairs, W);
+  }
+  return cudaGetLastError();
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace carve-up; with base == nullptr only the size is computed.
+// Query windows of the bucket keys, unless the key space would grow past kMaxKeys.
+static void bucket_windows(const Params& P, int* n_win, int64_t* win_rows) {
+  *n_win = (int)((P.L + kBucketWindow - 1) / kBucketWindow);
+  *win_rows = kBucketWindow;
+  if ((int64_t)P.B * P.Hkv * *n_win * P.max_chunks > kMaxKeys) {
+    *n_win = 1;
+    *win_rows = P.L > 0 ? P.L : 1;
+  }
+}
+
 size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   const int64_t rows = (int64_t)P.B * P.L * P.Hq;
   const int64_t n_pairs = rows * P.k;
-  // query windows, unless the key space would grow past kMaxKeys
-  int n_win = (int)((P.L + kBucketWindow - 1) / kBucketWindow);
-  int64_t win_rows = kBucketWindow;
-  if ((int64_t)P.B * P.Hkv * n_win * P.max_chunks > kMaxKeys) {
-    n_win = 1;
-    win_rows = P.L > 0 ? P.L : 1;
-  }
+  int n_win;
+  int64_t win_rows;
+  bucket_windows(P, &n_win, &win_rows);
   const int64_t n_keys = (int64_t)P.B * P.Hkv * n_win * P.max_chunks;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -635,6 +638,36 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   w.items = (int4*)take(sizeof(int4) * w.max_tiles);
   w.scan_totals = (int2*)take(sizeof(int2) * ((n_keys + 1023) / 1024));
   if (ws) *ws = w;
+  return off;
+}
+
+size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base) {
+  const int64_t n_pairs = (int64_t)P.B * P.L * P.Hq * P.k;
+  int n_win;
+  int64_t win_rows;
+  bucket_windows(P, &n_win, &win_rows);
+  const int64_t n_keys = (int64_t)P.B * P.Hkv * n_win * P.max_chunks;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  PrefillWs w{};
+  w.counts = (int32_t*)take(sizeof(int32_t) * n_keys);
+  w.offsets = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
+  w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  w.n_keys = (int)n_keys;
+  w.n_win = n_win;
+  w.win_rows = win_rows;
+  w.max_tiles = (n_pairs + kBackwardTilePairs - 1) / kBackwardTilePairs + n_keys;
+  w.items = (int4*)take(sizeof(int4) * w.max_tiles);
+  w.scan_totals = (int2*)take(sizeof(int2) * ((n_keys + 1023) / 1024));
+  float* g = (float*)take(sizeof(float) * n_pairs);
+  if (ws) *ws = w;
+  if (dw) *dw = g;
   return off;
 }
 

@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libhils.so")
 
 HILS_F32, HILS_BF16 = 0, 1
-OP_SCORE, OP_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2, 3
+OP_SCORE, OP_TOPK, OP_PREFILL, OP_DECODE, OP_PREFILL_BACKWARD = 0, 1, 2, 3, 4
 STATUS = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
           3: "HILS_ERR_WORKSPACE", 4: "HILS_ERR_CUDA", 5: "HILS_ERR_TIMEOUT",
           6: "HILS_ERR_DEVICE_CHECK"}
@@ -28,7 +28,7 @@ EXPORTED = ("hils_workspace_size", "hils_score", "hils_topk", "hils_prefill", "h
             "hils_profile_collect", "hils_profile_read", "hils_profile_reset",
             "hils_decode_noalloc", "hils_decode_noalloc_capacity", "hils_set_wait_limit_ns",
             "hils_decode_cp_candidates", "hils_decode_cp_select", "hils_decode_cp_attend",
-            "hils_decode_cp_finish")
+            "hils_decode_cp_finish", "hils_prefill_backward")
 
 
 class HilsError(RuntimeError):
@@ -72,6 +72,9 @@ def load(path: str = LIB_PATH):
     L.hils_topk.argtypes = [cfgp, P, I64, I64, I32, P, P, P]
     L.hils_prefill.restype = ctypes.c_int
     L.hils_prefill.argtypes = [cfgp, P, I64, I64, P, P, cachep, P, P, P, P, ctypes.c_size_t, P]
+    L.hils_prefill_backward.restype = ctypes.c_int
+    L.hils_prefill_backward.argtypes = [cfgp, P, I64, I64, P, P, cachep, P, P, P, P, P, P, P, P,
+                                        P, ctypes.c_size_t, P]
     L.hils_decode.restype = ctypes.c_int
     L.hils_decode.argtypes = [cfgp, P, P, P, P, P, cachep, P, P, P, P, ctypes.c_size_t, P]
     L.hils_device_status.restype = ctypes.c_int
@@ -186,6 +189,17 @@ def prefill(cfg, q, q_len, q_pos0, A, B, cache: Cache, out, idx_out, w_out, ws, 
     _check(load().hils_prefill(ctypes.byref(cfg.c()), _ptr(q), q_len, q_pos0, _ptr(A), _ptr(B),
                                ctypes.byref(cache.c()), _ptr(out), _ptr(idx_out), _ptr(w_out),
                                _ptr(ws), ws_bytes, _stream(stream)), "hils_prefill")
+
+
+def prefill_backward(cfg, q, q_len, q_pos0, A, B, cache: Cache, idx, w, dout, dq, dpages, dlm,
+                     dA, dB, ws, ws_bytes, stream=None):
+    """Gradients of sum(dout * out) of hils_prefill with its selection (idx, w)
+    held fixed; dq, dpages, dlm, dA and dB are float32 and added into."""
+    _check(load().hils_prefill_backward(ctypes.byref(cfg.c()), _ptr(q), q_len, q_pos0, _ptr(A),
+                                        _ptr(B), ctypes.byref(cache.c()), _ptr(idx), _ptr(w),
+                                        _ptr(dout), _ptr(dq), _ptr(dpages), _ptr(dlm), _ptr(dA),
+                                        _ptr(dB), _ptr(ws), ws_bytes, _stream(stream)),
+           "hils_prefill_backward")
 
 
 def decode(cfg, q, k_new, v_new, A, B, cache: Cache, out, idx_out, w_out, ws, ws_bytes,

@@ -49,6 +49,7 @@ TID_KNEW = 7       # decode appended keys [steps][B][Hkv][d]
 TID_VNEW = 8       # decode appended values [steps][B][Hkv][d]
 TID_PERM = 9       # page permutation keys
 TID_NEEDLE = 10    # needle chunk positions
+TID_DOUT = 11      # output gradients of the prefill backward [B][L][Hq][d]
 
 DT_F32 = 0
 DT_BF16 = 1

@@ -53,7 +53,13 @@ typedef enum {
 
 typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
 
-typedef enum { HILS_OP_SCORE = 0, HILS_OP_TOPK = 1, HILS_OP_PREFILL = 2, HILS_OP_DECODE = 3 } hils_op;
+typedef enum {
+  HILS_OP_SCORE = 0,
+  HILS_OP_TOPK = 1,
+  HILS_OP_PREFILL = 2,
+  HILS_OP_DECODE = 3,
+  HILS_OP_PREFILL_BACKWARD = 4
+} hils_op;
 
 typedef struct {
   int32_t batch;       /* B: sequences */
@@ -110,6 +116,41 @@ int hils_topk(const hils_config* cfg, const float* scores, int64_t q_len, int64_
 int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
                  const float* A, const float* B, const hils_kv_cache* cache, void* out,
                  int32_t* idx_out, float* w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of hils_prefill with the chunk selection held fixed: the gradients
+ * of sum(dout * out) for training end to end under the language-modelling
+ * loss (the digest, 关键模块 item 1: the retrieval scores are differentiable
+ * and optimised by that loss, item 3: native sparse training; 输出与训练).
+ * The selection is a discrete choice and has no gradient; the fusion weights
+ * (through the landmark scores and the calibration), the per-chunk attention
+ * and the calibration do.  Per row, with the forward's notation:
+ *   dw_j = dout . O_j,  ds_j = w_j (dw_j - sum_l w_l dw_l),
+ *   dq~ = sum_j ds_j lm_j / sqrt(d),  dlm_j += ds_j q~ / sqrt(d),
+ *   per chunk with G = w_j dout: dV += P_j^T G, dS = P_j (G V_j^T - G . O_j),
+ *     dq += dS K_j / sqrt(d), dK += dS^T q / sqrt(d),
+ *   dq += dq~ + (dq~ B^T) A^T,  dA += q^T (dq~ B^T),  dB += (qA)^T dq~.
+ * q, q_len, q_pos0, A, B, cache  as given to hils_prefill (seq_lens not read).
+ * idx, w     int32 / float32 [B][q_len][Hq][k]: the forward's selection and
+ *            weights (hils_prefill's idx_out and w_out).
+ * dout       [B][q_len][Hq][d] in cfg->dtype, 16-byte aligned.
+ * dq         float32 [B][q_len][Hq][d].
+ * dpages     float32 [num_pages][2][Hkv][S][d], the gradient of the page pool
+ *            (same layout as cache->pages).
+ * dlandmarks float32 [B][max_chunks][Hkv][d].
+ * dA, dB     float32 [d][r], [r][d] (may be NULL when calib_rank == 0).
+ * All five gradients are ADDED INTO: zero them before the first call; a long
+ * prefill split into query blocks (q_pos0 > 0) then accumulates its blocks'
+ * gradients of the shared pages, landmarks, A and B.  The order of the float
+ * additions is not fixed, so results may differ in the last bits from run
+ * to run.  All arithmetic is float32.
+ * ws         at least hils_workspace_size(cfg, HILS_OP_PREFILL_BACKWARD, q_len,
+ *            max_chunks) bytes, 256-byte aligned; its contents need not be
+ *            initialised. */
+int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
+                          const float* A, const float* B, const hils_kv_cache* cache,
+                          const int32_t* idx, const float* w, const void* dout, float* dq,
+                          float* dpages, float* dlandmarks, float* dA, float* dB, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /* a8: one decode step for every sequence of the batch.
  * q             [B][Hq][d]: one query per sequence.

@@ -1,0 +1,109 @@
+"""hils_prefill_backward against the backward oracle (oracle/backward.py).
+
+The forward runs first on the GPU (hils_prefill); its selection idx, held
+fixed, goes to both the GPU backward and the oracle, which recomputes the
+weights and every other quantity in float64 from the stored inputs.  The
+GPU's five gradients (float32) must match the oracle's element by element:
+dq; the page pool's gradient, read back into logical K and V order through
+the block table (pages no sequence uses must stay zero); the landmarks'; A's
+and B's.  The tolerance is 1e-4 of each gradient's largest magnitude: the
+GPU computes in float32 throughout, on inputs that both sides read exactly."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import backward as ob
+from problem import random_problem
+import hils_inputs as hi
+
+pytestmark = pytest.mark.gpu
+BF16, F32 = hi.DT_BF16, hi.DT_F32
+REL = 1e-4
+
+
+def _gu():
+    import gpu_util
+    return gpu_util
+
+
+def _check(name, got, ref):
+    scale = float(np.max(np.abs(ref)))
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    if scale == 0.0:   # k = 1: the weight is constant, the score path gives exact zeros
+        assert err == 0.0, f"{name}: expected zeros, max abs {err}"
+        return 0.0
+    assert err <= REL * scale, f"{name}: max abs error {err} against scale {scale}"
+    return err / scale
+
+
+def _run(case, seed, repeat=1):
+    gu = _gu()
+    from chunk_sparse_long_b200 import hils
+    p = random_problem(chunk_size=64, spare_pages=3, seed=seed, calib_std=0.2, **case)
+    dp = gu.DevProblem(p)
+    _, idx, w = gu.run_prefill(dp)
+    B, L, Hq, d, k = p.batch, p.q_len, p.n_q_heads, p.head_dim, p.top_k
+    dout_st = hi.normal(seed, hi.TID_DOUT, 0, B * L * Hq * d, 1.0, p.dtype).reshape(B, L, Hq, d)
+    dout = gu.dev(dout_st)
+    dq = torch.zeros((B, L, Hq, d), dtype=torch.float32, device="cuda")
+    dpages = torch.zeros(p.pages.shape, dtype=torch.float32, device="cuda")
+    dlm = torch.zeros(p.landmarks.shape, dtype=torch.float32, device="cuda")
+    dA = torch.zeros(p.A.shape, dtype=torch.float32, device="cuda")
+    dB = torch.zeros(p.B.shape, dtype=torch.float32, device="cuda")
+    nbytes = hils.workspace_size(dp.cfg, hils.OP_PREFILL_BACKWARD, L, p.max_chunks)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ws.fill_(0xCD)                                   # the workspace needs no initialisation
+    for _ in range(repeat):
+        hils.prefill_backward(dp.cfg, dp.q, L, p.q_pos0, dp.A, dp.B, dp.cache, idx, w, dout, dq,
+                              dpages, dlm, dA, dB, ws, nbytes)
+    hils.device_status()
+    # the oracle, on the GPU's selection
+    q = ob.from_storage(p.q, p.dtype)
+    K, V = ob.from_storage(p.K, p.dtype), ob.from_storage(p.V, p.dtype)
+    lm = ob.from_storage(p.landmarks, p.dtype)
+    g = ob.backward(q, p.q_pos0, p.A.astype(np.float64), p.B.astype(np.float64), K, V, lm,
+                    idx.cpu().numpy().reshape(B, L, Hq, k), ob.from_storage(dout_st, p.dtype), 64)
+    g = {n: v * repeat for n, v in g.items()}
+    rep = {"dq": _check("dq", dq.cpu().numpy(), g["dq"])}
+    dpg = dpages.cpu().numpy()
+    T = p.q_pos0 + L
+    bt = p.block_table
+    dK = np.stack([[dpg[bt[b, u // 64], 0, :, u % 64] for u in range(T)] for b in range(B)])
+    dV = np.stack([[dpg[bt[b, u // 64], 1, :, u % 64] for u in range(T)] for b in range(B)])
+    rep["dK"] = _check("dK", dK, g["dK"][:, :T])
+    rep["dV"] = _check("dV", dV, g["dV"][:, :T])
+    used = np.zeros(dpg.shape[0], dtype=bool)
+    used[bt[:, : (T + 63) // 64].reshape(-1)] = True
+    assert not np.any(dpg[~used]), "gradient written into a page no sequence uses"
+    rep["dlm"] = _check("dlm", dlm.cpu().numpy(), g["dlm"])
+    if p.calib_rank > 0:
+        rep["dA"] = _check("dA", dA.cpu().numpy(), g["dA"])
+        rep["dB"] = _check("dB", dB.cpu().numpy(), g["dB"])
+    return rep
+
+
+CASES = {
+    "f32_d64": dict(batch=2, n_q_heads=4, n_kv_heads=4, head_dim=64, top_k=4, calib_rank=8,
+                    seq_len=700, dtype=F32),
+    "f32_d128_gqa_window": dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, top_k=6,
+                                calib_rank=16, seq_len=1000, q_pos0=300, dtype=F32),
+    "bf16_d128_gqa": dict(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, top_k=8,
+                          calib_rank=32, seq_len=1200, dtype=BF16),
+    "bf16_d64_k1": dict(batch=2, n_q_heads=2, n_kv_heads=1, head_dim=64, top_k=1, calib_rank=4,
+                        seq_len=300, dtype=BF16),
+    "bf16_d64_rank64_k32": dict(batch=1, n_q_heads=2, n_kv_heads=2, head_dim=64, top_k=32,
+                                calib_rank=64, seq_len=2100, dtype=BF16),
+    "f32_no_calibration": dict(batch=1, n_q_heads=2, n_kv_heads=2, head_dim=64, top_k=5,
+                               calib_rank=0, seq_len=650, dtype=F32),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_backward_matches_oracle(name):
+    rep = _run(CASES[name], seed=40 + sorted(CASES).index(name))
+    print(name, rep)
+
+
+def test_gradients_are_added_into():
+    rep = _run(CASES["f32_d64"], seed=77, repeat=2)
+    print(rep)

@@ -24,7 +24,9 @@
 //              sqrt(d), and through q~ = q + (qA)B: dq += dq~ + (dq~ B^T) A^T,
 //              dA += q^T (dq~ B^T), dB += (qA)^T dq~, the last two as products
 //              over groups of 32 rows, added once per CTA.
-// All arithmetic is float32 on CUDA cores.  Every gradient output is added
+// All arithmetic here is float32 on CUDA cores; for bf16 storage at
+// head_dim 128 the attention part runs on the tensor cores instead
+// (backward_tc.cu).  Every gradient output is added
 // into (the caller zeroes it first); the order of the float additions into
 // dq, the pool and the landmarks is not fixed.
 #include "hils_common.cuh"
@@ -367,9 +369,11 @@ cudaError_t run_backward(const Params& P, const int32_t* idx, const float* w, co
   // pair the bucketing rejected (its chunk out of range) reads as 0
   if ((e = cudaMemsetAsync(dw, 0, sizeof(float) * rows * P.k, s)) != cudaSuccess) return e;
   if ((e = launch_bucketing(P, idx, w, ws, false, kBackwardTilePairs, "backward.bucket", s)) != cudaSuccess) return e;
-  constexpr size_t asm_ = AttnSmem<D>::kBytes;
-  if ((e = set_smem(attn_bwd_kernel<D>, asm_)) != cudaSuccess) return e;
-  {
+  if (D == 128 && P.dtype == HILS_BF16) {
+    if ((e = launch_attn_bwd_tc(P, ws, w, dout, dq, dpages, dw, s)) != cudaSuccess) return e;
+  } else {
+    constexpr size_t asm_ = AttnSmem<D>::kBytes;
+    if ((e = set_smem(attn_bwd_kernel<D>, asm_)) != cudaSuccess) return e;
     HILS_PROFILE("backward.attention", s);
     attn_bwd_kernel<D><<<(unsigned)ws.max_tiles, kThreads, asm_, s>>>(P, ws, w, dout, dq, dpages,
                                                                       dw);

@@ -216,6 +216,7 @@ int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, 
   if (!dout || !aligned16(dout)) return fail(HILS_ERR_INVALID_ARG, "dout is NULL or misaligned");
   if (!dq || !dpages || !dlandmarks)
     return fail(HILS_ERR_INVALID_ARG, "dq, dpages and dlandmarks are required");
+  if (!aligned16(dq)) return fail(HILS_ERR_INVALID_ARG, "dq not 16-byte aligned");
   if (P.r > 0 && (!dA || !dB)) return fail(HILS_ERR_INVALID_ARG, "dA and dB are required when calib_rank > 0");
   P.q = q;
   P.L = q_len;

@@ -195,6 +195,10 @@ size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base)
 cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
                             float* dq, float* dpages, float* dlm, float* dA, float* dB,
                             const PrefillWs& ws, float* dw, cudaStream_t s);
+// The attention part of that backward on the tensor cores (bf16, head_dim 128).
+cudaError_t launch_attn_bwd_tc(const Params& P, const PrefillWs& ws, const float* w,
+                               const void* dout, float* dq, float* dpages, float* dw,
+                               cudaStream_t s);
 cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
                            const PrefillWs& ws, cudaStream_t s);
 cudaError_t launch_select_tc(const Params& P, const PrefillWs& ws, int32_t* idx, float* w,

@@ -433,6 +433,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, uint32
          ((M >> 4) << 24);
 }
 
+// The same with either operand's major-ness chosen: a_mn_major = 1 reads A
+// (M x K) with M contiguous, b_mn_major = 1 reads B (N x K) with N contiguous.
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(uint32_t M, uint32_t N, uint32_t a_mn_major,
+                                                     uint32_t b_mn_major) {
+  return idesc_bf16(M, N, b_mn_major) | (a_mn_major << 15);
+}
+
 // 2^x by the hardware approximation (MUFU), flushing denormal results to zero.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -133,7 +133,7 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
  * idx, w     int32 / float32 [B][q_len][Hq][k]: the forward's selection and
  *            weights (hils_prefill's idx_out and w_out).
  * dout       [B][q_len][Hq][d] in cfg->dtype, 16-byte aligned.
- * dq         float32 [B][q_len][Hq][d].
+ * dq         float32 [B][q_len][Hq][d], 16-byte aligned.
  * dpages     float32 [num_pages][2][Hkv][S][d], the gradient of the page pool
  *            (same layout as cache->pages).
  * dlandmarks float32 [B][max_chunks][Hkv][d].
@@ -142,7 +142,10 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
  * prefill split into query blocks (q_pos0 > 0) then accumulates its blocks'
  * gradients of the shared pages, landmarks, A and B.  The order of the float
  * additions is not fixed, so results may differ in the last bits from run
- * to run.  All arithmetic is float32.
+ * to run.  Arithmetic is float32, except that for bf16 storage at head_dim
+ * 128 the per-chunk attention products run on the tensor cores with bf16
+ * operands (the probabilities, G = w dout and dS rounded to bf16, as the
+ * forward rounds the probabilities) and float32 accumulation.
  * ws         at least hils_workspace_size(cfg, HILS_OP_PREFILL_BACKWARD, q_len,
  *            max_chunks) bytes, 256-byte aligned; its contents need not be
  *            initialised. */

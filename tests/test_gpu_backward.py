@@ -6,8 +6,12 @@ weights and every other quantity in float64 from the stored inputs.  The
 GPU's five gradients (float32) must match the oracle's element by element:
 dq; the page pool's gradient, read back into logical K and V order through
 the block table (pages no sequence uses must stay zero); the landmarks'; A's
-and B's.  The tolerance is 1e-4 of each gradient's largest magnitude: the
-GPU computes in float32 throughout, on inputs that both sides read exactly."""
+and B's.  The tolerance is 1e-4 of each gradient's largest magnitude where
+the GPU computes in float32 throughout (float32 storage, and head_dim 64),
+on inputs that both sides read exactly.  For bf16 storage at head_dim 128
+the attention products run on the tensor cores with P, G = w dout and dS
+rounded to bf16 (relative rounding error 2^-9 per element), and the bar is
+1e-2 of the largest magnitude."""
 import numpy as np
 import pytest
 import torch
@@ -18,7 +22,8 @@ import hils_inputs as hi
 
 pytestmark = pytest.mark.gpu
 BF16, F32 = hi.DT_BF16, hi.DT_F32
-REL = 1e-4
+REL_F32 = 1e-4
+REL_TC = 1e-2
 
 
 def _gu():
@@ -26,13 +31,13 @@ def _gu():
     return gpu_util
 
 
-def _check(name, got, ref):
+def _check(name, got, ref, rel):
     scale = float(np.max(np.abs(ref)))
     err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
     if scale == 0.0:   # k = 1: the weight is constant, the score path gives exact zeros
         assert err == 0.0, f"{name}: expected zeros, max abs {err}"
         return 0.0
-    assert err <= REL * scale, f"{name}: max abs error {err} against scale {scale}"
+    assert err <= rel * scale, f"{name}: max abs error {err} against scale {scale}"
     return err / scale
 
 
@@ -64,21 +69,22 @@ def _run(case, seed, repeat=1):
     g = ob.backward(q, p.q_pos0, p.A.astype(np.float64), p.B.astype(np.float64), K, V, lm,
                     idx.cpu().numpy().reshape(B, L, Hq, k), ob.from_storage(dout_st, p.dtype), 64)
     g = {n: v * repeat for n, v in g.items()}
-    rep = {"dq": _check("dq", dq.cpu().numpy(), g["dq"])}
+    rel = REL_TC if (p.dtype == BF16 and d == 128) else REL_F32
+    rep = {"dq": _check("dq", dq.cpu().numpy(), g["dq"], rel)}
     dpg = dpages.cpu().numpy()
     T = p.q_pos0 + L
     bt = p.block_table
     dK = np.stack([[dpg[bt[b, u // 64], 0, :, u % 64] for u in range(T)] for b in range(B)])
     dV = np.stack([[dpg[bt[b, u // 64], 1, :, u % 64] for u in range(T)] for b in range(B)])
-    rep["dK"] = _check("dK", dK, g["dK"][:, :T])
-    rep["dV"] = _check("dV", dV, g["dV"][:, :T])
+    rep["dK"] = _check("dK", dK, g["dK"][:, :T], rel)
+    rep["dV"] = _check("dV", dV, g["dV"][:, :T], rel)
     used = np.zeros(dpg.shape[0], dtype=bool)
     used[bt[:, : (T + 63) // 64].reshape(-1)] = True
     assert not np.any(dpg[~used]), "gradient written into a page no sequence uses"
-    rep["dlm"] = _check("dlm", dlm.cpu().numpy(), g["dlm"])
+    rep["dlm"] = _check("dlm", dlm.cpu().numpy(), g["dlm"], rel)
     if p.calib_rank > 0:
-        rep["dA"] = _check("dA", dA.cpu().numpy(), g["dA"])
-        rep["dB"] = _check("dB", dB.cpu().numpy(), g["dB"])
+        rep["dA"] = _check("dA", dA.cpu().numpy(), g["dA"], rel)
+        rep["dB"] = _check("dB", dB.cpu().numpy(), g["dB"], rel)
     return rep
 
 

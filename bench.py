@@ -38,6 +38,10 @@ import hils_inputs as hi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_KERNELS_PER_STEP = 7   # calib, score+select, bucket count, scan totals, scan, scatter, attend + merge (bf16)
+# backward: bucket count, scan totals, scan, scatter; then the tensor-core path's
+# delta, lm', attention, item sums, M sum, dA/dB, or the CUDA-core attention and scores
+BACKWARD_KERNELS_TC = 10
+BACKWARD_KERNELS_SIMT = 6
 # decode: one cooperative kernel per step when every CTA fits on the GPU at once,
 # else scan + attend; counted from the profiled eager steps (decode_report)
 
@@ -390,6 +394,97 @@ def prefill_report(w: hi.Workload, ms: float, phases: dict, steps: int, n_ranks:
     }
 
 
+def time_backward(hils, torch, wl, steps, warmup, barrier, maxreduce):
+    """hils_prefill_backward on the workload.  The forward runs once first: its
+    output and its selection (idx, w) are inputs of the backward, with a seeded
+    N(0,1) dout.  Each timed step adds the gradients into the same float32
+    buffers (the work does not depend on their contents)."""
+    w = wl["workload"]
+    cfg = cfg_of(hils, w)
+    cache = make_cache(hils, wl)
+    L, B, Hq, d, k = w.seq_len, w.batch, w.n_q_heads, w.head_dim, w.top_k
+    dt = torch.bfloat16 if w.dtype == hi.DT_BF16 else torch.float32
+    out = torch.empty((B, L, Hq, d), dtype=dt, device="cuda")
+    idx = torch.empty((B * L * Hq, k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((B * L * Hq, k), dtype=torch.float32, device="cuda")
+    nf = hils.workspace_size(cfg, hils.OP_PREFILL, L, wl["max_chunks"])
+    wsf = torch.empty(nf, dtype=torch.uint8, device="cuda")
+    hils.prefill(cfg, wl["q"], L, 0, wl["A"], wl["B"], cache, out, idx, wt, wsf, nf)
+    torch.cuda.synchronize()
+    del wsf
+    torch.cuda.empty_cache()
+    dout = torch.empty_like(out)
+    hi.normal_device(dout, w.seed, hi.TID_DOUT)
+    dq = torch.zeros((B, L, Hq, d), dtype=torch.float32, device="cuda")
+    dpages = torch.zeros(wl["pages"].shape, dtype=torch.float32, device="cuda")
+    dlm = torch.zeros(wl["landmarks"].shape, dtype=torch.float32, device="cuda")
+    dA = torch.zeros((d, w.calib_rank), dtype=torch.float32, device="cuda")
+    dB = torch.zeros((w.calib_rank, d), dtype=torch.float32, device="cuda")
+    nb = hils.workspace_size(cfg, hils.OP_PREFILL_BACKWARD, L, wl["max_chunks"])
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hils.prefill_backward(cfg, wl["q"], L, 0, wl["A"], wl["B"], cache, idx, wt, out, dout, dq,
+                              dpages, dlm, dA, dB, ws, nb, stream)
+
+    for _ in range(warmup):
+        step()
+    hils.device_status(stream)
+    hils.profile_reset()
+    hils.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    hils.profile_enable(False)
+    phases = hils.profile_read()
+    hils.device_status(stream)
+    return maxreduce(e0.elapsed_time(e1)) / steps, phases, clk.summary(), nb
+
+
+def backward_report(w: hi.Workload, ms: float, phases: dict, steps: int, n_ranks: int,
+                    clocks: dict, ws_bytes: int) -> dict:
+    """Throughput and roofline of a timed backward run.  Algorithmic work: the
+    six products per (row, chunk) pair over the keys visible to the row (the
+    forward's QK^T and PV, recomputed, and dP, dQ, dK, dV), three times the
+    forward's useful attention flop.  The roofline is that of the attention
+    kernel against the measured dense bf16 peak (tensor-core path), or
+    float32 CUDA cores (no tensor-core roofline)."""
+    pk, pk_src = peaks()
+    counts = prefill_counts(w)
+    work = 3 * counts["attention_flop"]
+    name = "backward.attention"
+    tot, n = phases.get(name, (0.0, 0))
+    att_ms = tot / max(1, n)
+    tc = w.dtype == hi.DT_BF16 and w.head_dim == 128
+    at_max = bool(clocks.get("sm_mhz")) and clocks.get("sm_max_mhz") and \
+        clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"]
+    peak = pk["bf16_tflops"] if at_max else pk["bf16_tflops_sustained"]
+    achieved = work / (att_ms / 1e3) / 1e12 if att_ms > 0 else None
+    return {
+        "workload": w.name, "ms_per_step": ms, "steps": steps,
+        "tok_per_s": weak_scaling_value(w.batch * w.seq_len, n_ranks, ms),
+        "kernels_ms_per_step": {k: v[0] / max(1, steps) for k, v in phases.items()},
+        "gpu_launches": (BACKWARD_KERNELS_TC if tc else BACKWARD_KERNELS_SIMT) * steps,
+        "workspace_bytes": ws_bytes, "clocks": clocks,
+        "roofline": {"bound": "tensor" if tc else "alu", "kernel": name,
+                     "achieved": achieved, "peak": peak if tc else None, "unit": "TFLOP/s",
+                     "frac": achieved / peak if (tc and achieved) else None, "traffic": None,
+                     "work_per_launch": work,
+                     "work": "useful flop of the six per-pair products over visible keys "
+                             "(3x the forward's attention flop)",
+                     "peak_source": (f"{pk_src} bf16 " + ("burst" if at_max else "sustained"))
+                     if tc else "float32 CUDA-core path: no tensor-core roofline"},
+    }
+
+
 def decode_report(dw: hi.Workload, times: list, phases: dict, n_ranks: int, maxreduce) -> dict:
     """Step time and HBM roofline of a timed decode run: the step's algorithmic
     bytes (every visible landmark, the selected K/V, q, out and the appended
@@ -540,6 +635,8 @@ def main():
                     help="time only the headline prefill and decode workloads")
     ap.add_argument("--config-decode-steps", type=int, default=64,
                     help="timed decode steps of the B=32 and 4M decode workloads")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward (hils_prefill_backward) lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     args = ap.parse_args()
@@ -622,6 +719,10 @@ def main():
         result["e2e"] = {"value": weak_scaling_value(tokens_per_rank, nworld, e2e_ms), "unit": "tok/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                          "steps": args.steps}
+    if not args.no_backward:
+        bms, bph, bclk, bws = time_backward(hils, torch, wl, args.steps, args.warmup, barrier,
+                                            maxreduce)
+        result["backward"] = backward_report(w, bms, bph, args.steps, nworld, bclk, bws)
     del wl
     torch.cuda.empty_cache()
     configs = {}
@@ -641,7 +742,13 @@ def main():
                                                 barrier, maxreduce)
             configs[name] = prefill_report(pw, pms, pph, max(args.steps, 20), nworld, pclk)
             configs[name]["clocks"] = pclk
-            del keep, pwl
+            del keep
+            if not args.no_backward and name == "prefill_8k":
+                bms, bph, bclk, bws = time_backward(hils, torch, pwl, max(args.steps, 20),
+                                                    args.warmup, barrier, maxreduce)
+                configs[name]["backward"] = backward_report(pw, bms, bph, max(args.steps, 20),
+                                                            nworld, bclk, bws)
+            del pwl
             torch.cuda.empty_cache()
         for name, n in (("decode_128k_b32", args.config_decode_steps),
                         ("decode_4m", args.config_decode_steps)):

@@ -24,9 +24,10 @@
 //              sqrt(d), and through q~ = q + (qA)B: dq += dq~ + (dq~ B^T) A^T,
 //              dA += q^T (dq~ B^T), dB += (qA)^T dq~, the last two as products
 //              over groups of 32 rows, added once per CTA.
-// All arithmetic here is float32 on CUDA cores; for bf16 storage at
-// head_dim 128 the attention part runs on the tensor cores instead
-// (backward_tc.cu).  Every gradient output is added
+// All arithmetic here is float32 on CUDA cores.  For bf16 storage at
+// head_dim 128, backward_tc.cu takes the whole backward instead (tensor-core
+// attention, and the score path folded into per-item sums).  Every gradient
+// output is added
 // into (the caller zeroes it first); the order of the float additions into
 // dq, the pool and the landmarks is not fixed.
 #include "hils_common.cuh"
@@ -362,21 +363,21 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(Params P, const int
 template <int D>
 cudaError_t run_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
                          float* dq, float* dpages, float* dlm, float* dA, float* dB,
-                         const PrefillWs& ws, float* dw, cudaStream_t s) {
+                         const BackwardWs& ws, cudaStream_t s) {
   const int64_t rows = (int64_t)P.B * P.L * P.Hq;
   cudaError_t e;
   // every pair's dw is written by the attention pass; zero first, so that a
   // pair the bucketing rejected (its chunk out of range) reads as 0
-  if ((e = cudaMemsetAsync(dw, 0, sizeof(float) * rows * P.k, s)) != cudaSuccess) return e;
-  if ((e = launch_bucketing(P, idx, w, ws, false, kBackwardTilePairs, "backward.bucket", s)) != cudaSuccess) return e;
-  if (D == 128 && P.dtype == HILS_BF16) {
-    if ((e = launch_attn_bwd_tc(P, ws, w, dout, dq, dpages, dw, s)) != cudaSuccess) return e;
-  } else {
-    constexpr size_t asm_ = AttnSmem<D>::kBytes;
-    if ((e = set_smem(attn_bwd_kernel<D>, asm_)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ws.dw, 0, sizeof(float) * rows * P.k, s)) != cudaSuccess) return e;
+  if ((e = launch_bucketing(P, idx, w, ws.bk, false, kBackwardTilePairs, "backward.bucket", s)) !=
+      cudaSuccess)
+    return e;
+  constexpr size_t asm_ = AttnSmem<D>::kBytes;
+  if ((e = set_smem(attn_bwd_kernel<D>, asm_)) != cudaSuccess) return e;
+  {
     HILS_PROFILE("backward.attention", s);
-    attn_bwd_kernel<D><<<(unsigned)ws.max_tiles, kThreads, asm_, s>>>(P, ws, w, dout, dq, dpages,
-                                                                      dw);
+    attn_bwd_kernel<D><<<(unsigned)ws.bk.max_tiles, kThreads, asm_, s>>>(P, ws.bk, w, dout, dq,
+                                                                         dpages, ws.dw);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t ssm = score_bwd_smem<D>(P.r);
@@ -385,19 +386,25 @@ cudaError_t run_backward(const Params& P, const int32_t* idx, const float* w, co
   const unsigned nb = (unsigned)(n_groups < 2 * 148 ? n_groups : 2 * 148);
   {
     HILS_PROFILE("backward.scores", s);
-    score_bwd_kernel<D><<<nb, kThreads, ssm, s>>>(P, idx, w, dw, dq, dlm, dA, dB);
+    score_bwd_kernel<D><<<nb, kThreads, ssm, s>>>(P, idx, w, ws.dw, dq, dlm, dA, dB);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
-                            float* dq, float* dpages, float* dlm, float* dA, float* dB,
-                            const PrefillWs& ws, float* dw, cudaStream_t s) {
+cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* out,
+                            const void* dout, float* dq, float* dpages, float* dlm, float* dA,
+                            float* dB, const BackwardWs& ws, cudaStream_t s) {
   if (P.L == 0 || P.B == 0) return cudaSuccess;
-  return P.d == 64 ? run_backward<64>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, dw, s)
-                   : run_backward<128>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, dw, s);
+  if (backward_on_tc(P)) {
+    cudaError_t e =
+        launch_bucketing(P, idx, w, ws.bk, false, kBackwardTilePairs, "backward.bucket", s);
+    if (e != cudaSuccess) return e;
+    return launch_backward_tc(P, idx, w, out, dout, dq, dpages, dlm, dA, dB, ws, s);
+  }
+  return P.d == 64 ? run_backward<64>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, s)
+                   : run_backward<128>(P, idx, w, dout, dq, dpages, dlm, dA, dB, ws, s);
 }
 
 }  // namespace hils

@@ -136,7 +136,7 @@ size_t hils_workspace_size(const hils_config* cfg, int op, int64_t q_len, int32_
     case HILS_OP_DECODE:
       return hils::decode_ws_bytes(P, nullptr, nullptr);
     case HILS_OP_PREFILL_BACKWARD:
-      return hils::backward_ws_bytes(P, nullptr, nullptr, nullptr);
+      return hils::backward_ws_bytes(P, nullptr, nullptr);
     default:
       fail(HILS_ERR_INVALID_ARG, "unknown op %d", op);
       return 0;
@@ -203,9 +203,9 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
 
 int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
                           const float* A, const float* B, const hils_kv_cache* cache,
-                          const int32_t* idx, const float* w, const void* dout, float* dq,
-                          float* dpages, float* dlandmarks, float* dA, float* dB, void* ws,
-                          size_t ws_bytes, void* stream) {
+                          const int32_t* idx, const float* w, const void* out,
+                          const void* dout, float* dq, float* dpages, float* dlandmarks,
+                          float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
   hils::Params P{};
   int st;
   if ((st = check_config(cfg, &P)) || (st = check_calib(cfg, A, B, &P)) ||
@@ -214,6 +214,7 @@ int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, 
   if ((st = check_queries(q, q_len, q_pos0, P, cache->max_chunks))) return st;
   if (!idx || !w) return fail(HILS_ERR_INVALID_ARG, "idx and w (the forward's selection) are required");
   if (!dout || !aligned16(dout)) return fail(HILS_ERR_INVALID_ARG, "dout is NULL or misaligned");
+  if (!out || !aligned16(out)) return fail(HILS_ERR_INVALID_ARG, "out is NULL or misaligned");
   if (!dq || !dpages || !dlandmarks)
     return fail(HILS_ERR_INVALID_ARG, "dq, dpages and dlandmarks are required");
   if (!aligned16(dq)) return fail(HILS_ERR_INVALID_ARG, "dq not 16-byte aligned");
@@ -221,16 +222,15 @@ int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, 
   P.q = q;
   P.L = q_len;
   P.pos0 = q_pos0;
-  hils::PrefillWs w_ws{};
-  float* dw = nullptr;
-  const size_t need = hils::backward_ws_bytes(P, &w_ws, &dw, nullptr);
+  hils::BackwardWs w_ws{};
+  const size_t need = hils::backward_ws_bytes(P, &w_ws, nullptr);
   if (!ws || ws_bytes < need)
     return fail(HILS_ERR_WORKSPACE, "prefill backward needs %zu workspace bytes, got %zu", need,
                 ws_bytes);
   if (((uintptr_t)ws & 255u) != 0) return fail(HILS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  hils::backward_ws_bytes(P, &w_ws, &dw, (char*)ws);
-  cudaError_t e = hils::launch_backward(P, idx, w, dout, dq, dpages, dlandmarks, dA, dB, w_ws, dw,
-                                        (cudaStream_t)stream);
+  hils::backward_ws_bytes(P, &w_ws, (char*)ws);
+  cudaError_t e = hils::launch_backward(P, idx, w, out, dout, dq, dpages, dlandmarks, dA, dB,
+                                        w_ws, (cudaStream_t)stream);
   return e == cudaSuccess ? HILS_OK : cuda_fail(e, "hils_prefill_backward");
 }
 

@@ -187,17 +187,28 @@ cudaError_t launch_bucketing(const Params& P, const int32_t* idx, const float* w
                              const PrefillWs& ws, bool records, int tile_pairs, const char* label,
                              cudaStream_t s);
 
-// Prefill backward with the selection fixed (hils_prefill_backward): the
-// bucketing arrays of ws (pair ids, tiles of kBackwardTilePairs) and dw, one
-// float per pair.  With base == nullptr only the size is computed.
+// Prefill backward with the selection fixed (hils_prefill_backward).
 constexpr int kBackwardTilePairs = 128;
-size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base);
-cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* dout,
-                            float* dq, float* dpages, float* dlm, float* dA, float* dB,
-                            const PrefillWs& ws, float* dw, cudaStream_t s);
-// The attention part of that backward on the tensor cores (bf16, head_dim 128).
-cudaError_t launch_attn_bwd_tc(const Params& P, const PrefillWs& ws, const float* w,
-                               const void* dout, float* dq, float* dpages, float* dw,
+constexpr int kBackwardMaxCtas = 160;   // per-CTA partial sums of the tensor-core path
+// True where the attention part runs on the tensor cores (bf16, head_dim 128).
+inline bool backward_on_tc(const Params& P) { return P.dtype == HILS_BF16 && P.d == 128; }
+struct BackwardWs {
+  PrefillWs bk;     // bucketing: pair ids in key order, items of kBackwardTilePairs pairs
+  float* dw;        // CUDA-core path: [rows * k] dout . O_j per pair
+  float* delta;     // tensor-core path: [rows] dout . out per row
+  float* lmc;       // tensor-core path: [B][max_chunks][Hkv][d] lm + (lm B^T) A^T
+  float* vchunk;    // tensor-core path: [B][max_chunks][Hkv][d] sum over chunk j's pairs of ds q
+  float* mpart;     // tensor-core path: [kBackwardMaxCtas + 1][d][d] per-CTA sums of v lm^T
+};
+// Workspace carve-up; with base == nullptr only the size is computed.
+size_t backward_ws_bytes(const Params& P, BackwardWs* ws, char* base);
+cudaError_t launch_backward(const Params& P, const int32_t* idx, const float* w, const void* out,
+                            const void* dout, float* dq, float* dpages, float* dlm, float* dA,
+                            float* dB, const BackwardWs& ws, cudaStream_t s);
+// The tensor-core path after the bucketing: everything but the bucketing.
+cudaError_t launch_backward_tc(const Params& P, const int32_t* idx, const float* w,
+                               const void* out, const void* dout, float* dq, float* dpages,
+                               float* dlm, float* dA, float* dB, const BackwardWs& ws,
                                cudaStream_t s);
 cudaError_t launch_prefill(const Params& P, void* out, int32_t* idx_out, float* w_out,
                            const PrefillWs& ws, cudaStream_t s);

@@ -641,8 +641,9 @@ size_t prefill_ws_bytes(const Params& P, PrefillWs* ws, char* base) {
   return off;
 }
 
-size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base) {
-  const int64_t n_pairs = (int64_t)P.B * P.L * P.Hq * P.k;
+size_t backward_ws_bytes(const Params& P, BackwardWs* ws, char* base) {
+  const int64_t rows = (int64_t)P.B * P.L * P.Hq;
+  const int64_t n_pairs = rows * P.k;
   int n_win;
   int64_t win_rows;
   bucket_windows(P, &n_win, &win_rows);
@@ -653,21 +654,28 @@ size_t backward_ws_bytes(const Params& P, PrefillWs* ws, float** dw, char* base)
     off += align256(bytes);
     return p;
   };
-  PrefillWs w{};
-  w.counts = (int32_t*)take(sizeof(int32_t) * n_keys);
-  w.offsets = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
-  w.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
-  w.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
-  w.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
-  w.n_keys = (int)n_keys;
-  w.n_win = n_win;
-  w.win_rows = win_rows;
-  w.max_tiles = (n_pairs + kBackwardTilePairs - 1) / kBackwardTilePairs + n_keys;
-  w.items = (int4*)take(sizeof(int4) * w.max_tiles);
-  w.scan_totals = (int2*)take(sizeof(int2) * ((n_keys + 1023) / 1024));
-  float* g = (float*)take(sizeof(float) * n_pairs);
+  BackwardWs w{};
+  PrefillWs& k = w.bk;
+  k.counts = (int32_t*)take(sizeof(int32_t) * n_keys);
+  k.offsets = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  k.tile_off = (int32_t*)take(sizeof(int32_t) * (n_keys + 1));
+  k.cursor = (int32_t*)take(sizeof(int32_t) * n_keys);
+  k.pairs = (int32_t*)take(sizeof(int32_t) * n_pairs);
+  k.n_keys = (int)n_keys;
+  k.n_win = n_win;
+  k.win_rows = win_rows;
+  k.max_tiles = (n_pairs + kBackwardTilePairs - 1) / kBackwardTilePairs + n_keys;
+  k.items = (int4*)take(sizeof(int4) * k.max_tiles);
+  k.scan_totals = (int2*)take(sizeof(int2) * ((n_keys + 1023) / 1024));
+  if (backward_on_tc(P)) {
+    w.delta = (float*)take(sizeof(float) * rows);
+    w.lmc = (float*)take(sizeof(float) * (size_t)P.B * P.max_chunks * P.Hkv * P.d);
+    w.vchunk = (float*)take(sizeof(float) * (size_t)P.B * P.max_chunks * P.Hkv * P.d);
+    w.mpart = (float*)take(sizeof(float) * (size_t)(kBackwardMaxCtas + 1) * P.d * P.d);
+  } else {
+    w.dw = (float*)take(sizeof(float) * n_pairs);
+  }
   if (ws) *ws = w;
-  if (dw) *dw = g;
   return off;
 }
 

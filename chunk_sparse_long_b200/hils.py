@@ -74,7 +74,7 @@ def load(path: str = LIB_PATH):
     L.hils_prefill.argtypes = [cfgp, P, I64, I64, P, P, cachep, P, P, P, P, ctypes.c_size_t, P]
     L.hils_prefill_backward.restype = ctypes.c_int
     L.hils_prefill_backward.argtypes = [cfgp, P, I64, I64, P, P, cachep, P, P, P, P, P, P, P, P,
-                                        P, ctypes.c_size_t, P]
+                                        P, P, ctypes.c_size_t, P]
     L.hils_decode.restype = ctypes.c_int
     L.hils_decode.argtypes = [cfgp, P, P, P, P, P, cachep, P, P, P, P, ctypes.c_size_t, P]
     L.hils_device_status.restype = ctypes.c_int
@@ -191,14 +191,15 @@ def prefill(cfg, q, q_len, q_pos0, A, B, cache: Cache, out, idx_out, w_out, ws, 
                                _ptr(ws), ws_bytes, _stream(stream)), "hils_prefill")
 
 
-def prefill_backward(cfg, q, q_len, q_pos0, A, B, cache: Cache, idx, w, dout, dq, dpages, dlm,
-                     dA, dB, ws, ws_bytes, stream=None):
-    """Gradients of sum(dout * out) of hils_prefill with its selection (idx, w)
-    held fixed; dq, dpages, dlm, dA and dB are float32 and added into."""
+def prefill_backward(cfg, q, q_len, q_pos0, A, B, cache: Cache, idx, w, out, dout, dq, dpages,
+                     dlm, dA, dB, ws, ws_bytes, stream=None):
+    """Gradients of sum(dout * out) of hils_prefill (its output `out`, its
+    selection idx and w held fixed); dq, dpages, dlm, dA and dB are float32
+    and added into."""
     _check(load().hils_prefill_backward(ctypes.byref(cfg.c()), _ptr(q), q_len, q_pos0, _ptr(A),
                                         _ptr(B), ctypes.byref(cache.c()), _ptr(idx), _ptr(w),
-                                        _ptr(dout), _ptr(dq), _ptr(dpages), _ptr(dlm), _ptr(dA),
-                                        _ptr(dB), _ptr(ws), ws_bytes, _stream(stream)),
+                                        _ptr(out), _ptr(dout), _ptr(dq), _ptr(dpages), _ptr(dlm),
+                                        _ptr(dA), _ptr(dB), _ptr(ws), ws_bytes, _stream(stream)),
            "hils_prefill_backward")
 
 

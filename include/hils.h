@@ -132,6 +132,10 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
  * q, q_len, q_pos0, A, B, cache  as given to hils_prefill (seq_lens not read).
  * idx, w     int32 / float32 [B][q_len][Hq][k]: the forward's selection and
  *            weights (hils_prefill's idx_out and w_out).
+ * out        [B][q_len][Hq][d] in cfg->dtype, 16-byte aligned: the forward's
+ *            output for the same inputs.  sum_l w_l dw_l = dout . out, so the
+ *            bf16 head_dim-128 path takes that row term from it before the
+ *            attention pass; the other configurations sum the dw_l instead.
  * dout       [B][q_len][Hq][d] in cfg->dtype, 16-byte aligned.
  * dq         float32 [B][q_len][Hq][d], 16-byte aligned.
  * dpages     float32 [num_pages][2][Hkv][S][d], the gradient of the page pool
@@ -151,9 +155,9 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
  *            initialised. */
 int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
                           const float* A, const float* B, const hils_kv_cache* cache,
-                          const int32_t* idx, const float* w, const void* dout, float* dq,
-                          float* dpages, float* dlandmarks, float* dA, float* dB, void* ws,
-                          size_t ws_bytes, void* stream);
+                          const int32_t* idx, const float* w, const void* out,
+                          const void* dout, float* dq, float* dpages, float* dlandmarks,
+                          float* dA, float* dB, void* ws, size_t ws_bytes, void* stream);
 
 /* a8: one decode step for every sequence of the batch.
  * q             [B][Hq][d]: one query per sequence.

@@ -53,7 +53,10 @@ struct TLay {
   static constexpr uint32_t kV = kK + kKVB;
   static constexpr uint32_t kP = kV + kKVB;
   static constexpr uint32_t kS = kP + kPB;          // dS, then one more block whose
-  static constexpr uint32_t kBytes = kS + 2 * kPB;   // column 0 holds ds: 144 KB
+                                                     // column 0 holds ds
+  static constexpr uint32_t kStage = kS + 2 * kPB;   // per warp 32 rows x 32 floats of dQ
+  static constexpr uint32_t kStageLd = 36;           // floats per staged row (16-byte rows)
+  static constexpr uint32_t kBytes = kStage + 4 * 32 * kStageLd * 4;   // 162 KB
 };
 // TMEM columns: S / dP, O / dQ (per item); dK^T with v in its column 64, and
 // dV^T (summed over a run of items of one key)
@@ -86,6 +89,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   __shared__ uint32_t tmem_sh;
   __shared__ float slm[kD];        // the item's lm'_j
   __shared__ float sds[kRowsT];    // ds of every tile row (0 past the item's pairs)
+  __shared__ int32_t srow[kRowsT]; // query row of every tile row (-1 past the item's pairs)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t sb = tc::smem_u32(smem);
@@ -108,272 +112,282 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   constexpr uint32_t kIdT = tc::idesc_bf16_ab(kD, kChunk, 1, 1);      // M = d, N = 64, both MN-major
   constexpr uint32_t kIdTV = tc::idesc_bf16_ab(kD, kChunk + 16, 1, 1); // the same with N = 80
   const float sc = P.inv_sqrt_d;
-  // this CTA's contiguous range of items: the items of one key follow one
-  // another, so dK^T, dV^T and v add up in tensor memory over a key's run and
+  // keys go round-robin over the CTAs, so the CTAs at work share a query
+  // window, whose q, dout and dq rows stay in L2; a key's items are taken in
+  // turn, so dK^T, dV^T and v add up in tensor memory over the key's run and
   // go out once at its end
-  const int n_items = ws.tile_off[ws.n_keys];
-  const int per = (n_items + (int)gridDim.x - 1) / (int)gridDim.x;
-  const int it0 = (int)blockIdx.x * per;
-  const int it1 = it0 + per < n_items ? it0 + per : n_items;
   uint32_t phase = 0;
   bool ok = true;
-  for (int it = it0; ok && it < it1; ++it) {
-    const int4 item = ws.items[it];
-    const int key = item.x;
-    const bool run_first = it == it0 || ws.items[it - 1].x != key;
-    const bool run_last = it == it1 - 1 || ws.items[it + 1].x != key;
+  for (int key = blockIdx.x; ok && key < ws.n_keys; key += gridDim.x) {
+    const int t0 = ws.tile_off[key], t1 = ws.tile_off[key + 1];
+    if (t0 == t1) continue;
     const int j = key % P.max_chunks;
     const int bg = key / P.max_chunks / ws.n_win;
     const int g = bg % P.Hkv, b = bg / P.Hkv;
     const int64_t page = page_of(P, b, j);
     if (page < 0) continue;   // the same for every thread of the CTA
-    const int n = item.z - item.y;
-    const int row = tid;
-    const bool live = row < n;
-    int32_t pid = 0;
-    int64_t r = 0;
-    int nk = 0;
-    float wj = 0.f, dl = 0.f;
-    if (live) {
-      pid = ws.pairs[item.y + row];
-      r = pid / P.k;
-      const int64_t pos = P.pos0 + (r / P.Hq) % P.L;
-      nk = pos / kChunk == j ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
-      wj = __ldg(wts + pid);
-      dl = __ldg(delta + r);
-    }
-    slm[tid] = __ldg(lmc + (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * kD + tid);
-    // ---- the pair's q row into Q (zeros past the item's pairs), K and V
-    {
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(P.q) + r * (kD * 2);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        tc::cp_async16(sb + TLay::kQ + tile_at(kRowsT, row, c), src + c * 16, live ? 16u : 0u);
-      const uint8_t* kp =
-          reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 0, g, 0) * 2;
-      const uint8_t* vp =
-          reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 1, g, 0) * 2;
-      for (int x = tid; x < kChunk * 16; x += kThreadsT) {
-        const int kr = x >> 4, c = x & 15;
-        tc::cp_async16(sb + TLay::kK + tile_at(kChunk, kr, c), kp + kr * (kD * 2) + c * 16, 16u);
-        tc::cp_async16(sb + TLay::kV + tile_at(kChunk, kr, c), vp + kr * (kD * 2) + c * 16, 16u);
+    for (int it = t0; it < t1; ++it) {
+      const int4 item = ws.items[it];
+      const bool run_first = it == t0;
+      const bool run_last = it == t1 - 1;
+      const int n = item.z - item.y;
+      const int row = tid;
+      const bool live = row < n;
+      int32_t pid = 0;
+      int64_t r = 0;
+      int nk = 0;
+      float wj = 0.f, dl = 0.f;
+      if (live) {
+        pid = ws.pairs[item.y + row];
+        r = pid / P.k;
+        const int64_t pos = P.pos0 + (r / P.Hq) % P.L;
+        nk = pos / kChunk == j ? (int)(pos - (int64_t)j * kChunk + 1) : kChunk;
+        wj = __ldg(wts + pid);
+        dl = __ldg(delta + r);
       }
-      tc::cp_async_commit();
-      tc::cp_async_wait<0>();
+      slm[tid] = __ldg(lmc + (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * kD + tid);
+      // ---- the pair's q row into Q (zeros past the item's pairs), K and V
+      {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.q) + r * (kD * 2);
+  #pragma unroll
+        for (int c = 0; c < 16; ++c)
+          tc::cp_async16(sb + TLay::kQ + tile_at(kRowsT, row, c), src + c * 16, live ? 16u : 0u);
+        const uint8_t* kp =
+            reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 0, g, 0) * 2;
+        const uint8_t* vp =
+            reinterpret_cast<const uint8_t*>(P.pages) + page_offset(P, page, 1, g, 0) * 2;
+        for (int x = tid; x < kChunk * 16; x += kThreadsT) {
+          const int kr = x >> 4, c = x & 15;
+          tc::cp_async16(sb + TLay::kK + tile_at(kChunk, kr, c), kp + kr * (kD * 2) + c * 16, 16u);
+          tc::cp_async16(sb + TLay::kV + tile_at(kChunk, kr, c), vp + kr * (kD * 2) + c * 16, 16u);
+        }
+        tc::cp_async_commit();
+        tc::cp_async_wait<0>();
+        tc::fence_proxy_async();
+      }
+      __syncthreads();
+      // ---- S = Q K^T
+      if (tid == 0) {
+        tc::tc_fence_after();
+  #pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t a =
+              tc::smem_desc(sb + TLay::kQ + (kk >> 2) * (kRowsT * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              tc::smem_desc(sb + TLay::kK + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + kColS, a, bd, kIdS, kk > 0);
+        }
+        tc::mma_commit(&mma_bar);
+      }
+      if (!(ok = wait_products(&mma_bar, phase))) break;
+      tc::tc_fence_after();
+      // ---- this row's P (float32, kept) into the P tile; G = w dout into the G tile
+      float p[kChunk];
+      {
+        uint32_t v[32];
+        tc::tmem_ld32(tl + kColS, v);
+        tc::tmem_ld_wait();
+  #pragma unroll
+        for (int x = 0; x < 32; ++x) p[x] = __uint_as_float(v[x]);
+        tc::tmem_ld32(tl + kColS + 32, v);
+        tc::tmem_ld_wait();
+  #pragma unroll
+        for (int x = 0; x < 32; ++x) p[32 + x] = __uint_as_float(v[x]);
+        float mx = -INFINITY;
+  #pragma unroll
+        for (int x = 0; x < kChunk; ++x) {
+          p[x] = x < nk ? p[x] * sc : -INFINITY;
+          mx = fmaxf(mx, p[x]);
+        }
+        float l = 0.f;
+  #pragma unroll
+        for (int x = 0; x < kChunk; ++x) {
+          p[x] = x < nk ? __expf(p[x] - mx) : 0.f;
+          l += p[x];
+        }
+        const float il = live ? 1.f / l : 0.f;
+  #pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u;
+          u.x = tc::pack_bf16x2(p[8 * c] * il, p[8 * c + 1] * il);
+          u.y = tc::pack_bf16x2(p[8 * c + 2] * il, p[8 * c + 3] * il);
+          u.z = tc::pack_bf16x2(p[8 * c + 4] * il, p[8 * c + 5] * il);
+          u.w = tc::pack_bf16x2(p[8 * c + 6] * il, p[8 * c + 7] * il);
+          *reinterpret_cast<uint4*>(smem + TLay::kP + tc::swz(row, c)) = u;
+        }
+  #pragma unroll
+        for (int x = 0; x < kChunk; ++x) p[x] *= il;
+        const uint4* dsrc = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(dout) + r * (kD * 2));
+  #pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          const uint4 d4 = live ? __ldg(dsrc + c) : make_uint4(0, 0, 0, 0);
+          uint4 u;
+          u.x = tc::pack_bf16x2(wj * bf16_lo(d4.x), wj * bf16_hi(d4.x));
+          u.y = tc::pack_bf16x2(wj * bf16_lo(d4.y), wj * bf16_hi(d4.y));
+          u.z = tc::pack_bf16x2(wj * bf16_lo(d4.z), wj * bf16_hi(d4.z));
+          u.w = tc::pack_bf16x2(wj * bf16_lo(d4.w), wj * bf16_hi(d4.w));
+          *reinterpret_cast<uint4*>(smem + TLay::kG + tile_at(kRowsT, row, c)) = u;
+        }
+      }
       tc::fence_proxy_async();
-    }
-    __syncthreads();
-    // ---- S = Q K^T
-    if (tid == 0) {
-      tc::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint64_t a =
-            tc::smem_desc(sb + TLay::kQ + (kk >> 2) * (kRowsT * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd =
-            tc::smem_desc(sb + TLay::kK + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
-        tc::mma_bf16(tmem + kColS, a, bd, kIdS, kk > 0);
-      }
-      tc::mma_commit(&mma_bar);
-    }
-    if (!(ok = wait_products(&mma_bar, phase))) break;
-    tc::tc_fence_after();
-    // ---- this row's P (float32, kept) into the P tile; G = w dout into the G tile
-    float p[kChunk];
-    {
-      uint32_t v[32];
-      tc::tmem_ld32(tl + kColS, v);
-      tc::tmem_ld_wait();
-#pragma unroll
-      for (int x = 0; x < 32; ++x) p[x] = __uint_as_float(v[x]);
-      tc::tmem_ld32(tl + kColS + 32, v);
-      tc::tmem_ld_wait();
-#pragma unroll
-      for (int x = 0; x < 32; ++x) p[32 + x] = __uint_as_float(v[x]);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < kChunk; ++x) {
-        p[x] = x < nk ? p[x] * sc : -INFINITY;
-        mx = fmaxf(mx, p[x]);
-      }
-      float l = 0.f;
-#pragma unroll
-      for (int x = 0; x < kChunk; ++x) {
-        p[x] = x < nk ? __expf(p[x] - mx) : 0.f;
-        l += p[x];
-      }
-      const float il = live ? 1.f / l : 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = tc::pack_bf16x2(p[8 * c] * il, p[8 * c + 1] * il);
-        u.y = tc::pack_bf16x2(p[8 * c + 2] * il, p[8 * c + 3] * il);
-        u.z = tc::pack_bf16x2(p[8 * c + 4] * il, p[8 * c + 5] * il);
-        u.w = tc::pack_bf16x2(p[8 * c + 6] * il, p[8 * c + 7] * il);
-        *reinterpret_cast<uint4*>(smem + TLay::kP + tc::swz(row, c)) = u;
-      }
-#pragma unroll
-      for (int x = 0; x < kChunk; ++x) p[x] *= il;
-      const uint4* dsrc = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint8_t*>(dout) + r * (kD * 2));
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        const uint4 d4 = live ? __ldg(dsrc + c) : make_uint4(0, 0, 0, 0);
-        uint4 u;
-        u.x = tc::pack_bf16x2(wj * bf16_lo(d4.x), wj * bf16_hi(d4.x));
-        u.y = tc::pack_bf16x2(wj * bf16_lo(d4.y), wj * bf16_hi(d4.y));
-        u.z = tc::pack_bf16x2(wj * bf16_lo(d4.z), wj * bf16_hi(d4.z));
-        u.w = tc::pack_bf16x2(wj * bf16_lo(d4.w), wj * bf16_hi(d4.w));
-        *reinterpret_cast<uint4*>(smem + TLay::kG + tile_at(kRowsT, row, c)) = u;
-      }
-    }
-    tc::fence_proxy_async();
-    tc::tc_fence_before();
-    __syncthreads();
-    // ---- O = P V (into the O columns) and dP = G V^T (into the S columns)
-    if (tid == 0) {
-      tc::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kChunk / 16; ++kk) {
-        const uint64_t a = tc::smem_desc(sb + TLay::kP + kk * 32, 16, 1024);
-        const uint64_t bd = tc::smem_desc(sb + TLay::kV + kk * 2048, kChunk * 128, 1024);
-        tc::mma_bf16(tmem + kColO, a, bd, kIdO, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint64_t a =
-            tc::smem_desc(sb + TLay::kG + (kk >> 2) * (kRowsT * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd =
-            tc::smem_desc(sb + TLay::kV + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
-        tc::mma_bf16(tmem + kColS, a, bd, kIdS, kk > 0);
-      }
-      tc::mma_commit(&mma_bar);
-    }
-    if (!(ok = wait_products(&mma_bar, phase))) break;
-    tc::tc_fence_after();
-    // ---- dw = dout . O; dS = P (dP - w dw) into the dS tile
-    {
-      const uint4* dsrc = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint8_t*>(dout) + r * (kD * 2));
-      float dwp = 0.f;
-      uint32_t v[32];
-#pragma unroll
-      for (int blk = 0; blk < kD / 32; ++blk) {
-        tc::tmem_ld32(tl + kColO + 32 * blk, v);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 d4 = live ? __ldg(dsrc + 4 * blk + c) : make_uint4(0, 0, 0, 0);
-          dwp = fmaf(bf16_lo(d4.x), __uint_as_float(v[8 * c + 0]), dwp);
-          dwp = fmaf(bf16_hi(d4.x), __uint_as_float(v[8 * c + 1]), dwp);
-          dwp = fmaf(bf16_lo(d4.y), __uint_as_float(v[8 * c + 2]), dwp);
-          dwp = fmaf(bf16_hi(d4.y), __uint_as_float(v[8 * c + 3]), dwp);
-          dwp = fmaf(bf16_lo(d4.z), __uint_as_float(v[8 * c + 4]), dwp);
-          dwp = fmaf(bf16_hi(d4.z), __uint_as_float(v[8 * c + 5]), dwp);
-          dwp = fmaf(bf16_lo(d4.w), __uint_as_float(v[8 * c + 6]), dwp);
-          dwp = fmaf(bf16_hi(d4.w), __uint_as_float(v[8 * c + 7]), dwp);
+      tc::tc_fence_before();
+      __syncthreads();
+      // ---- O = P V (into the O columns) and dP = G V^T (into the S columns)
+      if (tid == 0) {
+        tc::tc_fence_after();
+  #pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(sb + TLay::kP + kk * 32, 16, 1024);
+          const uint64_t bd = tc::smem_desc(sb + TLay::kV + kk * 2048, kChunk * 128, 1024);
+          tc::mma_bf16(tmem + kColO, a, bd, kIdO, kk > 0);
         }
-      }
-      const float go = wj * dwp;
-      sds[row] = live ? wj * (dwp - dl) : 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tc::tmem_ld32(tl + kColS + 32 * h, v);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          p[32 * h + x] = p[32 * h + x] * (__uint_as_float(v[x]) - go);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = tc::pack_bf16x2(p[8 * c], p[8 * c + 1]);
-        u.y = tc::pack_bf16x2(p[8 * c + 2], p[8 * c + 3]);
-        u.z = tc::pack_bf16x2(p[8 * c + 4], p[8 * c + 5]);
-        u.w = tc::pack_bf16x2(p[8 * c + 6], p[8 * c + 7]);
-        *reinterpret_cast<uint4*>(smem + TLay::kS + tc::swz(row, c)) = u;
-      }
-      // ds as column 0 of the next block (columns 1..15 zero): B of v = Q^T ds
-      const uint4 z = make_uint4(0, 0, 0, 0);
-      uint4 u0 = z;
-      u0.x = tc::pack_bf16x2(sds[row], 0.f);
-      *reinterpret_cast<uint4*>(smem + TLay::kS + kPB + tc::swz(row, 0)) = u0;
-      *reinterpret_cast<uint4*>(smem + TLay::kS + kPB + tc::swz(row, 1)) = z;
-    }
-    tc::fence_proxy_async();
-    tc::tc_fence_before();
-    __syncthreads();
-    // ---- dQ = dS K (into the O columns), dK^T = Q^T dS, dV^T = G^T P
-    if (tid == 0) {
-      tc::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kChunk / 16; ++kk) {
-        const uint64_t a = tc::smem_desc(sb + TLay::kS + kk * 32, 16, 1024);
-        const uint64_t bd = tc::smem_desc(sb + TLay::kK + kk * 2048, kChunk * 128, 1024);
-        tc::mma_bf16(tmem + kColO, a, bd, kIdO, kk > 0);
-      }
-      // [dK^T | v] = Q^T [dS | ds] (N = 80) and dV^T = G^T P, added to the run's sums
-#pragma unroll
-      for (int kk = 0; kk < kRowsT / 16; ++kk) {
-        const uint64_t a = tc::smem_desc(sb + TLay::kQ + kk * 2048, kRowsT * 128, 1024);
-        const uint64_t bd = tc::smem_desc(sb + TLay::kS + kk * 2048, kRowsT * 128, 1024);
-        tc::mma_bf16(tmem + kColDK, a, bd, kIdTV, (kk > 0 || !run_first) ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < kRowsT / 16; ++kk) {
-        const uint64_t a = tc::smem_desc(sb + TLay::kG + kk * 2048, kRowsT * 128, 1024);
-        const uint64_t bd = tc::smem_desc(sb + TLay::kP + kk * 2048, kRowsT * 128, 1024);
-        tc::mma_bf16(tmem + kColDV, a, bd, kIdT, (kk > 0 || !run_first) ? 1u : 0u);
-      }
-      tc::mma_commit(&mma_bar);
-    }
-    if (!(ok = wait_products(&mma_bar, phase))) break;
-    tc::tc_fence_after();
-    // ---- dq row += (dQ + ds lm'_j) / sqrt(d); this thread's element of dK and dV
-    {
-      uint32_t v[32];
-#pragma unroll
-      for (int blk = 0; blk < kD / 32; ++blk) {
-        tc::tmem_ld32(tl + kColO + 32 * blk, v);
-        tc::tmem_ld_wait();
-        if (live) {
-          const float dsr = sds[row];
-          float4* dst = reinterpret_cast<float4*>(dq + r * kD + 32 * blk);
-          const float* lmr = slm + 32 * blk;
-#pragma unroll
-          for (int x = 0; x < 8; ++x)
-            atomicAdd(dst + x,
-                      make_float4((__uint_as_float(v[4 * x]) + dsr * lmr[4 * x]) * sc,
-                                  (__uint_as_float(v[4 * x + 1]) + dsr * lmr[4 * x + 1]) * sc,
-                                  (__uint_as_float(v[4 * x + 2]) + dsr * lmr[4 * x + 2]) * sc,
-                                  (__uint_as_float(v[4 * x + 3]) + dsr * lmr[4 * x + 3]) * sc));
+  #pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t a =
+              tc::smem_desc(sb + TLay::kG + (kk >> 2) * (kRowsT * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              tc::smem_desc(sb + TLay::kV + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + kColS, a, bd, kIdS, kk > 0);
         }
+        tc::mma_commit(&mma_bar);
       }
-      if (run_last) {
-        const int e = tid;   // TMEM lane of dK^T and dV^T = head-dimension element
-        float* dk = dpages + page_offset(P, page, 0, g, 0) + e;
-        float* dv = dpages + page_offset(P, page, 1, g, 0) + e;
-#pragma unroll
+      if (!(ok = wait_products(&mma_bar, phase))) break;
+      tc::tc_fence_after();
+      // ---- w dw = G . O (G from its tile); ds = w (dw - delta); dS = P (dP - w dw)
+      {
+        float go = 0.f;
+        uint32_t v[32];
+  #pragma unroll
+        for (int blk = 0; blk < kD / 32; ++blk) {
+          tc::tmem_ld32(tl + kColO + 32 * blk, v);
+          tc::tmem_ld_wait();
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 g4 =
+                *reinterpret_cast<const uint4*>(smem + TLay::kG + tile_at(kRowsT, row, 4 * blk + c));
+            go = fmaf(bf16_lo(g4.x), __uint_as_float(v[8 * c + 0]), go);
+            go = fmaf(bf16_hi(g4.x), __uint_as_float(v[8 * c + 1]), go);
+            go = fmaf(bf16_lo(g4.y), __uint_as_float(v[8 * c + 2]), go);
+            go = fmaf(bf16_hi(g4.y), __uint_as_float(v[8 * c + 3]), go);
+            go = fmaf(bf16_lo(g4.z), __uint_as_float(v[8 * c + 4]), go);
+            go = fmaf(bf16_hi(g4.z), __uint_as_float(v[8 * c + 5]), go);
+            go = fmaf(bf16_lo(g4.w), __uint_as_float(v[8 * c + 6]), go);
+            go = fmaf(bf16_hi(g4.w), __uint_as_float(v[8 * c + 7]), go);
+          }
+        }
+        sds[row] = live ? go - wj * dl : 0.f;
+        srow[row] = live ? (int32_t)r : -1;
+  #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tc::tmem_ld32(tl + kColDK + 32 * h, v);
+          tc::tmem_ld32(tl + kColS + 32 * h, v);
           tc::tmem_ld_wait();
-#pragma unroll
+  #pragma unroll
           for (int x = 0; x < 32; ++x)
-            atomicAdd(dk + (32 * h + x) * kD, __uint_as_float(v[x]) * sc);
-          tc::tmem_ld32(tl + kColDV + 32 * h, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) atomicAdd(dv + (32 * h + x) * kD, __uint_as_float(v[x]));
+            p[32 * h + x] = p[32 * h + x] * (__uint_as_float(v[x]) - go);
         }
-        uint32_t v16[16];
-        tc::tmem_ld16(tl + kColV, v16);
-        tc::tmem_ld_wait();
-        atomicAdd(vchunk + (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * kD + e,
-                  __uint_as_float(v16[0]));
+  #pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u;
+          u.x = tc::pack_bf16x2(p[8 * c], p[8 * c + 1]);
+          u.y = tc::pack_bf16x2(p[8 * c + 2], p[8 * c + 3]);
+          u.z = tc::pack_bf16x2(p[8 * c + 4], p[8 * c + 5]);
+          u.w = tc::pack_bf16x2(p[8 * c + 6], p[8 * c + 7]);
+          *reinterpret_cast<uint4*>(smem + TLay::kS + tc::swz(row, c)) = u;
+        }
+        // ds as column 0 of the next block (columns 1..15 zero): B of v = Q^T ds
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        uint4 u0 = z;
+        u0.x = tc::pack_bf16x2(sds[row], 0.f);
+        *reinterpret_cast<uint4*>(smem + TLay::kS + kPB + tc::swz(row, 0)) = u0;
+        *reinterpret_cast<uint4*>(smem + TLay::kS + kPB + tc::swz(row, 1)) = z;
       }
+      tc::fence_proxy_async();
+      tc::tc_fence_before();
+      __syncthreads();
+      // ---- dQ = dS K (into the O columns), dK^T = Q^T dS, dV^T = G^T P
+      if (tid == 0) {
+        tc::tc_fence_after();
+  #pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(sb + TLay::kS + kk * 32, 16, 1024);
+          const uint64_t bd = tc::smem_desc(sb + TLay::kK + kk * 2048, kChunk * 128, 1024);
+          tc::mma_bf16(tmem + kColO, a, bd, kIdO, kk > 0);
+        }
+        // [dK^T | v] = Q^T [dS | ds] (N = 80) and dV^T = G^T P, added to the run's sums
+  #pragma unroll
+        for (int kk = 0; kk < kRowsT / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(sb + TLay::kQ + kk * 2048, kRowsT * 128, 1024);
+          const uint64_t bd = tc::smem_desc(sb + TLay::kS + kk * 2048, kRowsT * 128, 1024);
+          tc::mma_bf16(tmem + kColDK, a, bd, kIdTV, (kk > 0 || !run_first) ? 1u : 0u);
+        }
+  #pragma unroll
+        for (int kk = 0; kk < kRowsT / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(sb + TLay::kG + kk * 2048, kRowsT * 128, 1024);
+          const uint64_t bd = tc::smem_desc(sb + TLay::kP + kk * 2048, kRowsT * 128, 1024);
+          tc::mma_bf16(tmem + kColDV, a, bd, kIdT, (kk > 0 || !run_first) ? 1u : 0u);
+        }
+        tc::mma_commit(&mma_bar);
+      }
+      if (!(ok = wait_products(&mma_bar, phase))) break;
+      tc::tc_fence_after();
+      // ---- dq row += (dQ + ds lm'_j) / sqrt(d); this thread's element of dK and dV
+      {
+        // each warp stages its 32 rows, 32 columns at a time, and adds them row
+        // by row: 8 lanes cover one row's 128 bytes
+        uint32_t v[32];
+        const int lr = tid & 31;
+        float* stg = reinterpret_cast<float*>(smem + TLay::kStage) + warp * 32 * TLay::kStageLd;
+        const float dsr = sds[row];
+  #pragma unroll 1
+        for (int blk = 0; blk < kD / 32; ++blk) {
+          tc::tmem_ld32(tl + kColO + 32 * blk, v);
+          tc::tmem_ld_wait();
+          const float* lmr = slm + 32 * blk;
+  #pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(stg + lr * TLay::kStageLd + x) =
+                make_float4((__uint_as_float(v[x]) + dsr * lmr[x]) * sc,
+                            (__uint_as_float(v[x + 1]) + dsr * lmr[x + 1]) * sc,
+                            (__uint_as_float(v[x + 2]) + dsr * lmr[x + 2]) * sc,
+                            (__uint_as_float(v[x + 3]) + dsr * lmr[x + 3]) * sc);
+          __syncwarp();
+  #pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            const int rr = pass * 4 + (lr >> 3), cc = (lr & 7) * 4;
+            const int32_t gr = srow[warp * 32 + rr];
+            if (gr >= 0)
+              tc::red_add_f32x4(dq + (int64_t)gr * kD + 32 * blk + cc,
+                                *reinterpret_cast<const float4*>(stg + rr * TLay::kStageLd + cc));
+          }
+          __syncwarp();
+        }
+        if (run_last) {
+          const int e = tid;   // TMEM lane of dK^T and dV^T = head-dimension element
+          float* dk = dpages + page_offset(P, page, 0, g, 0) + e;
+          float* dv = dpages + page_offset(P, page, 1, g, 0) + e;
+  #pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tc::tmem_ld32(tl + kColDK + 32 * h, v);
+            tc::tmem_ld_wait();
+  #pragma unroll
+            for (int x = 0; x < 32; ++x)
+              tc::red_add_f32(dk + (32 * h + x) * kD, __uint_as_float(v[x]) * sc);
+            tc::tmem_ld32(tl + kColDV + 32 * h, v);
+            tc::tmem_ld_wait();
+  #pragma unroll
+            for (int x = 0; x < 32; ++x) tc::red_add_f32(dv + (32 * h + x) * kD, __uint_as_float(v[x]));
+          }
+          uint32_t v16[16];
+          tc::tmem_ld16(tl + kColV, v16);
+          tc::tmem_ld_wait();
+          tc::red_add_f32(vchunk + (((int64_t)b * P.max_chunks + j) * P.Hkv + g) * kD + e,
+                          __uint_as_float(v16[0]));
+        }
+      }
+      tc::tc_fence_before();
+      __syncthreads();   // shared and tensor memory are free for the next item
     }
-    tc::tc_fence_before();
-    __syncthreads();   // shared and tensor memory are free for the next item
   }
   if (!ok) {
     // a wait ran out: let the products in flight finish before the memory goes
@@ -571,7 +585,7 @@ cudaError_t launch_backward_tc(const Params& P, const int32_t* idx, const float*
     return e;
   const size_t vbytes = sizeof(float) * (size_t)P.B * P.max_chunks * P.Hkv * kD;
   if ((e = cudaMemsetAsync(ws.vchunk, 0, vbytes, s)) != cudaSuccess) return e;
-  const int64_t grid = ws.bk.max_tiles < n_sm ? ws.bk.max_tiles : n_sm;
+  const int64_t grid = ws.bk.n_keys < n_sm ? ws.bk.n_keys : n_sm;
   {
     HILS_PROFILE("backward.attention", s);
     attn_bwd_tc_kernel<<<(unsigned)(grid > 0 ? grid : 1), kThreadsT, smem, s>>>(

@@ -309,6 +309,17 @@ __device__ __forceinline__ void red_add_bf16x8(void* addr, uint4 v) {
                "r"(v.y), "r"(v.z), "r"(v.w));
 }
 
+// Adds four floats to 16 bytes of global memory in L2 (16-byte aligned); no
+// result is returned.  Not ordered against the thread's other accesses.
+__device__ __forceinline__ void red_add_f32x4(float* addr, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w));
+}
+// Adds one float to global memory in L2; no result is returned.
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v));
+}
+
 // ---- tcgen05 ---------------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -123,3 +123,73 @@ def test_score_and_topk_argument_checks(lib):
 def test_workspace_size_rejects_bad_op(lib):
     assert hils.workspace_size(cfg(), 9, 10, 10) == 0
     assert b"unknown op" in lib.hils_last_error()
+
+
+def test_prefill_backward_argument_checks(lib):
+    c = cfg(head_dim=128)
+    ws = hils.workspace_size(c, hils.OP_PREFILL_BACKWARD, 128, 8)
+    assert ws > 0
+
+    def call(**over):
+        a = dict(q=FAKE, q_len=128, q_pos0=0, A=FAKE, B=FAKE, cache=cache(), idx=FAKE, w=FAKE,
+                 out=FAKE, dout=FAKE, dq=FAKE, dpages=FAKE, dlm=FAKE, dA=FAKE, dB=FAKE, ws=FAKE,
+                 ws_bytes=ws)
+        a.update(over)
+        return status_of(hils.prefill_backward, c if "c" not in over else over.pop("c"),
+                         *[a[k] for k in ("q", "q_len", "q_pos0", "A", "B", "cache", "idx", "w",
+                                          "out", "dout", "dq", "dpages", "dlm", "dA", "dB", "ws",
+                                          "ws_bytes")], 0)
+
+    assert call(idx=None)[0] == 1
+    assert call(w=None)[0] == 1
+    st, msg = call(out=None)
+    assert st == 1 and "out" in msg
+    assert call(out=FAKE + 8)[0] == 1
+    assert call(dout=FAKE + 2)[0] == 1
+    st, msg = call(dq=FAKE + 4)
+    assert st == 1 and "dq" in msg
+    assert call(dpages=None)[0] == 1
+    assert call(dlm=None)[0] == 1
+    st, msg = call(dA=None)
+    assert st == 1 and "calib_rank" in msg
+    st, msg = call(ws_bytes=ws - 1)
+    assert st == 3 and "workspace" in msg
+    assert call(ws=FAKE + 16)[0] == 1
+    # the last query's chunk must be inside the block table
+    assert call(q_len=8 * 64 + 1, ws_bytes=1 << 40)[0] == 1
+
+
+def test_backward_workspace_depends_on_the_path(lib):
+    # bf16 at head_dim 128 keeps per-row and per-chunk sums; the CUDA-core
+    # path keeps one float per (row, slot) pair instead
+    tc = hils.workspace_size(cfg(head_dim=128), hils.OP_PREFILL_BACKWARD, 4096, 64)
+    simt = hils.workspace_size(cfg(head_dim=128, dtype=hils.HILS_F32), hils.OP_PREFILL_BACKWARD,
+                               4096, 64)
+    assert tc > 0 and simt > 0 and tc != simt
+    # both grow with the query block
+    assert hils.workspace_size(cfg(head_dim=128), hils.OP_PREFILL_BACKWARD, 8192, 64) > tc
+
+
+def test_context_parallel_argument_checks(lib):
+    c = cfg()
+    ws = hils.workspace_size(c, hils.OP_DECODE, 1, 8)
+    cand = hils.decode_cp_candidates
+    assert status_of(cand, c, FAKE, None, None, FAKE, FAKE, cache(seq_lens=None), 0, FAKE, FAKE,
+                     FAKE, ws, 0)[0] == 1
+    assert status_of(cand, c, FAKE, None, None, FAKE, FAKE, cache(), -1, FAKE, FAKE, FAKE, ws,
+                     0)[0] == 1
+    assert status_of(cand, c, FAKE, None, None, FAKE, FAKE, cache(), 0, None, FAKE, FAKE, ws,
+                     0)[0] == 1
+    assert status_of(cand, c, FAKE, FAKE, None, FAKE, FAKE, cache(), 0, FAKE, FAKE, FAKE, ws,
+                     0)[0] == 1
+    st, msg = status_of(cand, c, FAKE, None, None, FAKE, FAKE, cache(), 0, FAKE, FAKE, FAKE,
+                        ws - 1, 0)
+    assert st == 3 and "workspace" in msg
+    assert status_of(hils.decode_cp_select, c, 0, FAKE, FAKE, FAKE, True, FAKE, FAKE, 0)[0] == 1
+    assert status_of(hils.decode_cp_select, c, 2, FAKE, FAKE, None, True, FAKE, FAKE, 0)[0] == 1
+    assert status_of(hils.decode_cp_attend, c, FAKE, None, None, cache(), 0, FAKE, FAKE, None,
+                     0)[0] == 1
+    assert status_of(hils.decode_cp_attend, c, FAKE, None, None, cache(), -3, FAKE, FAKE, FAKE,
+                     0)[0] == 1
+    assert status_of(hils.decode_cp_finish, c, FAKE, FAKE, None, True, 0)[0] == 1
+    assert status_of(hils.decode_cp_finish, c, None, FAKE, FAKE, False, 0)[0] == 1

@@ -148,11 +148,16 @@ int hils_prefill(const hils_config* cfg, const void* q, int64_t q_len, int64_t q
  * additions is not fixed, so results may differ in the last bits from run
  * to run.  Arithmetic is float32, except that for bf16 storage at head_dim
  * 128 the per-chunk attention products run on the tensor cores with bf16
- * operands (the probabilities, G = w dout and dS rounded to bf16, as the
+ * operands (the probabilities, G = w dout, dS and ds rounded to bf16, as the
  * forward rounds the probabilities) and float32 accumulation.
  * ws         at least hils_workspace_size(cfg, HILS_OP_PREFILL_BACKWARD, q_len,
  *            max_chunks) bytes, 256-byte aligned; its contents need not be
- *            initialised. */
+ *            initialised.
+ * Errors: HILS_ERR_INVALID_ARG (a missing or misaligned pointer, a query
+ * position beyond the block table), HILS_ERR_UNSUPPORTED (configuration),
+ * HILS_ERR_WORKSPACE (ws too small); nothing is queued when a check fails.
+ * A block-table entry or selected chunk out of range is reported by
+ * hils_device_status(). */
 int hils_prefill_backward(const hils_config* cfg, const void* q, int64_t q_len, int64_t q_pos0,
                           const float* A, const float* B, const hils_kv_cache* cache,
                           const int32_t* idx, const float* w, const void* out,

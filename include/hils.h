@@ -1,6 +1,7 @@
 /*
- * hils.h -- C ABI of the HiLS (Hierarchical Landmark Sparse) attention forward
- * on NVIDIA B200 (sm_100a).
+ * hils.h -- C ABI of HiLS (Hierarchical Landmark Sparse) attention on NVIDIA
+ * B200 (sm_100a): the forward (prefill and decode), its backward with the
+ * chunk selection held fixed, and the decode step split over several GPUs.
  *
  * The method ("Hierarchical Sparse Attention Done Right"; ai-feeds.com digest,
  * section 方法; oopus.info review, section 二; chatpaper abstract):
@@ -14,6 +15,8 @@
  *   a6  fused output out = sum_j w_j O_j                            (review, 融合; abstract)
  *   a7  chunk-granular paged KV access: one page = one chunk        (digest, 关键模块 item 3)
  *   a8  decode step: append k_t, v_t, then row t of the prefill     (digest, 局限: per-step scan)
+ *   backward of a1..a6 with the selection fixed                      (digest, 关键模块 items 1, 3;
+ *                                                                     输出与训练)
  *
  * Conventions shared by every entry point:
  *   - All tensor arguments are caller-owned DEVICE pointers, 16-byte aligned,

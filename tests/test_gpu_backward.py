@@ -108,6 +108,8 @@ CASES = {
                                 calib_rank=16, seq_len=1000, q_pos0=300, dtype=F32),
     "bf16_d128_gqa": dict(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, top_k=8,
                           calib_rank=32, seq_len=1200, dtype=BF16),
+    "bf16_d128_b2_window": dict(batch=2, n_q_heads=4, n_kv_heads=1, head_dim=128, top_k=8,
+                                calib_rank=16, seq_len=900, q_pos0=320, dtype=BF16),
     "bf16_d64_k1": dict(batch=2, n_q_heads=2, n_kv_heads=1, head_dim=64, top_k=1, calib_rank=4,
                         seq_len=300, dtype=BF16),
     "bf16_d64_rank64_k32": dict(batch=1, n_q_heads=2, n_kv_heads=2, head_dim=64, top_k=32,

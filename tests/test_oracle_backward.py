@@ -163,3 +163,30 @@ def test_planted_mistake_is_caught(monkeypatch, fn, patch):
     t = _tiny(seed=5, k=3)
     errs = _fd_errors(t)
     assert any(err > 1e-7 + 1e-6 * scale for err, scale in errs.values()), errs
+
+
+def test_two_single_token_chunks_closed_form():
+    """Chunks of one token, d = 1, no calibration, two positions, k = 2.
+    Row 0 sees only its own chunk: out_0 = v_0, so dv_0 gets dout_0 and
+    nothing else moves (a softmax over one key has no gradient).  Row 1
+    fuses chunk 1 (its own) and chunk 0 with w = softmax(q_1 [lm_1, lm_0]):
+    out_1 = w_1 v_1 + w_0 v_0.  By hand:
+        dv_1 = w_1 dout_1,  dv_0 = dout_0 + w_0 dout_1,  dK = 0,
+        ds_1 = -ds_0 = w_0 w_1 dout_1 (v_1 - v_0),
+        dq_1 = ds_1 (lm_1 - lm_0),  dlm_1 = ds_1 q_1,  dlm_0 = -ds_1 q_1."""
+    q = np.array([0.3, 0.5]).reshape(1, 2, 1, 1)
+    K = np.array([0.7, -0.2]).reshape(1, 2, 1, 1)
+    V = np.array([1.5, -0.5]).reshape(1, 2, 1, 1)
+    lm = np.array([1.0, -1.0]).reshape(1, 2, 1, 1)
+    A, B = np.zeros((1, 0)), np.zeros((0, 1))
+    idx = np.array([[0, -1], [1, 0]]).reshape(1, 2, 1, 2)
+    dout = np.array([0.25, 2.0]).reshape(1, 2, 1, 1)
+    g = ob.backward(q, 0, A, B, K, V, lm, idx, dout, 1)
+    e1, e0 = np.exp(0.5 * -1.0), np.exp(0.5 * 1.0)
+    w1, w0 = e1 / (e1 + e0), e0 / (e1 + e0)
+    ds1 = w0 * w1 * 2.0 * (-0.5 - 1.5)
+    np.testing.assert_allclose(g["dV"].reshape(2), [0.25 + w0 * 2.0, w1 * 2.0], rtol=1e-14)
+    np.testing.assert_allclose(g["dK"].reshape(2), [0.0, 0.0], atol=1e-15)
+    np.testing.assert_allclose(g["dq"].reshape(2), [0.0, ds1 * (-1.0 - 1.0)], atol=1e-15)
+    np.testing.assert_allclose(g["dlm"].reshape(2), [-ds1 * 0.5, ds1 * 0.5], atol=1e-15)
+    np.testing.assert_allclose(g["ds"].reshape(2, 2), [[0.0, 0.0], [ds1, -ds1]], atol=1e-15)
